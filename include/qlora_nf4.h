@@ -1,0 +1,174 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so: a LoRA-adapted linear layer over a frozen NF4
+ * (4-bit NormalFloat) base weight, forward and hand-derived backward, for sm_100a (B200).
+ *
+ * The operation ("Unsloth vs QLoRA vs Liger-Kernel", section 1, LoRA forward formula; FAQ
+ * "What is the difference between LoRA and QLoRA?", NF4 base weights):
+ *
+ *     XA = X A^T                                   [M, r]
+ *     h  = X deq(W0)^T + s XA B^T,   s = alpha / r [M, N]
+ *
+ * and its exact gradients for dY = dL/dh with W0 frozen ("Unsloth vs QLoRA vs
+ * Liger-Kernel", section 2, hand-derived backward; "FTDD-03" teaching script, [SLIDE 3]):
+ *
+ *     dYB = dY B,  dX = dY deq(W0) + s dYB A,  dB = s dY^T XA,  dA = s dYB^T X.
+ *
+ * Shapes and layouts (all row-major, C order):
+ *   X  [M, K] bf16   tokens x in-features          W0 [N, K] (nn.Linear weight [out, in])
+ *   A  [r, K] bf16   LoRA down-projection          B  [N, r] bf16  LoRA up-projection
+ *   h, dY [M, N] bf16                              dX [M, K] bf16
+ *   dA [r, K] fp32, dB [N, r] fp32 (overwritten, not accumulated)
+ *
+ * NF4 storage (the readings the pages leave open are fixed here):
+ *   q       [N, K/2] uint8  two 4-bit codes per byte, element 2j of a row in the HIGH nibble
+ *   absmax  [N, K/64] fp32  per 64-element block of a row (block index n*K/64 + kb)
+ *   double-quantised variant: absmax_q8 [N*K/64] uint8 and absmax_scale [ceil(N*K/64/256)]
+ *   fp32, effective absmax = fp32(q8 * scale[block/256]).
+ *   Codebook: the 16 NormalFloat levels (asymmetric N(0,1) quantiles with an exact zero,
+ *   normalised to [-1, 1]) in fp32; code c dequantises to bf16(fp32(level[c] * absmax)).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device memory are caller-owned device allocations on the current
+ *     device; the library allocates nothing and keeps no state between calls.
+ *   - Device pointers must be 16-byte aligned (QLORA_ERR_ALIGN otherwise).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the call
+ *     returns without synchronising.  Launch failures are returned as QLORA_ERR_CUDA; a fault
+ *     during execution surfaces at the caller's next synchronisation.
+ *   - Shape errors are reported before any work is enqueued (QLORA_ERR_SHAPE).
+ *   - Kernels bound every wait on another warp's progress; a wait that runs out sets the
+ *     device error word read by qlora_device_error() and the kernel returns early.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = 1,      /* a required pointer is NULL */
+  QLORA_ERR_SHAPE = 2,     /* M < 1, N or K not a multiple of 64, r not in {8,16,...,128} */
+  QLORA_ERR_ALIGN = 3,     /* a device pointer is not 16-byte aligned */
+  QLORA_ERR_ARCH = 4,      /* current device is not compute capability 10.0 (sm_100a) */
+  QLORA_ERR_WORKSPACE = 5, /* workspace NULL or smaller than qlora_workspace_bytes() */
+  QLORA_ERR_CUDA = 6,      /* a CUDA runtime/driver call or kernel launch failed */
+  QLORA_ERR_TIMEOUT = 7    /* a kernel's bounded wait ran out (see qlora_device_error) */
+} qlora_status;
+
+typedef void* qlora_stream_t; /* a cudaStream_t */
+
+/* A packed NF4 weight: caller-owned device memory.  With double_quant == 0, `absmax` is
+ * used and absmax_q8 / absmax_scale are ignored; with double_quant != 0 the reverse. */
+typedef struct {
+  const uint8_t* q;            /* [N, K/2] */
+  const float* absmax;         /* [N*K/64] or NULL when double_quant */
+  const uint8_t* absmax_q8;    /* [N*K/64] when double_quant */
+  const float* absmax_scale;   /* [ceil(N*K/64/256)] when double_quant */
+  int N;
+  int K;
+  int double_quant;
+} qlora_nf4_weight;
+
+/* Human-readable name of a status code (static string, never NULL). */
+QLORA_API const char* qlora_status_str(qlora_status s);
+
+/* Host-only: the fp32 NF4 codebook (16 ascending levels, out[0] = -1, out[7] = 0,
+ * out[15] = +1), derived at library load from the NormalFloat construction.  Needs no GPU. */
+QLORA_API qlora_status qlora_nf4_codebook(float out[16]);
+
+/* NF4 quantise + pack ("Unsloth vs QLoRA vs Liger-Kernel", FAQ on LoRA vs QLoRA: base
+ * weights in 4-bit NormalFloat; "Speed up fine-tuning 2x", internals item 1).
+ *   W       [N, K] bf16 device, read only.
+ *   q       [N, K/2] uint8 device, written.
+ *   absmax  [N*K/64] fp32 device, written: first-level absmax (also when double_quant).
+ *   absmax_q8 [N*K/64] uint8 and absmax_scale [ceil(N*K/64/256)] fp32 device, written only
+ *           when double_quant != 0 (may be NULL otherwise).
+ * Codes are chosen with the effective absmax (the double-quantised one when requested):
+ * x = fp32(w / absmax), code = number of codebook midpoints strictly below x; a block
+ * whose effective absmax is 0 gets code 7 (the exact zero) everywhere. */
+QLORA_API qlora_status qlora_nf4_pack(const void* W, int N, int K, int double_quant, uint8_t* q,
+                            float* absmax, uint8_t* absmax_q8, float* absmax_scale,
+                            qlora_stream_t stream);
+
+/* Dequantise a packed weight to bf16 Wd [N, K] device (diagnostic/test export; the linear
+ * entry points never materialise it).  Uses the same device routine as the GEMM mainloop. */
+QLORA_API qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, qlora_stream_t stream);
+
+/* Scratch bytes the linear entry points need for (M, N, K, r): the scaled rank-r
+ * activations and the fixed-order split partials of the rank-r reductions. */
+QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
+
+/* Forward.  X [M, K], A [r, K], B [N, r] bf16 device (read); H [M, N] bf16 device (written);
+ * XA_saved [M, r] bf16 device (written: X A^T rounded to bf16, kept for the backward).
+ * ws: device scratch of at least qlora_workspace_bytes(M, N, K, r) bytes.
+ * alpha: LoRA alpha; s = alpha / r.  r must be a multiple of 8 in [8, 128]. */
+QLORA_API qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
+                              const void* B, int M, int r, float alpha, void* H, void* XA_saved,
+                              void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Backward.  dY [M, N], X [M, K], A, B, XA_saved [M, r] bf16 device (read).
+ * dX [M, K] bf16 device (written; may be NULL to skip the dX GEMM).
+ * dA [r, K] and dB [N, r] fp32 device (overwritten).  ws as for the forward. */
+QLORA_API qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
+                              const void* A, const void* B, const void* XA_saved, int M, int r,
+                              float alpha, void* dX, float* dA, float* dB, void* ws,
+                              size_t ws_bytes, qlora_stream_t stream);
+
+/* SwiGLU glue for the MLP workload: a = g * sigmoid(g) * u (elementwise, n elements, bf16
+ * device), and its exact backward dg = da*u*sig(g)*(1 + g*(1 - sig(g))), du = da*g*sig(g).
+ * Computed in fp32, rounded to bf16.  ("Unsloth vs QLoRA vs Liger-Kernel", section 2: the
+ * SwiGLU MLP is among the hand-differentiated ops.) */
+QLORA_API qlora_status qlora_swiglu_fwd(const void* g, const void* u, void* a, int64_t n,
+                              qlora_stream_t stream);
+QLORA_API qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void* da, void* dg, void* du,
+                              int64_t n, qlora_stream_t stream);
+
+/* ---- The stages the two linear entry points are composed of (same validation rules). ---- */
+
+/* Rank-r down-projection: out = in . Wl^T with in [M, C] bf16 and Wl given either as
+ * w [r, C] (w_is_r_by_c = 1, the LoRA A) or as w [C, r] (w_is_r_by_c = 0, the LoRA B).
+ * Writes bf16(out) to `saved` [M, r] (may be NULL) and bf16(scale * out) to `scaled` [M, r].
+ * ws: device scratch of at least qlora_workspace_bytes(M, C, C, r) bytes. */
+QLORA_API qlora_status qlora_lora_down(const void* in, int M, int C, const void* w,
+                                       int w_is_r_by_c, int r, float scale, void* saved,
+                                       void* scaled, void* ws, size_t ws_bytes,
+                                       qlora_stream_t stream);
+
+/* The dequant GEMM with the fused rank-r extension (no workspace):
+ *   transpose_w = 0: out[M, N] = act[M, K] . deq(W0)^T + ext_act[M, r] . ext_w^T, ext_w = B [N, r]
+ *   transpose_w = 1: out[M, K] = act[M, N] . deq(W0)   + ext_act[M, r] . ext_w,   ext_w = A [r, K]
+ * act, ext_w, ext_act bf16 device (read); out bf16 device (written).  The scale s is expected
+ * to be folded into ext_act already (qlora_lora_down's `scaled` output). */
+QLORA_API qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
+                                      const void* ext_w, const void* ext_act, int M, int r,
+                                      void* out, qlora_stream_t stream);
+
+/* Rank-r weight gradient: G[c, j] = scale * sum_m big[m, c] small[m, j] with big [M, C] and
+ * small [M, r] bf16 device; written fp32 as out [C, r] (out_r_by_c = 0, e.g. dB) or
+ * out [r, C] (out_r_by_c = 1, e.g. dA).  ws: at least qlora_workspace_bytes(M, C, C, r). */
+QLORA_API qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, int r,
+                                       float scale, float* out, int out_r_by_c, void* ws,
+                                       size_t ws_bytes, qlora_stream_t stream);
+
+/* Number of kernels this library has launched in this process so far (all devices). */
+QLORA_API uint64_t qlora_launch_counter(void);
+
+/* Synchronising: returns the device error word of the current device (0 = none; otherwise
+ * a code naming the wait that ran out) and clears it. */
+QLORA_API qlora_status qlora_device_error(int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

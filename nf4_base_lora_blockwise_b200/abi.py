@@ -1,0 +1,175 @@
+"""ctypes binding of libqlora_nf4.so -- argument marshalling only.
+
+Every function here mirrors one entry point of ``include/qlora_nf4.h`` with the same name and
+takes raw integers (device addresses, sizes, a cudaStream_t handle).  Nothing is computed in
+Python.  The library is loaded on first use; if it is missing the call raises -- there is no
+fallback path.
+"""
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
+
+# Exported entry points of include/qlora_nf4.h (kept in sync by tests/test_abi.py).
+EXPORTS = (
+    "qlora_status_str",
+    "qlora_nf4_codebook",
+    "qlora_nf4_pack",
+    "qlora_nf4_dequant",
+    "qlora_workspace_bytes",
+    "qlora_linear_fwd",
+    "qlora_linear_bwd",
+    "qlora_swiglu_fwd",
+    "qlora_swiglu_bwd",
+    "qlora_lora_down",
+    "qlora_nf4_gemm",
+    "qlora_lora_grad",
+    "qlora_launch_counter",
+    "qlora_device_error",
+)
+
+STATUS = {
+    0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGN",
+    4: "QLORA_ERR_ARCH", 5: "QLORA_ERR_WORKSPACE", 6: "QLORA_ERR_CUDA", 7: "QLORA_ERR_TIMEOUT",
+}
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({_lib().qlora_status_str(code).decode()})")
+
+
+class Nf4Weight(ctypes.Structure):
+    """Mirror of ``qlora_nf4_weight``."""
+    _fields_ = [
+        ("q", ctypes.c_void_p),
+        ("absmax", ctypes.c_void_p),
+        ("absmax_q8", ctypes.c_void_p),
+        ("absmax_scale", ctypes.c_void_p),
+        ("N", ctypes.c_int),
+        ("K", ctypes.c_int),
+        ("double_quant", ctypes.c_int),
+    ]
+
+
+_LIB = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+_I64 = ctypes.c_int64
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m nf4_base_lora_blockwise_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "qlora_status_str": (ctypes.c_char_p, [_I]),
+            "qlora_nf4_codebook": (_I, [ctypes.POINTER(ctypes.c_float)]),
+            "qlora_nf4_pack": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP]),
+            "qlora_nf4_dequant": (_I, [ctypes.POINTER(Nf4Weight), _VP, _VP]),
+            "qlora_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+            "qlora_linear_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _I, _I, _F, _VP,
+                                      _VP, _VP, _SZ, _VP]),
+            "qlora_linear_bwd": (_I, [_VP, _VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _VP, _I, _I,
+                                      _F, _VP, _VP, _VP, _VP, _SZ, _VP]),
+            "qlora_swiglu_fwd": (_I, [_VP, _VP, _VP, _I64, _VP]),
+            "qlora_swiglu_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _VP]),
+            "qlora_lora_down": (_I, [_VP, _I, _I, _VP, _I, _I, _F, _VP, _VP, _VP, _SZ, _VP]),
+            "qlora_nf4_gemm": (_I, [_VP, ctypes.POINTER(Nf4Weight), _I, _VP, _VP, _I, _I, _VP,
+                                    _VP]),
+            "qlora_lora_grad": (_I, [_VP, _I, _I, _VP, _I, _F, _VP, _I, _VP, _SZ, _VP]),
+            "qlora_launch_counter": (ctypes.c_uint64, []),
+            "qlora_device_error": (_I, [ctypes.POINTER(ctypes.c_int)]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _check(fn, code):
+    if code != 0:
+        raise QLoraError(fn, code)
+
+
+def loaded_path():
+    """Path of the loaded shared library (loads it)."""
+    _lib()
+    return LIB_PATH
+
+
+def qlora_nf4_codebook():
+    buf = (ctypes.c_float * 16)()
+    _check("qlora_nf4_codebook", _lib().qlora_nf4_codebook(buf))
+    return [buf[i] for i in range(16)]
+
+
+def qlora_nf4_pack(W, N, K, double_quant, q, absmax, absmax_q8, absmax_scale, stream):
+    _check("qlora_nf4_pack", _lib().qlora_nf4_pack(W, N, K, int(double_quant), q, absmax,
+                                                   absmax_q8, absmax_scale, stream))
+
+
+def qlora_nf4_dequant(weight, Wd, stream):
+    _check("qlora_nf4_dequant", _lib().qlora_nf4_dequant(ctypes.byref(weight), Wd, stream))
+
+
+def qlora_workspace_bytes(M, N, K, r):
+    return int(_lib().qlora_workspace_bytes(M, N, K, r))
+
+
+def qlora_linear_fwd(X, weight, A, B, M, r, alpha, H, XA_saved, ws, ws_bytes, stream):
+    _check("qlora_linear_fwd", _lib().qlora_linear_fwd(X, ctypes.byref(weight), A, B, M, r,
+                                                       float(alpha), H, XA_saved, ws, ws_bytes,
+                                                       stream))
+
+
+def qlora_linear_bwd(dY, X, weight, A, B, XA_saved, M, r, alpha, dX, dA, dB, ws, ws_bytes,
+                     stream):
+    _check("qlora_linear_bwd", _lib().qlora_linear_bwd(dY, X, ctypes.byref(weight), A, B,
+                                                       XA_saved, M, r, float(alpha), dX, dA, dB,
+                                                       ws, ws_bytes, stream))
+
+
+def qlora_swiglu_fwd(g, u, a, n, stream):
+    _check("qlora_swiglu_fwd", _lib().qlora_swiglu_fwd(g, u, a, n, stream))
+
+
+def qlora_swiglu_bwd(g, u, da, dg, du, n, stream):
+    _check("qlora_swiglu_bwd", _lib().qlora_swiglu_bwd(g, u, da, dg, du, n, stream))
+
+
+def qlora_lora_down(inp, M, C, w, w_is_r_by_c, r, scale, saved, scaled, ws, ws_bytes, stream):
+    _check("qlora_lora_down", _lib().qlora_lora_down(inp, M, C, w, int(w_is_r_by_c), r,
+                                                     float(scale), saved, scaled, ws, ws_bytes,
+                                                     stream))
+
+
+def qlora_nf4_gemm(act, weight, transpose_w, ext_w, ext_act, M, r, out, stream):
+    _check("qlora_nf4_gemm", _lib().qlora_nf4_gemm(act, ctypes.byref(weight), int(transpose_w),
+                                                   ext_w, ext_act, M, r, out, stream))
+
+
+def qlora_lora_grad(big, M, C, small, r, scale, out, out_r_by_c, ws, ws_bytes, stream):
+    _check("qlora_lora_grad", _lib().qlora_lora_grad(big, M, C, small, r, float(scale), out,
+                                                     int(out_r_by_c), ws, ws_bytes, stream))
+
+
+def qlora_launch_counter():
+    return int(_lib().qlora_launch_counter())
+
+
+def qlora_device_error():
+    code = ctypes.c_int(0)
+    st = _lib().qlora_device_error(ctypes.byref(code))
+    if st not in (0, 7):
+        _check("qlora_device_error", st)
+    return code.value

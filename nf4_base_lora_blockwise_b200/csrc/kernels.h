@@ -1,0 +1,90 @@
+// kernels.h -- internal launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "nf4_dequant.cuh"
+
+namespace qlora {
+
+// ------------------------------ NF4 pack / dequant -----------------------------------------
+cudaError_t launch_nf4_pack(const __nv_bfloat16* W, int N, int K, int dq, uint8_t* q,
+                            float* absmax, uint8_t* absmax_q8, float* absmax_scale,
+                            const Codebook& cb, cudaStream_t stream);
+cudaError_t launch_nf4_dequant(const uint8_t* q, const float* absmax, const uint8_t* q8,
+                               const float* scale, int dq, int N, int K, __nv_bfloat16* out,
+                               const Codebook& cb, cudaStream_t stream);
+
+// ------------------------------ dequant GEMM (tcgen05) -------------------------------------
+// out[M, rows_w] = act[M, red] . deq(W)^T-or-not + s_small[M, r] . ext^T, where the weight
+// operand is dequantised in the mainloop.  kTransW = false: forward (rows_w = N, red = K);
+// kTransW = true: dX (rows_w = K, red = N).
+struct GemmArgs {
+  int M;
+  int rows_w;
+  int kt;          // reduction steps of 64
+  int n_ext;       // LoRA extension chunks (64 wide along r)
+  int r_pad16;     // r rounded up to a multiple of 16
+  int bt;          // token tile = MMA N
+  int stages;
+  int kblocks;     // K / 64 = absmax blocks per row of W0
+  int N;           // rows of W0
+  int dq;
+  const float* absmax;
+  const uint8_t* absmax_q8;
+  const float* absmax_scale;
+  __nv_bfloat16* out;
+  int* err;  // device error word
+  Codebook cb;
+};
+
+struct GemmMaps {
+  CUtensorMap act;      // [M, red] bf16, box {64, bt}, 128B swizzle
+  CUtensorMap q;        // [N, K/2] u8
+  CUtensorMap ext_w;    // B_lora [N, r] (fwd) or A_lora [r, K] (dX), bf16
+  CUtensorMap ext_act;  // scaled rank-r activation [M, r] bf16, box {64, bt}
+};
+
+int gemm_pick_bt(int M);
+int gemm_pick_stages(int bt);
+size_t gemm_smem_bytes(int bt, int stages);
+cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, const GemmArgs& args,
+                              cudaStream_t stream);
+
+// ------------------------------ rank-r skinny products (mma.sync) --------------------------
+// out[m, j] = sum_c in[m, c] * Wl(j, c); Wl(j, c) = w[j * C + c] (w_is_rc = true, i.e. A [r, C])
+// or w[c * r + j] (w_is_rc = false, i.e. B [C, r]).  Writes bf16 RN(v) to `saved` (if not
+// null) and bf16 RN(scale * v) to `scaled`.  `partial` is fp32 scratch [split, M, r].
+struct DownPlan {
+  int split;
+  size_t partial_floats;
+};
+DownPlan lora_down_plan(int M, int C, int r);
+cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_bfloat16* w,
+                             bool w_is_rc, int r, float scale, __nv_bfloat16* saved,
+                             __nv_bfloat16* scaled, float* partial, const DownPlan& plan,
+                             cudaStream_t stream);
+
+// G[c, j] = scale * sum_m big[m, c] * small[m, j]; written as out[c * r + j] (out_cr) or
+// out[j * C + c].  `partial` is fp32 scratch [split, C, r].
+struct GradPlan {
+  int split;
+  size_t partial_floats;
+};
+GradPlan lora_grad_plan(int M, int C, int r);
+cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_bfloat16* small,
+                             int r, float scale, float* out, bool out_cr, float* partial,
+                             const GradPlan& plan, cudaStream_t stream);
+
+// ------------------------------ SwiGLU ------------------------------------------------------
+cudaError_t launch_swiglu_fwd(const __nv_bfloat16* g, const __nv_bfloat16* u, __nv_bfloat16* a,
+                              int64_t n, cudaStream_t stream);
+cudaError_t launch_swiglu_bwd(const __nv_bfloat16* g, const __nv_bfloat16* u,
+                              const __nv_bfloat16* da, __nv_bfloat16* dg, __nv_bfloat16* du,
+                              int64_t n, cudaStream_t stream);
+
+}  // namespace qlora

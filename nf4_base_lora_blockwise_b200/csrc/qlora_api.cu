@@ -1,0 +1,516 @@
+// qlora_api.cu -- the C ABI of libqlora_nf4.so (declared in include/qlora_nf4.h): argument
+// validation, the NF4 codebook, TMA descriptor encoding, workspace carving and the launch
+// sequence of the forward and backward passes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qlora_nf4.h"
+#include "kernels.h"
+
+namespace qlora {
+
+__device__ int g_qlora_error_word = 0;
+
+namespace {
+
+// ---------------------------------------------------------------------------------------------
+// NF4 codebook, derived here independently of any table: quantiles of N(0, 1) at evenly spaced
+// probabilities between 1/2 and an offset p* close to 1 -- 8 positive levels, 7 negative ones
+// and an exact zero -- divided by the largest one so the set spans [-1, 1].
+// p* = 1 - (1/32 + 1/30) / 2.  The inverse normal CDF is found by bisection on erfc.
+// ("Unsloth vs QLoRA vs Liger-Kernel", FAQ "What is the difference between LoRA and QLoRA?":
+// base weights in 4-bit NormalFloat.)
+// ---------------------------------------------------------------------------------------------
+double normal_cdf(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+double normal_quantile(double p) {
+  double lo = -12.0, hi = 12.0;
+  for (int i = 0; i < 2000; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid <= lo || mid >= hi) break;
+    if (normal_cdf(mid) < p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+Codebook make_codebook() {
+  const double pstar = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
+  double lv[16];
+  int n = 0;
+  for (int j = 0; j < 7; ++j) lv[n++] = -normal_quantile(pstar + (0.5 - pstar) * j / 7.0);
+  lv[n++] = 0.0;
+  for (int j = 0; j < 8; ++j) lv[n++] = normal_quantile(pstar + (0.5 - pstar) * j / 8.0);
+  std::sort(lv, lv + 16);
+  double mx = 0.0;
+  for (double v : lv) mx = std::max(mx, std::fabs(v));
+  Codebook cb;
+  for (int i = 0; i < 16; ++i) cb.level[i] = static_cast<float>(lv[i] / mx);
+  for (int i = 0; i < 15; ++i) cb.mid[i] = (cb.level[i] + cb.level[i + 1]) * 0.5f;
+  return cb;
+}
+
+const Codebook& codebook() {
+  static const Codebook cb = make_codebook();
+  return cb;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Device checks and the per-device error word.
+// ---------------------------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 wrong arch
+int* g_err_ptr[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+qlora_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_arch_ok[*dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    g_arch_ok[*dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_arch_ok[*dev] == 1 ? QLORA_OK : QLORA_ERR_ARCH;
+}
+
+qlora_status error_word_ptr(int dev, int** p) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_qlora_error_word) != cudaSuccess) return QLORA_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<int*>(a);
+  }
+  *p = g_err_ptr[dev];
+  return QLORA_OK;
+}
+
+qlora_status encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f)
+      return QLORA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  *fn = g_encode;
+  return QLORA_OK;
+}
+
+// 2-D row-major tensor [outer, inner] of `dtype`, row pitch `pitch_bytes`, box {bi, bo}.
+qlora_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                       uint64_t inner, uint64_t outer, uint64_t pitch_bytes, uint32_t bi,
+                       uint32_t bo, CUtensorMapSwizzle swz) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn;
+  qlora_status st = encoder(&fn);
+  if (st != QLORA_OK) return st;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {bi, bo};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qlora_status check_weight(const qlora_nf4_weight* W) {
+  if (!W || !W->q) return QLORA_ERR_NULL;
+  if (W->double_quant) {
+    if (!W->absmax_q8 || !W->absmax_scale) return QLORA_ERR_NULL;
+  } else if (!W->absmax) {
+    return QLORA_ERR_NULL;
+  }
+  if (W->N < 64 || W->K < 64 || (W->N % 64) || (W->K % 64)) return QLORA_ERR_SHAPE;
+  if (!aligned16(W->q) || (W->absmax && !aligned16(W->absmax)) ||
+      (W->absmax_q8 && !aligned16(W->absmax_q8)) ||
+      (W->absmax_scale && !aligned16(W->absmax_scale)))
+    return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+bool rank_ok(int r) { return r >= 8 && r <= 128 && (r % 8) == 0; }
+
+// ---------------------------------------------------------------------------------------------
+// Workspace layout (each region 256-byte aligned):
+//   [0]  small0  bf16 [M, r]   s*XA (forward) / dYB (backward)
+//   [1]  small1  bf16 [M, r]   s*dYB (backward)
+//   [2]  down    fp32 split partials of the rank-r down-projection
+//   [3]  grad    fp32 split partials of dB / dA (used one after the other)
+// ---------------------------------------------------------------------------------------------
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+  size_t small0, small1, down, grad, total;
+};
+
+WsLayout ws_layout(int M, int N, int K, int r) {
+  WsLayout L;
+  const size_t small = align256(static_cast<size_t>(M) * r * 2);
+  const size_t down = align256(4 * std::max(lora_down_plan(M, K, r).partial_floats,
+                                            lora_down_plan(M, N, r).partial_floats));
+  const size_t grad = align256(4 * std::max(lora_grad_plan(M, N, r).partial_floats,
+                                            lora_grad_plan(M, K, r).partial_floats));
+  L.small0 = 0;
+  L.small1 = small;
+  L.down = 2 * small;
+  L.grad = L.down + down;
+  L.total = L.grad + grad;
+  return L;
+}
+
+GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, bool trans, void* out, int* err) {
+  GemmArgs a;
+  a.M = M;
+  a.rows_w = trans ? W->K : W->N;
+  a.kt = (trans ? W->N : W->K) / 64;
+  a.r_pad16 = (r + 15) / 16 * 16;
+  a.n_ext = (a.r_pad16 + 63) / 64;
+  a.bt = gemm_pick_bt(M);
+  a.stages = gemm_pick_stages(a.bt);
+  a.kblocks = W->K / 64;
+  a.N = W->N;
+  a.dq = W->double_quant ? 1 : 0;
+  a.absmax = W->absmax;
+  a.absmax_q8 = W->absmax_q8;
+  a.absmax_scale = W->absmax_scale;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.err = err;
+  a.cb = codebook();
+  return a;
+}
+
+// Maps for the dequant GEMM.  act: [M, red] bf16; ext_act: [M, r] bf16 (scaled rank-r term).
+qlora_status gemm_maps(GemmMaps* m, const qlora_nf4_weight* W, bool trans, const void* act,
+                       const void* ext_w, const void* ext_act, int M, int r, int bt) {
+  const uint64_t red = trans ? W->N : W->K;
+  qlora_status st;
+  st = encode_2d(&m->act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, red, M, red * 2, 64, bt,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLORA_OK) return st;
+  if (!trans)
+    st = encode_2d(&m->q, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->q, W->K / 2, W->N, W->K / 2, 32, 128,
+                   CU_TENSOR_MAP_SWIZZLE_32B);
+  else
+    st = encode_2d(&m->q, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->q, W->K / 2, W->N, W->K / 2, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != QLORA_OK) return st;
+  if (!trans)  // B_lora [N, r]
+    st = encode_2d(&m->ext_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ext_w, r, W->N, r * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  else  // A_lora [r, K]
+    st = encode_2d(&m->ext_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ext_w, W->K, r, W->K * 2, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLORA_OK) return st;
+  return encode_2d(&m->ext_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ext_act, r, M, r * 2, 64, bt,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+std::atomic<uint64_t> g_launches{0};
+void count(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------------------------------------
+// Stage bodies (validated by their callers).
+// ---------------------------------------------------------------------------------------------
+qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc, int r,
+                          float scale, void* saved, void* scaled, float* partial,
+                          cudaStream_t s) {
+  const DownPlan dp = lora_down_plan(M, C, r);
+  cudaError_t e = launch_lora_down(static_cast<const __nv_bfloat16*>(in), M, C,
+                                   static_cast<const __nv_bfloat16*>(w), w_rc, r, scale,
+                                   static_cast<__nv_bfloat16*>(saved),
+                                   static_cast<__nv_bfloat16*>(scaled), partial, dp, s);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  count(dp.split > 1 ? 2 : 1);
+  return QLORA_OK;
+}
+
+qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
+                     const void* ext_act, int M, int r, void* out, int* err, cudaStream_t s) {
+  GemmArgs a = gemm_args(W, M, r, trans, out, err);
+  GemmMaps maps;
+  qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, a.bt);
+  if (st != QLORA_OK) return st;
+  if (launch_qlora_gemm(trans, maps, a, s) != cudaSuccess) return QLORA_ERR_CUDA;
+  count(1);
+  return QLORA_OK;
+}
+
+qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int r, float scale,
+                          float* out, bool out_cr, float* partial, cudaStream_t s) {
+  const GradPlan gp = lora_grad_plan(M, C, r);
+  cudaError_t e = launch_lora_grad(static_cast<const __nv_bfloat16*>(big), M, C,
+                                   static_cast<const __nv_bfloat16*>(small), r, scale, out,
+                                   out_cr, partial, gp, s);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  count(gp.split > 1 ? 2 : 1);
+  return QLORA_OK;
+}
+
+size_t down_ws_bytes(int M, int C, int r) { return 4 * lora_down_plan(M, C, r).partial_floats; }
+size_t grad_ws_bytes(int M, int C, int r) { return 4 * lora_grad_plan(M, C, r).partial_floats; }
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+const char* qlora_status_str(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_NULL: return "null pointer";
+    case QLORA_ERR_SHAPE: return "bad shape";
+    case QLORA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QLORA_ERR_ARCH: return "device is not sm_100 (B200)";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+qlora_status qlora_nf4_codebook(float out[16]) {
+  if (!out) return QLORA_ERR_NULL;
+  const Codebook& cb = codebook();
+  for (int i = 0; i < 16; ++i) out[i] = cb.level[i];
+  return QLORA_OK;
+}
+
+qlora_status qlora_nf4_pack(const void* W, int N, int K, int double_quant, uint8_t* q,
+                            float* absmax, uint8_t* absmax_q8, float* absmax_scale,
+                            qlora_stream_t stream) {
+  if (!W || !q || !absmax) return QLORA_ERR_NULL;
+  if (double_quant && (!absmax_q8 || !absmax_scale)) return QLORA_ERR_NULL;
+  if (N < 1 || K < 64 || (K % 64)) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(q) || !aligned16(absmax) ||
+      (double_quant && (!aligned16(absmax_q8) || !aligned16(absmax_scale))))
+    return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_nf4_pack(static_cast<const __nv_bfloat16*>(W), N, K,
+                                   double_quant ? 1 : 0, q, absmax, absmax_q8, absmax_scale,
+                                   codebook(), static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(double_quant ? 3 : 1);
+  return st;
+}
+
+qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, qlora_stream_t stream) {
+  if (!W || !W->q || !Wd) return QLORA_ERR_NULL;
+  if (W->double_quant ? (!W->absmax_q8 || !W->absmax_scale) : !W->absmax) return QLORA_ERR_NULL;
+  if (W->N < 1 || W->K < 64 || (W->K % 64)) return QLORA_ERR_SHAPE;
+  if (!aligned16(W->q) || !aligned16(Wd)) return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_nf4_dequant(W->q, W->absmax, W->absmax_q8, W->absmax_scale,
+                                      W->double_quant ? 1 : 0, W->N, W->K,
+                                      static_cast<__nv_bfloat16*>(Wd), codebook(),
+                                      static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+size_t qlora_workspace_bytes(int M, int N, int K, int r) {
+  if (M < 1 || N < 64 || K < 64 || !rank_ok(r)) return 0;
+  return ws_layout(M, N, K, r).total;
+}
+
+qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
+                              const void* B, int M, int r, float alpha, void* H, void* XA_saved,
+                              void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!X || !A || !B || !H || !XA_saved) return QLORA_ERR_NULL;
+  qlora_status st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
+    return QLORA_ERR_ALIGN;
+  const WsLayout L = ws_layout(M, W->N, W->K, r);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
+  const float scale = alpha / static_cast<float>(r);
+
+  // XA = X A^T (saved, bf16) and s * XA (the scaled operand of the fused up-projection).
+  st = do_lora_down(X, M, W->K, A, true, r, scale, XA_saved, sxa,
+                    reinterpret_cast<float*>(w8 + L.down), s);
+  if (st != QLORA_OK) return st;
+  // h = X deq(W0)^T + (s XA) B^T.
+  return do_gemm(X, W, false, B, sxa, M, r, H, err, s);
+}
+
+qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
+                              const void* A, const void* B, const void* XA_saved, int M, int r,
+                              float alpha, void* dX, float* dA, float* dB, void* ws,
+                              size_t ws_bytes, qlora_stream_t stream) {
+  if (!dY || !X || !A || !B || !XA_saved || !dA || !dB) return QLORA_ERR_NULL;
+  qlora_status st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) ||
+      !aligned16(XA_saved) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)))
+    return QLORA_ERR_ALIGN;
+  const WsLayout L = ws_layout(M, W->N, W->K, r);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  auto* dyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
+  auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
+  float* grad_part = reinterpret_cast<float*>(w8 + L.grad);
+  const float scale = alpha / static_cast<float>(r);
+  const auto* dYb = static_cast<const __nv_bfloat16*>(dY);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+
+  // dYB = dY B (bf16, for dA) and s * dYB (operand of the fused dX up-projection).
+  st = do_lora_down(dY, M, W->N, B, false, r, scale, dyb, sdyb,
+                    reinterpret_cast<float*>(w8 + L.down), s);
+  if (st != QLORA_OK) return st;
+  // dX = dY deq(W0) + (s dYB) A.
+  if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, r, dX, err, s)) != QLORA_OK) return st;
+  // dB = s dY^T XA  [N, r];  dA = s dYB^T X  [r, K].
+  st = do_lora_grad(dY, M, W->N, XA_saved, r, scale, dB, true, grad_part, s);
+  if (st != QLORA_OK) return st;
+  return do_lora_grad(X, M, W->K, dyb, r, scale, dA, false, grad_part, s);
+}
+
+qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_is_r_by_c, int r,
+                             float scale, void* saved, void* scaled, void* ws, size_t ws_bytes,
+                             qlora_stream_t stream) {
+  if (!in || !w || !scaled) return QLORA_ERR_NULL;
+  if (M < 1 || C < 64 || (C % 64) || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (!aligned16(in) || !aligned16(w) || !aligned16(scaled) || (saved && !aligned16(saved)))
+    return QLORA_ERR_ALIGN;
+  const size_t need = down_ws_bytes(M, C, r);
+  if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  return do_lora_down(in, M, C, w, w_is_r_by_c != 0, r, scale, saved, scaled,
+                      static_cast<float*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
+                            const void* ext_w, const void* ext_act, int M, int r, void* out,
+                            qlora_stream_t stream) {
+  if (!act || !ext_w || !ext_act || !out) return QLORA_ERR_NULL;
+  qlora_status st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (!aligned16(act) || !aligned16(ext_w) || !aligned16(ext_act) || !aligned16(out))
+    return QLORA_ERR_ALIGN;
+  int dev;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  return do_gemm(act, W, transpose_w != 0, ext_w, ext_act, M, r, out, err,
+                 static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, int r,
+                             float scale, float* out, int out_r_by_c, void* ws, size_t ws_bytes,
+                             qlora_stream_t stream) {
+  if (!big || !small || !out) return QLORA_ERR_NULL;
+  if (M < 1 || C < 64 || (C % 64) || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (!aligned16(big) || !aligned16(small) || !aligned16(out)) return QLORA_ERR_ALIGN;
+  const size_t need = grad_ws_bytes(M, C, r);
+  if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  return do_lora_grad(big, M, C, small, r, scale, out, out_r_by_c == 0, static_cast<float*>(ws),
+                      static_cast<cudaStream_t>(stream));
+}
+
+uint64_t qlora_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qlora_status qlora_swiglu_fwd(const void* g, const void* u, void* a, int64_t n,
+                              qlora_stream_t stream) {
+  if (!g || !u || !a) return QLORA_ERR_NULL;
+  if (n < 0) return QLORA_ERR_SHAPE;
+  if (!aligned16(g) || !aligned16(u) || !aligned16(a)) return QLORA_ERR_ALIGN;
+  if (n == 0) return QLORA_OK;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_swiglu_fwd(static_cast<const __nv_bfloat16*>(g),
+                                     static_cast<const __nv_bfloat16*>(u),
+                                     static_cast<__nv_bfloat16*>(a), n,
+                                     static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void* da, void* dg, void* du,
+                              int64_t n, qlora_stream_t stream) {
+  if (!g || !u || !da || !dg || !du) return QLORA_ERR_NULL;
+  if (n < 0) return QLORA_ERR_SHAPE;
+  if (!aligned16(g) || !aligned16(u) || !aligned16(da) || !aligned16(dg) || !aligned16(du))
+    return QLORA_ERR_ALIGN;
+  if (n == 0) return QLORA_OK;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_swiglu_bwd(
+      static_cast<const __nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(u),
+      static_cast<const __nv_bfloat16*>(da), static_cast<__nv_bfloat16*>(dg),
+      static_cast<__nv_bfloat16*>(du), n, static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+qlora_status qlora_device_error(int* code) {
+  if (!code) return QLORA_ERR_NULL;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_qlora_error_word, sizeof(int)) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  *code = v;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_qlora_error_word, &zero, sizeof(int)) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return QLORA_ERR_TIMEOUT;
+  }
+  return QLORA_OK;
+}
+
+}  // extern "C"

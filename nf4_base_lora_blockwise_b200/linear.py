@@ -1,0 +1,140 @@
+"""Tensor-level API over the C ABI: torch tensors in, torch tensors out.
+
+PyTorch provides device memory and the current CUDA stream; every step of the computation runs
+in libqlora_nf4.so.  All tensors must be contiguous CUDA tensors on the current device.
+"""
+
+from dataclasses import dataclass
+
+import torch
+
+from . import abi
+
+
+def _ptr(t):
+    return t.data_ptr() if t is not None else None
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _need(t, dtype, shape, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+@dataclass
+class NF4Weight:
+    """A packed NF4 base weight W0 [N, K] (device tensors owned by this object)."""
+    q: torch.Tensor                      # [N, K/2] uint8
+    absmax: torch.Tensor                 # [N*K/64] fp32 (first-level absmax)
+    absmax_q8: torch.Tensor = None       # [N*K/64] uint8 (double-quantised)
+    absmax_scale: torch.Tensor = None    # [ceil(N*K/64/256)] fp32
+    N: int = 0
+    K: int = 0
+    double_quant: bool = False
+
+    def c_struct(self):
+        return abi.Nf4Weight(
+            _ptr(self.q), None if self.double_quant else _ptr(self.absmax),
+            _ptr(self.absmax_q8) if self.double_quant else None,
+            _ptr(self.absmax_scale) if self.double_quant else None,
+            self.N, self.K, 1 if self.double_quant else 0)
+
+
+def nf4_pack(W, double_quant=False):
+    """Quantise a bf16 weight [N, K] to NF4 (qlora_nf4_pack)."""
+    N, K = W.shape
+    _need(W, torch.bfloat16, (N, K), "W")
+    dev = W.device
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    nb = N * (K // 64)
+    absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    q8 = scale = None
+    if double_quant:
+        q8 = torch.empty(nb, dtype=torch.uint8, device=dev)
+        scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    abi.qlora_nf4_pack(W.data_ptr(), N, K, double_quant, q.data_ptr(), absmax.data_ptr(),
+                       _ptr(q8), _ptr(scale), _stream())
+    return NF4Weight(q, absmax, q8, scale, N, K, bool(double_quant))
+
+
+def nf4_dequant(w: NF4Weight):
+    """bf16 [N, K] dequantised weight (test / diagnostic export, qlora_nf4_dequant)."""
+    out = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.q.device)
+    abi.qlora_nf4_dequant(w.c_struct(), out.data_ptr(), _stream())
+    return out
+
+
+def workspace_bytes(M, N, K, r):
+    return abi.qlora_workspace_bytes(M, N, K, r)
+
+
+def alloc_workspace(M, N, K, r, device):
+    n = workspace_bytes(M, N, K, r)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def forward(X, w: NF4Weight, A, B, alpha, H=None, XA=None, ws=None):
+    """h = X deq(W0)^T + (alpha/r) (X A^T) B^T.  Returns (h, XA_saved)."""
+    M, K = X.shape
+    r = A.shape[0]
+    _need(X, torch.bfloat16, (M, w.K), "X")
+    _need(A, torch.bfloat16, (r, w.K), "A")
+    _need(B, torch.bfloat16, (w.N, r), "B")
+    if H is None:
+        H = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    if XA is None:
+        XA = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = alloc_workspace(M, w.N, w.K, r, X.device)
+    abi.qlora_linear_fwd(X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(), M, r, alpha,
+                         H.data_ptr(), XA.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
+    return H, XA
+
+
+def backward(dY, X, w: NF4Weight, A, B, XA, alpha, need_dx=True, dX=None, dA=None, dB=None,
+             ws=None):
+    """Hand-derived gradients.  Returns (dX or None, dA fp32 [r, K], dB fp32 [N, r])."""
+    M = X.shape[0]
+    r = A.shape[0]
+    _need(dY, torch.bfloat16, (M, w.N), "dY")
+    _need(X, torch.bfloat16, (M, w.K), "X")
+    _need(XA, torch.bfloat16, (M, r), "XA")
+    dev = X.device
+    if need_dx and dX is None:
+        dX = torch.empty((M, w.K), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, w.K), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((w.N, r), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_workspace(M, w.N, w.K, r, dev)
+    abi.qlora_linear_bwd(dY.data_ptr(), X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(),
+                         XA.data_ptr(), M, r, alpha, _ptr(dX) if need_dx else None,
+                         dA.data_ptr(), dB.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
+    return (dX if need_dx else None), dA, dB
+
+
+def swiglu_forward(g, u, a=None):
+    if a is None:
+        a = torch.empty_like(g)
+    abi.qlora_swiglu_fwd(g.data_ptr(), u.data_ptr(), a.data_ptr(), g.numel(), _stream())
+    return a
+
+
+def swiglu_backward(g, u, da, dg=None, du=None):
+    if dg is None:
+        dg = torch.empty_like(g)
+    if du is None:
+        du = torch.empty_like(g)
+    abi.qlora_swiglu_bwd(g.data_ptr(), u.data_ptr(), da.data_ptr(), dg.data_ptr(), du.data_ptr(),
+                         g.numel(), _stream())
+    return dg, du
+
+
+def device_error():
+    """Synchronising: the device error word (0 = none), cleared after reading."""
+    return abi.qlora_device_error()

@@ -4,8 +4,9 @@ This module only draws random numbers in a fixed order and casts them to bf16; i
 of the method's arithmetic (no quantisation, no products).  Both the GPU tests and the CPU
 oracle take their inputs from here.
 
-Recipe: one ``torch.Generator`` (CPU) seeded with ``seed`` draws, in this order, X, then for
-each linear W0, A, B, then dY.  Values are drawn in fp32 and cast to bf16 (round to nearest
+Recipe: one ``torch.Generator`` (CPU) seeded with ``seed`` draws, in this order: for a single
+linear (or independent projections, one after the other) X, W0, A, B, dY; for the MLP
+workload X, then W0, A, B of gate, up and down, then dY.  Values are drawn in fp32 and cast to bf16 (round to nearest
 even).  "N(0, s)" means standard deviation s.  The LoRA down-projection A is either uniform
 on (-a, a) with a = 1/sqrt(in) ("Kaiming-uniform" with torch's nn.Linear default slope
 sqrt(5)), or the explicit bound of the tiny workload.  B is N(0, 0.01) -- non-zero, so the
@@ -13,7 +14,7 @@ LoRA path contributes to h and to dX.
 """
 
 import math
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import torch
 
@@ -93,22 +94,37 @@ def _uniform(gen, shape, bound):
 def make_inputs(w, seed=0):
     """Draw the inputs of workload ``w`` on the CPU as bf16 tensors.
 
-    Returns ``{"X": [M, K0], "linears": [{"W0", "A", "B"} per linear], "dY": [M, N_last]}``.
-    For the MLP workload X feeds gate and up, and dY is the gradient at the down output.
+    MLP workload: X [M, K_gate], then W0, A, B of gate, up and down, then dY [M, N_down] (the
+    gradient at the down output).  Other workloads: for each linear, X [M, K], W0, A, B, then
+    dY [M, N] -- independent projections, each with its own activations.
+
+    Returns ``{"X", "dY", "linears": [{"W0", "A", "B", "X", "dY"}]}``; the top-level X and dY
+    are those of the first linear (MLP: the MLP input and the down-output gradient).
     """
     gen = torch.Generator(device="cpu")
     gen.manual_seed(seed)
-    K0 = w.linears[0].K
-    X = _normal(gen, (w.M, K0), w.x_std)
-    lins = []
-    for L in w.linears:
+
+    def draw_weights(L):
         W0 = _normal(gen, (L.N, L.K), L.w_std)
         bound = w.a_bound if w.a_bound > 0 else 1.0 / math.sqrt(L.K)
         A = _uniform(gen, (L.r, L.K), bound)
         B = _normal(gen, (L.N, L.r), w.b_std)
-        lins.append({"W0": W0, "A": A, "B": B})
-    dY = _normal(gen, (w.M, w.linears[-1].N), w.dy_std)
-    return {"X": X, "linears": lins, "dY": dY}
+        return {"W0": W0, "A": A, "B": B}
+
+    lins = []
+    if w.mlp:
+        X = _normal(gen, (w.M, w.linears[0].K), w.x_std)
+        for L in w.linears:
+            lins.append(draw_weights(L))
+        dY = _normal(gen, (w.M, w.linears[-1].N), w.dy_std)
+        return {"X": X, "linears": lins, "dY": dY}
+    for L in w.linears:
+        X = _normal(gen, (w.M, L.K), w.x_std)
+        d = draw_weights(L)
+        d["X"] = X
+        d["dY"] = _normal(gen, (w.M, L.N), w.dy_std)
+        lins.append(d)
+    return {"X": lins[0]["X"], "linears": lins, "dY": lins[0]["dY"]}
 
 
 def make_linear(M, K, N, r, alpha=None, seed=0, x_std=1.0, w_std=0.02, a_bound=0.0,

@@ -1,0 +1,115 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI and the CPU
+oracle on the same seeded inputs, and compare (bit-exact for codes, absmax and dequantised
+weights; max|err| / max|ref| <= TOL for the floating-point outputs)."""
+
+import numpy as np
+import torch
+
+from nf4_base_lora_blockwise_b200 import linear, synth
+from oracle import nf4, qlora
+
+# Tolerance stated for the bf16-in / fp32-accumulate outputs h, dX, dA, dB.
+TOL = 2e-2
+
+
+def f32(t):
+    """bf16/fp32 torch tensor (any device) -> float32 numpy (exact for bf16 values)."""
+    return t.detach().to("cpu").float().numpy()
+
+
+def bits(t):
+    """bf16 torch tensor -> uint16 numpy bit patterns."""
+    return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_pack(W_bf16_cpu, dq, rows=None):
+    """Oracle quantisation of W0.  With ``rows``, codes are produced for those rows only
+    (absmax and the double-quant groups always cover the whole weight)."""
+    w = f32(W_bf16_cpu)
+    N, K = w.shape
+    am = nf4.block_absmax(w)
+    out = {"absmax": am.reshape(-1)}
+    if dq:
+        q8, sc = nf4.double_quant(am.reshape(-1))
+        eff = nf4.dq_effective_absmax(q8, sc).reshape(N, K // 64)
+        out["absmax_q8"], out["absmax_scale"] = q8, sc
+    else:
+        eff = am
+    out["absmax_eff"] = eff
+    sel = np.arange(N) if rows is None else np.asarray(rows)
+    out["rows"] = sel
+    out["q"] = nf4.pack_codes(nf4.choose_codes(w[sel], eff[sel]))
+    return out
+
+
+def gpu_pack(W_bf16_cpu, dq):
+    W = W_bf16_cpu.cuda()
+    w = linear.nf4_pack(W, double_quant=dq)
+    torch.cuda.synchronize()
+    return w
+
+
+def check_pack(wg, ref, dq):
+    """Bit-exact: codes, absmax (and q8 / scale), and the dequantised weight."""
+    rows = ref["rows"]
+    q = wg.q.cpu().numpy()[rows]
+    assert np.array_equal(q, ref["q"]), "packed codes differ"
+    assert np.array_equal(wg.absmax.cpu().numpy().view(np.uint32),
+                          ref["absmax"].view(np.uint32)), "absmax differs"
+    if dq:
+        assert np.array_equal(wg.absmax_q8.cpu().numpy(), ref["absmax_q8"]), "q8 differs"
+        assert np.array_equal(wg.absmax_scale.cpu().numpy().view(np.uint32),
+                              ref["absmax_scale"].view(np.uint32)), "scale differs"
+    deq = bits(linear.nf4_dequant(wg))[rows]
+    N, K = wg.N, wg.K
+    ref_deq = nf4.dequantize_bits(ref["q"], ref["absmax_eff"][rows], len(rows), K)
+    assert np.array_equal(deq, ref_deq), "dequantised weight differs"
+
+
+def oracle_deq(W_bf16_cpu, dq):
+    ref = oracle_pack(W_bf16_cpu, dq)
+    N, K = W_bf16_cpu.shape
+    return ref, nf4.dequantize(ref["q"], ref["absmax_eff"], N, K)
+
+
+def run_linear(inp, L, dq=None, need_dx=True):
+    """GPU pack + forward + backward of one linear; returns a dict of CPU tensors."""
+    dq = L.double_quant if dq is None else dq
+    lin = inp["linears"][0]
+    X, dY = inp["X"].cuda(), inp["dY"].cuda()
+    A, B = lin["A"].cuda(), lin["B"].cuda()
+    w = linear.nf4_pack(lin["W0"].cuda(), double_quant=dq)
+    H, XA = linear.forward(X, w, A, B, L.alpha)
+    dX, dA, dB = linear.backward(dY, X, w, A, B, XA, L.alpha, need_dx=need_dx)
+    torch.cuda.synchronize()
+    assert linear.device_error() == 0
+    return {"w": w, "H": H, "XA": XA, "dX": dX, "dA": dA, "dB": dB}
+
+
+def check_linear(inp, L, got, rows=None, dq=None):
+    """Compare the GPU outputs with the oracle (all rows, or the sampled ``rows``)."""
+    dq = L.double_quant if dq is None else dq
+    lin = inp["linears"][0]
+    ref, Wd = oracle_deq(lin["W0"], dq)
+    X, dY, A, B = (f32(inp["X"]), f32(inp["dY"]), f32(lin["A"]), f32(lin["B"]))
+    M = X.shape[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    errs = {}
+    h_ref = qlora.forward_rows(X, Wd, A, B, L.alpha, rows)
+    errs["h"] = qlora.rel_err(f32(got["H"])[rows], h_ref)
+    errs["XA"] = qlora.rel_err(f32(got["XA"]), qlora.lora_down(X, A))
+    wts = qlora.backward_weights(dY, X, A, B, L.alpha)
+    errs["dA"] = qlora.rel_err(f32(got["dA"]), wts["dA"])
+    errs["dB"] = qlora.rel_err(f32(got["dB"]), wts["dB"])
+    if got["dX"] is not None:
+        dx_ref = qlora.backward_dx_rows(dY, Wd, A, B, L.alpha, rows)
+        errs["dX"] = qlora.rel_err(f32(got["dX"])[rows], dx_ref)
+    for k, v in errs.items():
+        assert v <= TOL, f"{k}: max|err|/max|ref| = {v:.3e} > {TOL}"
+    return errs, ref
+
+
+def make(M, K, N, r, alpha=None, seed=0, **kw):
+    inp = synth.make_linear(M, K, N, r, alpha=alpha, seed=seed, **kw)
+    L = synth.LinearShape("linear", K, N, r, alpha if alpha else 2.0 * r)
+    return inp, L

@@ -1,0 +1,90 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point include/*.h declares,
+its host-side codebook equals the oracle's bit for bit, and its argument validation answers
+before any device work (no GPU needed: these paths return before the first CUDA call)."""
+
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+from nf4_base_lora_blockwise_b200 import abi
+from oracle import nf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(abi.LIB_PATH):
+        from nf4_base_lora_blockwise_b200 import build
+        build.build()
+    return abi._lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h).read()
+        names |= set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(qlora_\w+)\s*\(", txt))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert declared == set(abi.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.qlora_status_str(code)
+
+
+def test_codebook_matches_oracle_bit_exact(lib):
+    """Two independent derivations of the NF4 levels (C++ bisection on erfc in the library,
+    scipy's ndtri in the oracle) agree on every fp32 bit."""
+    got = np.array(abi.qlora_nf4_codebook(), dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), nf4.codebook_f32().view(np.uint32))
+
+
+FAKE = 1 << 20          # an aligned, non-null address: never dereferenced on these paths
+
+
+def _w(N=128, K=256, dq=0, q=FAKE, absmax=FAKE):
+    return abi.Nf4Weight(q, absmax if not dq else None, FAKE if dq else None,
+                         FAKE if dq else None, N, K, dq)
+
+
+def _fwd(lib, X=FAKE, W=None, M=64, r=16, H=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    W = W or _w()
+    return lib.qlora_linear_fwd(X, ctypes.byref(W), FAKE, FAKE, M, r, 32.0, H, FAKE, ws,
+                                ws_bytes, None)
+
+
+def test_validation_codes(lib):
+    assert _fwd(lib, X=None) == 1                      # NULL
+    assert _fwd(lib, W=_w(q=None)) == 1
+    assert _fwd(lib, W=_w(K=100)) == 2                 # K % 64
+    assert _fwd(lib, W=_w(N=96)) == 2                  # N % 64
+    assert _fwd(lib, M=0) == 2
+    assert _fwd(lib, r=12) == 2                        # r not a multiple of 8
+    assert _fwd(lib, r=136) == 2
+    assert _fwd(lib, X=FAKE + 8) == 3                  # misaligned
+    assert _fwd(lib, ws_bytes=16) == 5                 # workspace too small
+    assert _fwd(lib, ws=None) == 5
+    assert lib.qlora_nf4_pack(FAKE, 64, 100, 0, FAKE, FAKE, None, None, None) == 2
+    assert lib.qlora_nf4_pack(FAKE, 64, 128, 1, FAKE, FAKE, None, None, None) == 1
+
+
+def test_workspace_bytes(lib):
+    assert lib.qlora_workspace_bytes(0, 128, 128, 16) == 0
+    assert lib.qlora_workspace_bytes(64, 128, 128, 12) == 0
+    small = lib.qlora_workspace_bytes(64, 512, 256, 8)
+    big = lib.qlora_workspace_bytes(4096, 4096, 4096, 16)
+    assert 0 < small < big
+    assert big >= 2 * 4096 * 16 * 2                    # the two bf16 rank-r activations
