@@ -29,7 +29,8 @@ struct GemmArgs {
   int kt;          // reduction steps of 64
   int n_ext;       // LoRA extension chunks (64 wide along r)
   int r_pad16;     // r rounded up to a multiple of 16
-  int bt;          // token tile = MMA N
+  int bt;          // tokens per half tile = MMA N
+  int nh;          // token halves per tile (1 or 2)
   int stages;
   int kblocks;     // K / 64 = absmax blocks per row of W0
   int N;           // rows of W0
@@ -50,8 +51,9 @@ struct GemmMaps {
 };
 
 int gemm_pick_bt(int M);
+int gemm_pick_halves(int M);
 int gemm_pick_stages(int bt);
-size_t gemm_smem_bytes(int bt, int stages);
+size_t gemm_smem_bytes(int bt, int nh);
 cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, const GemmArgs& args,
                               cudaStream_t stream);
 

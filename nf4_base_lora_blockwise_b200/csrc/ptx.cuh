@@ -71,21 +71,63 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  Returns false (and records `site` in
-// the device error word `err`) if the limit runs out, or if another wait already failed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site, int* err) {
+// try_wait with a suspend-time hint: a thread whose phase is not yet complete is suspended in
+// hardware until the phase completes or about `hint_ns` pass, instead of re-polling the
+// barrier (many polling warps saturate the shared-memory barrier path and slow every other
+// barrier operation, the MMA issue included).
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false if the limit runs out --
+// recording in the device error word `err` the wait site (bits 0-3), the CTA (bits 4-11, low 8
+// bits of blockIdx.x) and a caller tag such as the pipeline step (bits 12-30) -- or if
+// another wait already failed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site, int* err,
+                                          int tag = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (*(volatile int*)err != 0) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicCAS(err, 0, site);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*(volatile int*)err != 0) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      const int code = (site & 0xF) | ((static_cast<int>(blockIdx.x) & 0xFF) << 4) |
+                       ((tag & 0x7FFFF) << 12);
+      atomicCAS(err, 0, code == 0 ? 1 : code);
+      return false;
     }
   }
+}
+
+// Warp-wide bounded wait: lane 0 polls (so a waiting warp costs one lane's polling, not 32),
+// then every lane takes the completed phase itself with one more try_wait (acquire per thread).
+// Must be called by all 32 lanes; returns a warp-uniform result.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int site,
+                                               int* err, int tag = 0) {
+  bool ok = true;
+  if ((threadIdx.x & 31u) == 0u) ok = mbar_wait(bar, parity, site, err, tag);
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+  if (ok) {
+    for (int i = 0; i < 64 && !mbar_try_wait(bar, parity); ++i) {
+    }
+  }
+  return ok;
+}
+
+// Bounded wait for a barrier that completes rarely (once per tile).
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, int site,
+                                                 int* err, int tag = 0) {
+  return mbar_wait(bar, parity, site, err, tag);
 }
 
 // ---------------------------------- TMA ---------------------------------------------------

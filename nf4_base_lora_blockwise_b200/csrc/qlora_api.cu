@@ -186,6 +186,7 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, bool trans, void* ou
   a.r_pad16 = (r + 15) / 16 * 16;
   a.n_ext = (a.r_pad16 + 63) / 64;
   a.bt = gemm_pick_bt(M);
+  a.nh = gemm_pick_halves(M);
   a.stages = gemm_pick_stages(a.bt);
   a.kblocks = W->K / 64;
   a.N = W->N;

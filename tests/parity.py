@@ -82,7 +82,8 @@ def run_linear(inp, L, dq=None, need_dx=True):
     H, XA = linear.forward(X, w, A, B, L.alpha)
     dX, dA, dB = linear.backward(dY, X, w, A, B, XA, L.alpha, need_dx=need_dx)
     torch.cuda.synchronize()
-    assert linear.device_error() == 0
+    code = linear.device_error()
+    assert code == 0, f"device error word set: {code}"
     return {"w": w, "H": H, "XA": XA, "dX": dX, "dA": dA, "dB": dB}
 
 
