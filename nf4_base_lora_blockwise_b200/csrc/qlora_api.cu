@@ -393,8 +393,6 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_wei
   auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
   float* grad_part = reinterpret_cast<float*>(w8 + L.grad);
   const float scale = alpha / static_cast<float>(r);
-  const auto* dYb = static_cast<const __nv_bfloat16*>(dY);
-  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
 
   // dYB = dY B (bf16, for dA) and s * dYB (operand of the fused dX up-projection).
   st = do_lora_down(dY, M, W->N, B, false, r, scale, dyb, sdyb,
