@@ -163,6 +163,30 @@ QLORA_API qlora_status qlora_lora_grad(const void* big, int M, int C, const void
 /* Number of kernels this library has launched in this process so far (all devices). */
 QLORA_API uint64_t qlora_launch_counter(void);
 
+/* ---- Allocation-free forward (no counterpart on the pages: an engineering addition). ----
+ *
+ * For callers that cannot allocate device memory at all -- for example code running inside
+ * a host framework that owns every device allocation and hands out no workspace, or a host
+ * that links this C ABI without any device allocator of its own -- and so cannot provide the
+ * `ws` buffer qlora_linear_fwd needs.  Same computation and arguments as qlora_linear_fwd
+ * minus the workspace: the scratch (the scaled rank-r activation s*XA and the down-projection
+ * partials) lives in a fixed array inside this library, qlora_noalloc_scratch_bytes() bytes
+ * per GPU (8 MiB), which every GPU that loads the library keeps until the process exits.
+ * Returns QLORA_ERR_WORKSPACE, before enqueuing anything, when (M, K, r) would need more
+ * scratch than that (roughly 2*M*r bytes plus M*r*4 bytes per split of the down-projection).
+ * The first call on a device looks up the array's device address (with that device current),
+ * so make that first call before any stream capture.  The entry point calls no cudaMalloc or
+ * cudaFree.  All calls on a device share the one array and each call overwrites it in full
+ * (it keeps the last call's contents; nothing in it must start at zero): calls whose kernels
+ * overlap on the GPU -- on different streams without ordering between them -- race. */
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W,
+                                                const void* A, const void* B, int M, int r,
+                                                float alpha, void* H, void* XA_saved,
+                                                qlora_stream_t stream);
+
+/* Size in bytes of the fixed scratch array used by qlora_linear_fwd_noalloc. */
+QLORA_API size_t qlora_noalloc_scratch_bytes(void);
+
 /* Synchronising: returns the device error word of the current device (0 = none; otherwise
  * a code naming the wait that ran out) and clears it. */
 QLORA_API qlora_status qlora_device_error(int* code);

@@ -26,6 +26,8 @@ EXPORTS = (
     "qlora_nf4_gemm",
     "qlora_lora_grad",
     "qlora_launch_counter",
+    "qlora_linear_fwd_noalloc",
+    "qlora_noalloc_scratch_bytes",
     "qlora_device_error",
 )
 
@@ -86,6 +88,9 @@ def _lib():
                                     _VP]),
             "qlora_lora_grad": (_I, [_VP, _I, _I, _VP, _I, _F, _VP, _I, _VP, _SZ, _VP]),
             "qlora_launch_counter": (ctypes.c_uint64, []),
+            "qlora_linear_fwd_noalloc": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _I, _I,
+                                              _F, _VP, _VP, _VP]),
+            "qlora_noalloc_scratch_bytes": (_SZ, []),
             "qlora_device_error": (_I, [ctypes.POINTER(ctypes.c_int)]),
         }
         for name, (res, args) in sig.items():
@@ -165,6 +170,16 @@ def qlora_lora_grad(big, M, C, small, r, scale, out, out_r_by_c, ws, ws_bytes, s
 
 def qlora_launch_counter():
     return int(_lib().qlora_launch_counter())
+
+
+def qlora_linear_fwd_noalloc(X, weight, A, B, M, r, alpha, H, XA_saved, stream):
+    _check("qlora_linear_fwd_noalloc",
+           _lib().qlora_linear_fwd_noalloc(X, ctypes.byref(weight), A, B, M, r, float(alpha), H,
+                                           XA_saved, stream))
+
+
+def qlora_noalloc_scratch_bytes():
+    return int(_lib().qlora_noalloc_scratch_bytes())
 
 
 def qlora_device_error():

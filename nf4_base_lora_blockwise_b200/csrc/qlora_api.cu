@@ -275,6 +275,32 @@ size_t grad_ws_bytes(int M, int C, int r) { return 4 * lora_grad_plan(M, C, r).p
 }  // namespace
 }  // namespace qlora
 
+// ---------------------------------------------------------------------------------------------
+// Fixed scratch for qlora_linear_fwd_noalloc: a file-scope device array, so that entry point
+// needs no caller-provided workspace and allocates nothing.  Every GPU that loads this library
+// holds the array until the process exits.  In host code the name is only a host-side stand-in
+// for the device symbol; kernels get its device address, looked up once per device with that
+// device current (cudaGetSymbolAddress).
+// ---------------------------------------------------------------------------------------------
+namespace qlora {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices];
+
+qlora_status noalloc_scratch(int dev, void** p) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || !a) return QLORA_ERR_CUDA;
+    g_noalloc_ptr[dev] = a;
+  }
+  *p = g_noalloc_ptr[dev];
+  return QLORA_OK;
+}
+}  // namespace
+}  // namespace qlora
+
 using namespace qlora;
 
 extern "C" {
@@ -492,6 +518,38 @@ qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void* da, void
   if (st == QLORA_OK) count(1);
   return st;
 }
+
+qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, const void* A,
+                                      const void* B, int M, int r, float alpha, void* H,
+                                      void* XA_saved, qlora_stream_t stream) {
+  if (!X || !A || !B || !H || !XA_saved) return QLORA_ERR_NULL;
+  qlora_status st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
+    return QLORA_ERR_ALIGN;
+  // The forward needs s*XA [M, r] bf16 plus the down-projection's split partials.
+  const size_t sxa_bytes = align256(static_cast<size_t>(M) * r * 2);
+  const size_t need = sxa_bytes + align256(down_ws_bytes(M, W->K, r));
+  if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+  int dev;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(scratch);
+  auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8);
+  const float scale = alpha / static_cast<float>(r);
+  // Both scratch regions are written in full before they are read: nothing needs clearing.
+  st = do_lora_down(X, M, W->K, A, true, r, scale, XA_saved, sxa,
+                    reinterpret_cast<float*>(w8 + sxa_bytes), s);
+  if (st != QLORA_OK) return st;
+  return do_gemm(X, W, false, B, sxa, M, r, H, err, s);
+}
+
+size_t qlora_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 qlora_status qlora_device_error(int* code) {
   if (!code) return QLORA_ERR_NULL;
