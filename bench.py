@@ -11,8 +11,8 @@ batch of synthetic tokens (seeded, resident in HBM before timing):
 
 run as the six library stages (lora_down, dequant GEMM, lora_down, dequant GEMM (dX),
 lora_grad x 2) with CUDA events between them on the launching stream, so the dominant
-kernel's own duration is measured live.  L2 is flushed (a 256 MiB write) before every step,
-outside the events.  One JSON line is printed by rank 0.
+kernel's own duration is measured live.  L2 is flushed before every step, outside the events:
+a 256 MiB write followed by a read of the same buffer, so no dirty line is left to write back.  One JSON line is printed by rank 0.
 
 Multi-GPU (torchrun): every rank runs an independent replica on its own batch (the layer's
 data path has no exchange step in one forward+backward); the step time is the max over ranks.
@@ -190,7 +190,10 @@ def run_steps(states, n, stream, flush, record):
     per_step = []
     per_stage = {}
     for _ in range(n):
+        # L2 flush: write 256 MiB, then read it back so the evicted lines are clean (the
+        # write-back of the flush's own dirty lines must not land on the first timed kernel).
         flush.zero_()
+        flush.max()
         evs = []
         calls = []
         for st in states:
@@ -381,7 +384,7 @@ def workload_config(w):
     c = {"workload": w.name, "M": w.M,
          "linears": [{"name": L.name, "K": L.K, "N": L.N, "r": L.r, "alpha": L.alpha,
                       "absmax": "double-quant" if L.double_quant else "fp32"} for L in w.linears],
-         "l2": "flushed before every step (256 MiB write)", "parallelism": "replicas"}
+         "l2": "flushed before every step (256 MiB write + read, outside the events)", "parallelism": "replicas"}
     return c
 
 

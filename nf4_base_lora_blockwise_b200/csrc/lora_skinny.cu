@@ -18,10 +18,25 @@ namespace qlora {
 
 namespace {
 
-constexpr int kTarget = 296;  // CTAs to aim for: two per SM on 148 SMs
-constexpr int kBM = 64;       // rows (tokens) per step
-constexpr int kBC = 64;       // columns per step
-constexpr int kPad = 8;       // bf16 padding per smem row (keeps ldmatrix conflict-free)
+constexpr int kTarget = 296;   // CTAs to aim for: two per SM on 148 SMs
+constexpr int kWarps = 8;      // 256 threads per CTA
+constexpr int kThreadsSk = 32 * kWarps;
+constexpr int kBM = 16 * kWarps;  // lora_down: token rows per CTA (16 per warp)
+constexpr int kBC = 64;        // lora_down: columns per pipeline step
+constexpr int kGC = 16 * kWarps;  // lora_grad: columns (of `big`) per CTA
+constexpr int kGM = 64;        // lora_grad: token rows per pipeline step
+constexpr int kPad = 8;        // bf16 padding per smem row (keeps ldmatrix conflict-free)
+
+// Pipeline depth: deeper for narrow ranks (small tiles), shallower when r is wide.
+__host__ __device__ constexpr int stages_for(int R) { return R <= 64 ? 4 : 3; }
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+  }
+}
 
 __device__ __forceinline__ uint32_t s_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -111,31 +126,35 @@ __device__ __forceinline__ void load_b_frags(uint32_t (&b)[NT][2], const __nv_bf
 }
 
 // ------------------------------------------------------------------------------------------
-// lora_down: grid (ceil(M/64), split).  4 warps, warp w owns rows 16w..16w+15 of the tile.
+// lora_down: grid (ceil(M/128), split).  8 warps, warp w owns rows 16w..16w+15 of the CTA's
+// 128 token rows; a multi-stage cp.async pipeline streams 64-column slices of `in` (and of Wl).
 // ------------------------------------------------------------------------------------------
 template <int NT, bool kWrc>
-__global__ void __launch_bounds__(128) lora_down_kernel(
+__global__ void __launch_bounds__(kThreadsSk) lora_down_kernel(
     const __nv_bfloat16* __restrict__ in, int M, int C, const __nv_bfloat16* __restrict__ w,
     float scale, __nv_bfloat16* __restrict__ saved, __nv_bfloat16* __restrict__ scaled,
     float* __restrict__ partial, int split) {
   constexpr int R = NT * 8;
+  constexpr int S = stages_for(R);
   constexpr int kInLd = kBC + kPad;
   constexpr int kWRows = kWrc ? R : kBC;
   constexpr int kWLd = kWrc ? (kBC + kPad) : (R + kPad);
   extern __shared__ __align__(16) uint8_t dsm_down[];
   auto s_in = reinterpret_cast<__nv_bfloat16(*)[kBM * kInLd]>(dsm_down);
   auto s_w = reinterpret_cast<__nv_bfloat16(*)[kWRows * kWLd]>(
-      dsm_down + 2 * kBM * kInLd * sizeof(__nv_bfloat16));
+      dsm_down + S * kBM * kInLd * sizeof(__nv_bfloat16));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * kBM;
   const int steps = C / kBC;
   const int sb = static_cast<int>((static_cast<long long>(steps) * blockIdx.y) / split);
   const int se = static_cast<int>((static_cast<long long>(steps) * (blockIdx.y + 1)) / split);
+  const int n = se - sb;
 
   auto load = [&](int buf, int step) {
     const int c0 = step * kBC;
-    for (int i = tid; i < kBM * (kBC / 8); i += 128) {
+#pragma unroll
+    for (int i = tid; i < kBM * (kBC / 8); i += kThreadsSk) {
       const int row = i >> 3, ch = i & 7;
       const int m = m0 + row;
       const bool ok = m < M;
@@ -143,35 +162,34 @@ __global__ void __launch_bounds__(128) lora_down_kernel(
                  in + static_cast<long long>(ok ? m : 0) * C + c0 + ch * 8, ok);
     }
     if (kWrc) {  // A [r, C]: rows j, 64 contiguous c
-      for (int i = tid; i < R * (kBC / 8); i += 128) {
+      for (int i = tid; i < R * (kBC / 8); i += kThreadsSk) {
         const int j = i >> 3, ch = i & 7;
         cp_async16(&s_w[buf][j * kWLd + ch * 8], w + static_cast<long long>(j) * C + c0 + ch * 8,
                    true);
       }
     } else {  // B [C, r]: rows c, r contiguous
-      for (int i = tid; i < kBC * (R / 8); i += 128) {
+      for (int i = tid; i < kBC * (R / 8); i += kThreadsSk) {
         const int c = i / (R / 8), ch = i % (R / 8);
         cp_async16(&s_w[buf][c * kWLd + ch * 8], w + static_cast<long long>(c0 + c) * R + ch * 8,
                    true);
       }
     }
-    cp_async_commit();
   };
 
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
-  if (sb < se) load(0, sb);
-  for (int st = sb; st < se; ++st) {
-    const int buf = (st - sb) & 1;
-    if (st + 1 < se) {
-      load(buf ^ 1, st + 1);
-      cp_async_wait1();
-    } else {
-      cp_async_wait0();
-    }
+  // Prologue: S-1 slices in flight (empty groups keep the group count uniform).
+#pragma unroll
+  for (int p = 0; p < S - 1; ++p) {
+    if (p < n) load(p, sb + p);
+    cp_async_commit();
+  }
+  for (int i = 0; i < n; ++i) {
+    cp_async_wait_n(S - 2);
     __syncthreads();
+    const int buf = i % S;
 #pragma unroll
     for (int kk = 0; kk < kBC / 16; ++kk) {
       uint32_t a[4];
@@ -181,8 +199,12 @@ __global__ void __launch_bounds__(128) lora_down_kernel(
 #pragma unroll
       for (int t = 0; t < NT; ++t) mma16816(acc[t], a, b[t][0], b[t][1]);
     }
-    __syncthreads();
+    // Refill the slot consumed one iteration ago (every warp has passed this iteration's
+    // barrier, so none still reads it).
+    if (i + S - 1 < n) load((i + S - 1) % S, sb + i + S - 1);
+    cp_async_commit();
   }
+  cp_async_wait0();
 
   const int r_lo = m0 + warp * 16 + (lane >> 2);
 #pragma unroll
@@ -207,73 +229,97 @@ __global__ void __launch_bounds__(128) lora_down_kernel(
   }
 }
 
+// Fixed-order sum of the split partials [split, n] (n = M * r, a multiple of 8): each thread
+// owns 4 consecutive values and issues all of its partial loads before summing, so the kernel
+// costs about one memory round trip.
+constexpr int kMaxSplit = 16;
+
 __global__ void lora_down_finalize(const float* __restrict__ partial, int split, long long n,
                                    float scale, __nv_bfloat16* __restrict__ saved,
                                    __nv_bfloat16* __restrict__ scaled) {
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  float v = 0.f;
-  for (int s = 0; s < split; ++s) v += partial[s * n + i];
-  if (saved) saved[i] = __float2bfloat16_rn(v);
-  scaled[i] = __float2bfloat16_rn(scale * v);
+  const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i4 >= n) return;
+  float4 p[kMaxSplit];
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s)
+    if (s < split) p[s] = __ldg(reinterpret_cast<const float4*>(partial + s * n + i4));
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s)
+    if (s < split) {
+      v.x += p[s].x;
+      v.y += p[s].y;
+      v.z += p[s].z;
+      v.w += p[s].w;
+    }
+  if (saved) {
+    *reinterpret_cast<__nv_bfloat162*>(saved + i4) = __floats2bfloat162_rn(v.x, v.y);
+    *reinterpret_cast<__nv_bfloat162*>(saved + i4 + 2) = __floats2bfloat162_rn(v.z, v.w);
+  }
+  *reinterpret_cast<__nv_bfloat162*>(scaled + i4) = __floats2bfloat162_rn(scale * v.x, scale * v.y);
+  *reinterpret_cast<__nv_bfloat162*>(scaled + i4 + 2) =
+      __floats2bfloat162_rn(scale * v.z, scale * v.w);
 }
 
 // ------------------------------------------------------------------------------------------
-// lora_grad: grid (C/64, split).  4 warps, warp w owns columns c0+16w..c0+16w+15.
+// lora_grad: grid (C/128, split).  8 warps, warp w owns columns c0+16w..c0+16w+15 of `big`;
+// a multi-stage cp.async pipeline streams 64-token slices of `big` and `small`.
 // ------------------------------------------------------------------------------------------
 template <int NT>
-__global__ void __launch_bounds__(128) lora_grad_kernel(
+__global__ void __launch_bounds__(kThreadsSk) lora_grad_kernel(
     const __nv_bfloat16* __restrict__ big, int M, int C, const __nv_bfloat16* __restrict__ small,
     float scale, float* __restrict__ out, int out_cr, float* __restrict__ partial, int split) {
   constexpr int R = NT * 8;
-  constexpr int kBigLd = kBC + kPad;
+  constexpr int S = stages_for(R);
+  constexpr int kBigLd = kGC + kPad;
   constexpr int kSmLd = R + kPad;
   extern __shared__ __align__(16) uint8_t dsm_grad[];
-  auto s_big = reinterpret_cast<__nv_bfloat16(*)[kBM * kBigLd]>(dsm_grad);
-  auto s_sm = reinterpret_cast<__nv_bfloat16(*)[kBM * kSmLd]>(
-      dsm_grad + 2 * kBM * kBigLd * sizeof(__nv_bfloat16));
+  auto s_big = reinterpret_cast<__nv_bfloat16(*)[kGM * kBigLd]>(dsm_grad);
+  auto s_sm = reinterpret_cast<__nv_bfloat16(*)[kGM * kSmLd]>(
+      dsm_grad + S * kGM * kBigLd * sizeof(__nv_bfloat16));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c0 = blockIdx.x * kBC;
-  const int steps = (M + kBM - 1) / kBM;
+  const int c0 = blockIdx.x * kGC;
+  const int steps = (M + kGM - 1) / kGM;
   const int sb = static_cast<int>((static_cast<long long>(steps) * blockIdx.y) / split);
   const int se = static_cast<int>((static_cast<long long>(steps) * (blockIdx.y + 1)) / split);
+  const int n = se - sb;
 
   auto load = [&](int buf, int step) {
-    const int mb = step * kBM;
-    for (int i = tid; i < kBM * (kBC / 8); i += 128) {
-      const int row = i >> 3, ch = i & 7;
+    const int mb = step * kGM;
+#pragma unroll
+    for (int i = tid; i < kGM * (kGC / 8); i += kThreadsSk) {
+      const int row = i / (kGC / 8), ch = i % (kGC / 8);
       const int m = mb + row;
-      const bool ok = m < M;
+      const int c = c0 + ch * 8;  // C is a multiple of 64, so a chunk is all in or all out
+      const bool ok = m < M && c < C;
       cp_async16(&s_big[buf][row * kBigLd + ch * 8],
-                 big + static_cast<long long>(ok ? m : 0) * C + c0 + ch * 8, ok);
+                 big + (ok ? static_cast<long long>(m) * C + c : 0), ok);
     }
-    for (int i = tid; i < kBM * (R / 8); i += 128) {
+    for (int i = tid; i < kGM * (R / 8); i += kThreadsSk) {
       const int row = i / (R / 8), ch = i % (R / 8);
       const int m = mb + row;
       const bool ok = m < M;
       cp_async16(&s_sm[buf][row * kSmLd + ch * 8],
                  small + static_cast<long long>(ok ? m : 0) * R + ch * 8, ok);
     }
-    cp_async_commit();
   };
 
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
-  if (sb < se) load(0, sb);
-  for (int st = sb; st < se; ++st) {
-    const int buf = (st - sb) & 1;
-    if (st + 1 < se) {
-      load(buf ^ 1, st + 1);
-      cp_async_wait1();
-    } else {
-      cp_async_wait0();
-    }
-    __syncthreads();
 #pragma unroll
-    for (int kk = 0; kk < kBM / 16; ++kk) {
+  for (int p = 0; p < S - 1; ++p) {
+    if (p < n) load(p, sb + p);
+    cp_async_commit();
+  }
+  for (int i = 0; i < n; ++i) {
+    cp_async_wait_n(S - 2);
+    __syncthreads();
+    const int buf = i % S;
+#pragma unroll
+    for (int kk = 0; kk < kGM / 16; ++kk) {
       // A = big^T: rows c, k = m; stored [m][c] -> transposed 8x8 loads.
       uint32_t a[4];
       const int q = lane >> 3, i8 = lane & 7;
@@ -283,8 +329,10 @@ __global__ void __launch_bounds__(128) lora_grad_kernel(
 #pragma unroll
       for (int t = 0; t < NT; ++t) mma16816(acc[t], a, b[t][0], b[t][1]);
     }
-    __syncthreads();
+    if (i + S - 1 < n) load((i + S - 1) % S, sb + i + S - 1);
+    cp_async_commit();
   }
+  cp_async_wait0();
 
   const int c_lo = c0 + warp * 16 + (lane >> 2);
 #pragma unroll
@@ -293,6 +341,7 @@ __global__ void __launch_bounds__(128) lora_grad_kernel(
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c = c_lo + h * 8;
+      if (c >= C) continue;
       const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
       if (split == 1) {
         if (out_cr) {
@@ -310,22 +359,38 @@ __global__ void __launch_bounds__(128) lora_grad_kernel(
   }
 }
 
-// Sum split partials [split, C, r] in order; write scale * sum as [C, r] or [r, C].
+// Sum split partials [split, C, r] in order; write scale * sum as [C, r] (out_cr) or [r, C].
+// Each thread owns 4 consecutive outputs and issues all of its partial loads first.
 __global__ void lora_grad_finalize(const float* __restrict__ partial, int split, int C, int R,
                                    float scale, float* __restrict__ out, int out_cr) {
   const long long n = static_cast<long long>(C) * R;
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  long long src;
-  if (out_cr) {
-    src = i;  // i = c * R + j
-  } else {
-    const long long j = i / C, c = i % C;  // i = j * C + c (coalesced writes)
-    src = c * R + j;
+  const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i4 >= n) return;
+  float4 p[kMaxSplit];
+  if (out_cr) {  // i4 = c * R + j: 4 consecutive j of one c
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s)
+      if (s < split) p[s] = __ldg(reinterpret_cast<const float4*>(partial + s * n + i4));
+  } else {       // i4 = j * C + c: 4 consecutive c of one j (coalesced writes)
+    const long long j = i4 / C, c = i4 % C;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s)
+      if (s < split) {
+        const float* q = partial + s * n + c * R + j;
+        p[s] = make_float4(__ldg(q), __ldg(q + R), __ldg(q + 2 * R), __ldg(q + 3 * R));
+      }
   }
-  float v = 0.f;
-  for (int s = 0; s < split; ++s) v += partial[s * n + src];
-  out[i] = scale * v;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s)
+    if (s < split) {
+      v.x += p[s].x;
+      v.y += p[s].y;
+      v.z += p[s].z;
+      v.w += p[s].w;
+    }
+  *reinterpret_cast<float4*>(out + i4) =
+      make_float4(scale * v.x, scale * v.y, scale * v.z, scale * v.w);
 }
 
 int clamp_split(int want, int maxv) { return want < 1 ? 1 : (want > maxv ? maxv : want); }
@@ -333,12 +398,13 @@ int clamp_split(int want, int maxv) { return want < 1 ? 1 : (want > maxv ? maxv 
 size_t down_smem(int R, bool w_rc) {
   const int w_rows = w_rc ? R : kBC;
   const int w_ld = w_rc ? (kBC + kPad) : (R + kPad);
-  return 2 * sizeof(__nv_bfloat16) * (static_cast<size_t>(kBM) * (kBC + kPad) + w_rows * w_ld);
+  return stages_for(R) * sizeof(__nv_bfloat16) *
+         (static_cast<size_t>(kBM) * (kBC + kPad) + static_cast<size_t>(w_rows) * w_ld);
 }
 
 size_t grad_smem(int R) {
-  return 2 * sizeof(__nv_bfloat16) *
-         (static_cast<size_t>(kBM) * (kBC + kPad) + static_cast<size_t>(kBM) * (R + kPad));
+  return stages_for(R) * sizeof(__nv_bfloat16) *
+         (static_cast<size_t>(kGM) * (kGC + kPad) + static_cast<size_t>(kGM) * (R + kPad));
 }
 
 template <typename F>
@@ -351,8 +417,9 @@ cudaError_t launch_dyn(F kernel, dim3 grid, size_t smem, cudaStream_t stream) {
 }  // namespace
 
 DownPlan lora_down_plan(int M, int C, int r) {
-  const int tiles = (M + kBM - 1) / kBM;
-  const int split = clamp_split((kTarget + tiles - 1) / tiles, C / kBC);
+  const int tiles = (M + kBM - 1) / kBM;  // 128-row tiles
+  // As many splits as fit one wave of kTarget CTAs (a partial second wave would double the time).
+  const int split = clamp_split(kTarget / tiles < kMaxSplit ? kTarget / tiles : kMaxSplit, C / kBC);
   DownPlan p;
   p.split = split;
   p.partial_floats = split > 1 ? static_cast<size_t>(split) * M * r : 0;
@@ -360,9 +427,9 @@ DownPlan lora_down_plan(int M, int C, int r) {
 }
 
 GradPlan lora_grad_plan(int M, int C, int r) {
-  const int tiles = C / kBC;
-  const int msteps = (M + kBM - 1) / kBM;
-  const int split = clamp_split((kTarget + tiles - 1) / tiles, msteps);
+  const int tiles = (C + kGC - 1) / kGC;
+  const int msteps = (M + kGM - 1) / kGM;
+  const int split = clamp_split(kTarget / tiles < kMaxSplit ? kTarget / tiles : kMaxSplit, msteps);
   GradPlan p;
   p.split = split;
   p.partial_floats = split > 1 ? static_cast<size_t>(split) * C * r : 0;
@@ -374,12 +441,12 @@ GradPlan lora_grad_plan(int M, int C, int r) {
     if (w_is_rc) {                                                                          \
       e = launch_dyn(lora_down_kernel<NTV, true>, grid, smem, stream);                      \
       if (e != cudaSuccess) return e;                                                       \
-      lora_down_kernel<NTV, true><<<grid, 128, smem, stream>>>(in, M, C, w, scale, saved,   \
+      lora_down_kernel<NTV, true><<<grid, kThreadsSk, smem, stream>>>(in, M, C, w, scale, saved,   \
                                                                scaled, partial, plan.split); \
     } else {                                                                                \
       e = launch_dyn(lora_down_kernel<NTV, false>, grid, smem, stream);                     \
       if (e != cudaSuccess) return e;                                                       \
-      lora_down_kernel<NTV, false><<<grid, 128, smem, stream>>>(in, M, C, w, scale, saved,  \
+      lora_down_kernel<NTV, false><<<grid, kThreadsSk, smem, stream>>>(in, M, C, w, scale, saved,  \
                                                                 scaled, partial, plan.split); \
     }                                                                                       \
     break;
@@ -414,7 +481,7 @@ cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_b
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.split == 1) return e;
   const long long n = static_cast<long long>(M) * r;
-  lora_down_finalize<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+  lora_down_finalize<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
       partial, plan.split, n, scale, saved, scaled);
   return cudaGetLastError();
 }
@@ -424,14 +491,14 @@ cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_b
   case NTV:                                                                                \
     e = launch_dyn(lora_grad_kernel<NTV>, grid, smem, stream);                             \
     if (e != cudaSuccess) return e;                                                        \
-    lora_grad_kernel<NTV><<<grid, 128, smem, stream>>>(big, M, C, small, scale, out,       \
+    lora_grad_kernel<NTV><<<grid, kThreadsSk, smem, stream>>>(big, M, C, small, scale, out,       \
                                                        out_cr ? 1 : 0, partial, plan.split); \
     break;
 
 cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_bfloat16* small,
                              int r, float scale, float* out, bool out_cr, float* partial,
                              const GradPlan& plan, cudaStream_t stream) {
-  dim3 grid(C / kBC, plan.split);
+  dim3 grid((C + kGC - 1) / kGC, plan.split);
   const size_t smem = grad_smem(r);
   cudaError_t e = cudaSuccess;
   switch (r / 8) {
@@ -457,7 +524,7 @@ cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.split == 1) return e;
   const long long n = static_cast<long long>(C) * r;
-  lora_grad_finalize<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+  lora_grad_finalize<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
       partial, plan.split, C, r, scale, out, out_cr ? 1 : 0);
   return cudaGetLastError();
 }
