@@ -260,7 +260,26 @@ def run_e2e(states, steps, dev):
     return a.elapsed_time(b) / steps, h2d, d2h
 
 
-def roofline(states, per_stage, peaks):
+def ncu_traffic(workload, stage):
+    """DRAM bytes per launch of `stage` from the committed ncu capture (profiles/ncu_traffic.json),
+    or None when there is none or the kernel sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(f"{workload}.{stage}")
+        if not rec:
+            return None
+        m = hashlib.sha256()
+        for name in rec["source_files"]:
+            with open(os.path.join(ROOT, name), "rb") as g:
+                m.update(g.read())
+        return rec["traffic_bytes"] if m.hexdigest() == rec["source_sha256"] else None
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+def roofline(states, per_stage, peaks, workload):
     """Roofline of the dominant kernel (largest total time among the stages)."""
     totals = {k: sum(v) for k, v in per_stage.items()}
     name = max(totals, key=totals.get)
@@ -286,7 +305,8 @@ def roofline(states, per_stage, peaks):
         r = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
              "frac": round(ach / peaks["hbm_gbs"], 4)}
     r.update({"kernel": name, "ms_per_launch": round(ms, 5), "flops_per_launch": flops,
-              "bytes_per_launch": byts, "traffic": None, "peak_source": peaks["source"]})
+              "bytes_per_launch": byts, "traffic": ncu_traffic(workload, stage),
+              "peak_source": peaks["source"]})
     return r
 
 
@@ -481,7 +501,7 @@ def main():
             "tflops": round(tflops, 2),
             "tflops_frac_of_peak": round(tflops / peaks["bf16_tflops"], 4),
             "stages_ms": {k: round(statistics.mean(v), 5) for k, v in per_stage.items()},
-            "roofline": roofline(states, per_stage, peaks),
+            "roofline": roofline(states, per_stage, peaks, w.name),
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches),
