@@ -134,7 +134,9 @@ class ClockSampler:
 # Our arm
 # ----------------------------------------------------------------------------------------------
 class LinearState:
-    """Device buffers of one QLoRA linear on M tokens, and its six timed stages."""
+    """Device buffers of one QLoRA linear on M tokens, and its timed stages: forward
+    (lora_down, dequant GEMM) and backward (lora_down, dequant GEMM for dX, lora_grad x 2).
+    X and dY may be buffers shared with other stages (the MLP block chains them)."""
 
     def __init__(self, L, M, X, dY, W0, A, B, dev):
         self.L, self.M = L, M
@@ -153,52 +155,129 @@ class LinearState:
         self.dA = torch.empty((L.r, L.K), dtype=torch.float32, device=dev)
         self.dB = torch.empty((L.N, L.r), dtype=torch.float32, device=dev)
         self.ws = linear.alloc_workspace(M, L.N, L.K, L.r, dev)
-        self.stage_names = ("lora_down_fwd", "gemm_fwd", "lora_down_bwd", "gemm_dx",
-                            "lora_grad_dB", "lora_grad_dA")
 
-    def stages(self, stream):
+    def fwd_stages(self, stream):
         M, L, p = self.M, self.L, lambda t: t.data_ptr()
         ws, wsb = p(self.ws), self.ws.numel()
-        return (
-            lambda: abi.qlora_lora_down(p(self.X), M, L.K, p(self.A), 1, L.r, self.s, p(self.XA),
-                                        p(self.sXA), ws, wsb, stream),
-            lambda: abi.qlora_nf4_gemm(p(self.X), self.cw, 0, p(self.B), p(self.sXA), M, L.r,
-                                       p(self.H), stream),
-            lambda: abi.qlora_lora_down(p(self.dY), M, L.N, p(self.B), 0, L.r, self.s,
-                                        p(self.dYB), p(self.sdYB), ws, wsb, stream),
-            lambda: abi.qlora_nf4_gemm(p(self.dY), self.cw, 1, p(self.A), p(self.sdYB), M, L.r,
-                                       p(self.dX), stream),
-            lambda: abi.qlora_lora_grad(p(self.dY), M, L.N, p(self.XA), L.r, self.s, p(self.dB),
-                                        0, ws, wsb, stream),
-            lambda: abi.qlora_lora_grad(p(self.X), M, L.K, p(self.dYB), L.r, self.s, p(self.dA),
-                                        1, ws, wsb, stream),
-        )
+        n = L.name
+        return [
+            (f"{n}.lora_down_fwd",
+             lambda: abi.qlora_lora_down(p(self.X), M, L.K, p(self.A), 1, L.r, self.s,
+                                         p(self.XA), p(self.sXA), ws, wsb, stream)),
+            (f"{n}.gemm_fwd",
+             lambda: abi.qlora_nf4_gemm(p(self.X), self.cw, 0, p(self.B), p(self.sXA), M, L.r,
+                                        p(self.H), stream)),
+        ]
+
+    def bwd_stages(self, stream):
+        M, L, p = self.M, self.L, lambda t: t.data_ptr()
+        ws, wsb = p(self.ws), self.ws.numel()
+        n = L.name
+        return [
+            (f"{n}.lora_down_bwd",
+             lambda: abi.qlora_lora_down(p(self.dY), M, L.N, p(self.B), 0, L.r, self.s,
+                                         p(self.dYB), p(self.sdYB), ws, wsb, stream)),
+            (f"{n}.gemm_dx",
+             lambda: abi.qlora_nf4_gemm(p(self.dY), self.cw, 1, p(self.A), p(self.sdYB), M, L.r,
+                                        p(self.dX), stream)),
+            (f"{n}.lora_grad_dB",
+             lambda: abi.qlora_lora_grad(p(self.dY), M, L.N, p(self.XA), L.r, self.s,
+                                         p(self.dB), 0, ws, wsb, stream)),
+            (f"{n}.lora_grad_dA",
+             lambda: abi.qlora_lora_grad(p(self.X), M, L.K, p(self.dYB), L.r, self.s,
+                                         p(self.dA), 1, ws, wsb, stream)),
+        ]
 
 
-def build_states(w, dev, seed):
-    inp = synth.make_inputs(w, seed=seed)
-    if w.mlp:
-        raise SystemExit("the MLP workload is benchmarked as its three projections: use "
-                         "--workload mlp_8b_proj")
-    return [LinearState(L, w.M, d["X"], d["dY"], d["W0"], d["A"], d["B"], dev)
-            for L, d in zip(w.linears, inp["linears"])]
+class Step:
+    """One step of a workload: its linears' states and the ordered (name, call) stages."""
+
+    def __init__(self, w, dev, seed):
+        self.w = w
+        inp = synth.make_inputs(w, seed=seed)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        if not w.mlp:
+            self.states = [LinearState(L, w.M, d["X"], d["dY"], d["W0"], d["A"], d["B"], dev)
+                           for L, d in zip(w.linears, inp["linears"])]
+            self.inputs = [(st, "X") for st in self.states] + [(st, "dY") for st in self.states]
+            self.glue = None
+            return
+        # MLP block: gate/up on the shared input X, SwiGLU, down; the backward runs down, the
+        # SwiGLU backward, then up and gate on their output gradients dg, du.
+        gate, up, down = w.linears
+        lg, lu, ld = inp["linears"]
+        X = inp["X"].to(dev)
+        I = gate.N
+        dg = torch.empty((w.M, I), **bf)
+        du = torch.empty((w.M, I), **bf)
+        self.a = torch.empty((w.M, I), **bf)
+        sg = LinearState(gate, w.M, X, dg, lg["W0"], lg["A"], lg["B"], dev)
+        su = LinearState(up, w.M, X, du, lu["W0"], lu["A"], lu["B"], dev)
+        sd = LinearState(down, w.M, self.a, inp["dY"], ld["W0"], ld["A"], ld["B"], dev)
+        su.X = sg.X  # one copy of the block input
+        self.states = [sg, su, sd]
+        self.glue = (sg, su, sd, dg, du)
+        self.inputs = [(sg, "X"), (sd, "dY")]
+
+    def stages(self, stream):
+        if self.glue is None:
+            out = []
+            for st in self.states:
+                out += st.fwd_stages(stream) + st.bwd_stages(stream)
+            return out
+        sg, su, sd, dg, du = self.glue
+        n = self.a.numel()
+        p = lambda t: t.data_ptr()
+        return (sg.fwd_stages(stream) + su.fwd_stages(stream)
+                + [("swiglu.fwd", lambda: abi.qlora_swiglu_fwd(p(sg.H), p(su.H), p(self.a), n,
+                                                               stream))]
+                + sd.fwd_stages(stream) + sd.bwd_stages(stream)
+                + [("swiglu.bwd", lambda: abi.qlora_swiglu_bwd(p(sg.H), p(su.H), p(sd.dX), p(dg),
+                                                               p(du), n, stream))]
+                + su.bwd_stages(stream) + sg.bwd_stages(stream))
+
+    def e2e(self):
+        """One step through the public Python entry points (linear.forward / backward and the
+        SwiGLU glue), on the device buffers already holding this step's inputs."""
+        if self.glue is None:
+            for st in self.states:
+                linear.forward(st.X, st.w, st.A, st.B, st.L.alpha, H=st.H, XA=st.XA, ws=st.ws)
+                linear.backward(st.dY, st.X, st.w, st.A, st.B, st.XA, st.L.alpha, dX=st.dX,
+                                dA=st.dA, dB=st.dB, ws=st.ws)
+            return
+        sg, su, sd, dg, du = self.glue
+        for st in (sg, su):
+            linear.forward(st.X, st.w, st.A, st.B, st.L.alpha, H=st.H, XA=st.XA, ws=st.ws)
+        linear.swiglu_forward(sg.H, su.H, a=self.a)
+        linear.forward(sd.X, sd.w, sd.A, sd.B, sd.L.alpha, H=sd.H, XA=sd.XA, ws=sd.ws)
+        linear.backward(sd.dY, sd.X, sd.w, sd.A, sd.B, sd.XA, sd.L.alpha, dX=sd.dX, dA=sd.dA,
+                        dB=sd.dB, ws=sd.ws)
+        linear.swiglu_backward(sg.H, su.H, sd.dX, dg=dg, du=du)
+        for st in (su, sg):
+            linear.backward(st.dY, st.X, st.w, st.A, st.B, st.XA, st.L.alpha, dX=st.dX,
+                            dA=st.dA, dB=st.dB, ws=st.ws)
+
+    def outputs(self):
+        """Result tensors a user reads back after a step."""
+        if self.glue is None:
+            return [t for st in self.states for t in (st.H, st.dX, st.dA, st.dB)]
+        sg, su, sd, _, _ = self.glue
+        return [sd.H, sg.dX, su.dX] + [t for st in self.states for t in (st.dA, st.dB)]
 
 
-def run_steps(states, n, stream, flush, record):
+def run_steps(step, n, stream, flush, record):
     """Run n steps; per step and per stage, CUDA events on `stream`.  Returns
     (per-step ms list, {stage: [ms...]})."""
     per_step = []
     per_stage = {}
+    calls = step.stages(stream.cuda_stream)
+    events = []
     for _ in range(n):
         # L2 flush: write 256 MiB, then read it back so the evicted lines are clean (the
         # write-back of the flush's own dirty lines must not land on the first timed kernel).
         flush.zero_()
         flush.max()
         evs = []
-        calls = []
-        for st in states:
-            for name, fn in zip(st.stage_names, st.stages(stream.cuda_stream)):
-                calls.append((f"{st.L.name}.{name}", fn))
         for name, fn in calls:
             e = torch.cuda.Event(enable_timing=True)
             e.record(stream)
@@ -208,44 +287,30 @@ def run_steps(states, n, stream, flush, record):
         end.record(stream)
         evs.append(("end", end))
         if record:
-            per_stage.setdefault("_events", []).append(evs)
+            events.append(evs)
     torch.cuda.synchronize()
-    if record:
-        for evs in per_stage.pop("_events"):
-            per_step.append(evs[0][1].elapsed_time(evs[-1][1]))
-            for (name, a), (_, b) in zip(evs[:-1], evs[1:]):
-                per_stage.setdefault(name, []).append(a.elapsed_time(b))
+    for evs in events:
+        per_step.append(evs[0][1].elapsed_time(evs[-1][1]))
+        for (name, a), (_, b) in zip(evs[:-1], evs[1:]):
+            per_stage.setdefault(name, []).append(a.elapsed_time(b))
     return per_step, per_stage
 
 
-def run_e2e(states, steps, dev):
-    """The same metric through the public entry points qlora_linear_fwd / qlora_linear_bwd with
-    host buffers: each step copies X and dY from pinned host memory, runs the layer, and copies
-    h, dX, dA and dB back."""
-    host = []
-    for st in states:
-        host.append({
-            "X": st.X.cpu().pin_memory(), "dY": st.dY.cpu().pin_memory(),
-            "H": torch.empty_like(st.H, device="cpu").pin_memory(),
-            "dX": torch.empty_like(st.dX, device="cpu").pin_memory(),
-            "dA": torch.empty_like(st.dA, device="cpu").pin_memory(),
-            "dB": torch.empty_like(st.dB, device="cpu").pin_memory(),
-        })
-    h2d = sum(h["X"].numel() * 2 + h["dY"].numel() * 2 for h in host)
-    d2h = sum(h["H"].numel() * 2 + h["dX"].numel() * 2 + h["dA"].numel() * 4 + h["dB"].numel() * 4
-              for h in host)
+def run_e2e(step, steps):
+    """The same metric through the public entry points (qlora_linear_fwd / qlora_linear_bwd, and
+    the SwiGLU glue for the MLP block) with host buffers: each step copies the step's inputs
+    from pinned host memory, runs the layer(s), and copies every result back."""
+    ins = [(st, attr, getattr(st, attr).cpu().pin_memory()) for st, attr in step.inputs]
+    outs = [(t, torch.empty_like(t, device="cpu").pin_memory()) for t in step.outputs()]
+    h2d = sum(h.numel() * h.element_size() for _, _, h in ins)
+    d2h = sum(h.numel() * h.element_size() for _, h in outs)
 
     def one():
-        for st, h in zip(states, host):
-            st.X.copy_(h["X"], non_blocking=True)
-            st.dY.copy_(h["dY"], non_blocking=True)
-            linear.forward(st.X, st.w, st.A, st.B, st.L.alpha, H=st.H, XA=st.XA, ws=st.ws)
-            linear.backward(st.dY, st.X, st.w, st.A, st.B, st.XA, st.L.alpha, dX=st.dX,
-                            dA=st.dA, dB=st.dB, ws=st.ws)
-            h["H"].copy_(st.H, non_blocking=True)
-            h["dX"].copy_(st.dX, non_blocking=True)
-            h["dA"].copy_(st.dA, non_blocking=True)
-            h["dB"].copy_(st.dB, non_blocking=True)
+        for st, attr, h in ins:
+            getattr(st, attr).copy_(h, non_blocking=True)
+        step.e2e()
+        for t, h in outs:
+            h.copy_(t, non_blocking=True)
 
     for _ in range(3):
         one()
@@ -279,21 +344,25 @@ def ncu_traffic(workload, stage):
         return None
 
 
-def roofline(states, per_stage, peaks, workload):
+def roofline(step, per_stage, peaks, workload):
     """Roofline of the dominant kernel (largest total time among the stages)."""
     totals = {k: sum(v) for k, v in per_stage.items()}
     name = max(totals, key=totals.get)
     lin_name, stage = name.split(".", 1)
-    st = next(s for s in states if s.L.name == lin_name)
     ms = statistics.mean(per_stage[name])
-    if stage.startswith("gemm"):
-        flops, byts = gemm_work(st.L, st.M, stage == "gemm_dx")
-    elif stage.startswith("lora_down"):
-        C = st.L.K if stage.endswith("fwd") else st.L.N
-        flops, byts = 2.0 * st.M * C * st.L.r, 2 * st.M * C + 4 * st.M * st.L.r
+    if lin_name == "swiglu":
+        n = step.a.numel()
+        flops, byts = 0.0, (3 if stage == "fwd" else 5) * 2 * n
     else:
-        C = st.L.N if stage.endswith("dB") else st.L.K
-        flops, byts = 2.0 * st.M * C * st.L.r, 2 * st.M * C + 4 * C * st.L.r
+        st = next(s for s in step.states if s.L.name == lin_name)
+        if stage.startswith("gemm"):
+            flops, byts = gemm_work(st.L, st.M, stage == "gemm_dx")
+        elif stage.startswith("lora_down"):
+            C = st.L.K if stage.endswith("fwd") else st.L.N
+            flops, byts = 2.0 * st.M * C * st.L.r, 2 * st.M * C + 4 * st.M * st.L.r
+        else:
+            C = st.L.N if stage.endswith("dB") else st.L.K
+            flops, byts = 2.0 * st.M * C * st.L.r, 2 * st.M * C + 4 * C * st.L.r
     ai = flops / byts
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if stage.startswith("gemm") and ai >= ridge:
@@ -313,17 +382,15 @@ def roofline(states, per_stage, peaks, workload):
 # ----------------------------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ----------------------------------------------------------------------------------------------
-def oracle_sample(w, seed, rows_per_linear, threads_note=True):
-    """Time the fp64 oracle: dequantise each W0 once (charged per step: once per batch of M
-    tokens), then forward + backward on `rows_per_linear` sampled token rows.  Returns
-    (seconds for the sample rows, seconds of one dequant per step, description)."""
-    from oracle import nf4, qlora  # test infrastructure: only here and in the reference arm
+def oracle_prepare(w, seed):
+    """Quantise every W0 with the fp64 oracle (not timed) and dequantise it (timed: the
+    dequant is charged once per step, i.e. once per batch of M tokens)."""
+    from oracle import nf4  # test infrastructure: only here and in the reference arm
     inp = synth.make_inputs(w, seed=seed)
     t_deq = 0.0
-    t_rows = 0.0
+    Wds = []
     for L, d in zip(w.linears, inp["linears"]):
         Wf = d["W0"].float().numpy()
-        t0 = time.perf_counter()
         am = nf4.block_absmax(Wf)
         if L.double_quant:
             q8, sc = nf4.double_quant(am.reshape(-1))
@@ -332,23 +399,40 @@ def oracle_sample(w, seed, rows_per_linear, threads_note=True):
             eff = am
         q = nf4.pack_codes(nf4.choose_codes(Wf, eff))
         t1 = time.perf_counter()
-        Wd = nf4.dequantize(q, eff, L.N, L.K).astype(np.float64)
-        t2 = time.perf_counter()
-        t_deq += t2 - t1
-        rows = np.arange(min(rows_per_linear, w.M))
-        X = d["X"][: len(rows)].float().numpy().astype(np.float64)
-        dY = d["dY"][: len(rows)].float().numpy().astype(np.float64)
-        A = d["A"].float().numpy().astype(np.float64)
-        B = d["B"].float().numpy().astype(np.float64)
-        t3 = time.perf_counter()
-        qlora.forward(X, Wd, A, B, L.alpha)
-        qlora.backward(dY, X, Wd, A, B, L.alpha)
-        t_rows += time.perf_counter() - t3
-        del t0
-    desc = (f"fp64 oracle fwd+bwd on {rows_per_linear} token rows per linear of {w.name} "
-            f"(M={w.M}), plus one deq(W0) per step charged per batch of M tokens; "
-            f"quantisation not timed")
-    return t_rows, t_deq, desc
+        Wds.append(nf4.dequantize(q, eff, L.N, L.K).astype(np.float64))
+        t_deq += time.perf_counter() - t1
+    return inp, Wds, t_deq
+
+
+def oracle_rows(w, prep, n):
+    """Seconds the fp64 oracle takes for forward + backward on the first n token rows of the
+    workload (for the MLP block: gate/up, SwiGLU, down, and back)."""
+    from oracle import qlora  # test infrastructure: only here and in the reference arm
+    inp, Wds, _ = prep
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+    lora = [(f64(d["A"]), f64(d["B"])) for d in inp["linears"]]
+    t0 = time.perf_counter()
+    if not w.mlp:
+        for L, d, Wd, (A, B) in zip(w.linears, inp["linears"], Wds, lora):
+            X, dY = f64(d["X"][:n]), f64(d["dY"][:n])
+            qlora.forward(X, Wd, A, B, L.alpha)
+            qlora.backward(dY, X, Wd, A, B, L.alpha)
+    else:
+        (gate, up, down), X, dY = w.linears, f64(inp["X"][:n]), f64(inp["dY"][:n])
+        g, _ = qlora.forward(X, Wds[0], *lora[0], gate.alpha)
+        u, _ = qlora.forward(X, Wds[1], *lora[1], up.alpha)
+        a = qlora.swiglu_forward(g, u)
+        qlora.forward(a, Wds[2], *lora[2], down.alpha)
+        da = qlora.backward(dY, a, Wds[2], *lora[2], down.alpha)["dX"]
+        dg, du = qlora.swiglu_backward(g, u, da)
+        qlora.backward(du, X, Wds[1], *lora[1], up.alpha)
+        qlora.backward(dg, X, Wds[0], *lora[0], gate.alpha)
+    return time.perf_counter() - t0
+
+
+def oracle_desc(w, n):
+    return (f"fp64 oracle fwd+bwd on {n} token rows of {w.name} (M={w.M}), plus one deq(W0) "
+            f"per linear per step charged per batch of M tokens; quantisation not timed")
 
 
 def blas_threads():
@@ -360,11 +444,11 @@ def blas_threads():
 
 
 def cpu_baseline(w, seed=0, rows=32):
-    t_rows, t_deq, desc = oracle_sample(w, seed, rows)
+    prep = oracle_prepare(w, seed)
     n = min(rows, w.M)
-    per_token = t_rows / n + t_deq / w.M
+    per_token = oracle_rows(w, prep, n) / n + prep[2] / w.M
     return {"value": round(1.0 / per_token, 2), "unit": "tokens/s", "cores": blas_threads(),
-            "kind": "oracle", "sample": desc}
+            "kind": "oracle", "sample": oracle_desc(w, n)}
 
 
 def run_reference(args):
@@ -372,18 +456,17 @@ def run_reference(args):
     if rank != 0:
         return
     w = synth.workload(args.workload)
-    # Calibrate: rows per step so the whole run stays within ~2 minutes.
-    t_rows, t_deq, desc = oracle_sample(w, 0, 8)
+    prep = oracle_prepare(w, 0)
+    t_deq = prep[2]
+    # Calibrate: rows per step so the whole run stays within about two minutes.
+    per_row = oracle_rows(w, prep, min(8, w.M)) / min(8, w.M)
     budget = 120.0 / max(1, args.steps + args.warmup)
-    per_row = t_rows / min(8, w.M)
-    rows = int(max(1, min(w.M, (budget - t_deq * 1.0 / max(1, w.M)) / max(per_row, 1e-9))))
+    n = int(max(1, min(w.M, budget / max(per_row, 1e-9))))
     times = []
     for i in range(args.warmup + args.steps):
-        tr, td, desc = oracle_sample(w, 0, rows)
-        n = min(rows, w.M)
+        tr = oracle_rows(w, prep, n)
         if i >= args.warmup:
-            times.append(tr + td * n / w.M)
-    n = min(rows, w.M)
+            times.append(tr + t_deq * n / w.M)
     tot = sum(times)
     value = args.steps * n / tot
     line = {
@@ -393,7 +476,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(),
-                         "kind": "oracle", "sample": desc.replace("32", str(n))},
+                         "kind": "oracle", "sample": oracle_desc(w, n)},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -440,12 +523,12 @@ def main():
                                 device_id=dev)
 
     w = synth.workload(args.workload)
-    states = build_states(w, dev, seed=rank)
+    step = Step(w, dev, seed=rank)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
 
-    run_steps(states, args.warmup, stream, flush, record=False)
+    run_steps(step, args.warmup, stream, flush, record=False)
     if abi.qlora_device_error() != 0:
         raise SystemExit("device error word set during warm-up")
 
@@ -457,7 +540,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     n0 = abi.qlora_launch_counter()
-    per_step, per_stage = run_steps(states, args.steps, stream, flush, record=True)
+    per_step, per_stage = run_steps(step, args.steps, stream, flush, record=True)
     torch.cuda.synchronize()
     launches = abi.qlora_launch_counter() - n0
     if dist:
@@ -475,7 +558,7 @@ def main():
     value = tokens / (total_ms * 1e-3)
     ms_per_step = total_ms / args.steps
 
-    e2e_ms, h2d, d2h = run_e2e(states, args.e2e_steps, dev)
+    e2e_ms, h2d, d2h = run_e2e(step, args.e2e_steps)
     te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if dist:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
@@ -501,7 +584,7 @@ def main():
             "tflops": round(tflops, 2),
             "tflops_frac_of_peak": round(tflops / peaks["bf16_tflops"], 4),
             "stages_ms": {k: round(statistics.mean(v), 5) for k, v in per_stage.items()},
-            "roofline": roofline(states, per_stage, peaks, w.name),
+            "roofline": roofline(step, per_stage, peaks, w.name),
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches),

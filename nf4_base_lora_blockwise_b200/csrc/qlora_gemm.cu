@@ -38,6 +38,9 @@
 // out of order; so every ring slot has exactly one producer and one consumer that each visit
 // its uses in order: W slots 2g, 2g+1 and Q slots 4g..4g+3 belong to dequant group g (the MMA,
 // resp. the Q producer, is the other side), and the X ring has one producer and one consumer.
+// A slot that threads read with ordinary loads and TMA then refills (the Q ring) needs a
+// generic -> async proxy fence between the reads and the release of the slot; without it the
+// refill was seen to overwrite codes not yet read, at large grids and long reductions.
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -436,6 +439,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!failed) failed = !mbar_wait_warp(qfull + qslot, qpar, kErrWaitFull, err, it);
         if (!failed) {
           const uint4 q4 = *reinterpret_cast<const uint4*>(QS(qslot) + q_off);
+          // The slot's next fill is a TMA write (async proxy): order this generic read before
+          // it, or the refill can overwrite the codes before the read has taken them.
+          fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(qempty + qslot);
           Nf4Lut lut;

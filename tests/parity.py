@@ -22,9 +22,11 @@ def bits(t):
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def oracle_pack(W_bf16_cpu, dq, rows=None):
+def oracle_pack(W_bf16_cpu, dq, rows=None, chunk=2048):
     """Oracle quantisation of W0.  With ``rows``, codes are produced for those rows only
-    (absmax and the double-quant groups always cover the whole weight)."""
+    (absmax and the double-quant groups always cover the whole weight).  Rows are independent
+    once the effective absmax is known, so codes are computed ``chunk`` rows at a time to bound
+    host memory (the arithmetic is unchanged)."""
     w = f32(W_bf16_cpu)
     N, K = w.shape
     am = nf4.block_absmax(w)
@@ -38,7 +40,30 @@ def oracle_pack(W_bf16_cpu, dq, rows=None):
     out["absmax_eff"] = eff
     sel = np.arange(N) if rows is None else np.asarray(rows)
     out["rows"] = sel
-    out["q"] = nf4.pack_codes(nf4.choose_codes(w[sel], eff[sel]))
+    q = np.empty((len(sel), K // 2), np.uint8)
+    for c in range(0, len(sel), chunk):
+        r = sel[c:c + chunk]
+        q[c:c + chunk] = nf4.pack_codes(nf4.choose_codes(w[r], eff[r]))
+    out["q"] = q
+    return out
+
+
+def oracle_dequant(ref, chunk=2048):
+    """deq(W0) as float32 (bf16-exact) for the rows in ``ref`` (row chunks bound memory)."""
+    q, eff, rows = ref["q"], ref["absmax_eff"], ref["rows"]
+    K = q.shape[1] * 2
+    out = np.empty((len(rows), K), np.float32)
+    for c in range(0, len(rows), chunk):
+        r = rows[c:c + chunk]
+        out[c:c + chunk] = nf4.dequantize(q[c:c + chunk], eff[r], len(r), K)
+    return out
+
+
+def subset(ref, rows):
+    """A copy of a full-weight oracle pack restricted to the given weight rows."""
+    out = dict(ref)
+    out["rows"] = np.asarray(rows)
+    out["q"] = ref["q"][np.asarray(rows)]
     return out
 
 

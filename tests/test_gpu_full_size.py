@@ -1,0 +1,181 @@
+"""GPU parity at the benchmark's full sizes, in the launch configuration bench.py times.
+
+Every workload the benchmark runs is checked here on the same seeded inputs:
+
+* NF4 codes, absmax (and the double-quant codes / scales) and the dequantised weight:
+  bit-exact, on a fixed sample of weight rows (absmax and the double-quant groups are checked in
+  full).
+* h and dX: on a fixed seeded sample of 512 token rows plus the first and last, every column.
+* XA, dA and dB: in full.
+
+The floating-point bar is max|err| / max|ref| <= 2e-2.  The oracle computes the sampled rows in
+float64 (its products are chunked over output columns only to bound host memory).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import parity
+from nf4_base_lora_blockwise_b200 import linear, synth
+from oracle import nf4, qlora
+
+pytestmark = pytest.mark.gpu
+
+W_ROWS = 96  # weight rows whose codes / dequantised values are compared bit for bit
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _weight_rows(N, seed=7):
+    g = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, N - 1], g.choice(N, W_ROWS, replace=False)]))
+    return rows
+
+
+def _rows_matmul(Xr, Wd_f32, chunk=2048):
+    """Xr [m, K] float64 times Wd^T (Wd [N, K] float32, bf16-exact) -> [m, N] float64."""
+    N = Wd_f32.shape[0]
+    out = np.empty((Xr.shape[0], N))
+    for c in range(0, N, chunk):
+        out[:, c:c + chunk] = Xr @ Wd_f32[c:c + chunk].astype(np.float64).T
+    return out
+
+
+def _rows_matmul_t(Yr, Wd_f32, chunk=2048):
+    """Yr [m, N] float64 times Wd (Wd [N, K]) -> [m, K] float64."""
+    K = Wd_f32.shape[1]
+    out = np.empty((Yr.shape[0], K))
+    for c in range(0, K, chunk):
+        out[:, c:c + chunk] = Yr @ Wd_f32[:, c:c + chunk].astype(np.float64)
+    return out
+
+
+def check_one_linear(X_cpu, dY_cpu, lin, L, tag):
+    X, dY = X_cpu.cuda(), dY_cpu.cuda()
+    A, B = lin["A"].cuda(), lin["B"].cuda()
+    w = linear.nf4_pack(lin["W0"].cuda(), double_quant=L.double_quant)
+    H, XA = linear.forward(X, w, A, B, L.alpha)
+    dX, dA, dB = linear.backward(dY, X, w, A, B, XA, L.alpha)
+    torch.cuda.synchronize()
+    assert linear.device_error() == 0
+
+    # --- NF4 storage: bit-exact on sampled weight rows, absmax / DQ arrays in full.
+    full = parity.oracle_pack(lin["W0"], L.double_quant)
+    parity.check_pack(w, parity.subset(full, _weight_rows(L.N)), L.double_quant)
+    del w
+
+    # --- Oracle on sampled token rows, in float64.
+    M = X_cpu.shape[0]
+    rows = synth.sample_rows(M).numpy()
+    Wd = parity.oracle_dequant(full)          # float32, bf16-exact, all rows
+    del full
+    Xf = parity.f32(X_cpu)
+    dYf = parity.f32(dY_cpu)
+    Af = parity.f32(lin["A"]).astype(np.float64)
+    Bf = parity.f32(lin["B"]).astype(np.float64)
+    s = L.alpha / L.r
+    Xr = Xf[rows].astype(np.float64)
+    dYr = dYf[rows].astype(np.float64)
+    h_ref = _rows_matmul(Xr, Wd) + s * ((Xr @ Af.T) @ Bf.T)
+    dx_ref = _rows_matmul_t(dYr, Wd) + s * ((dYr @ Bf) @ Af)
+    wts = qlora.backward_weights(dYf, Xf, Af, Bf, L.alpha)
+    errs = {
+        "h": qlora.rel_err(parity.f32(H)[rows], h_ref),
+        "dX": qlora.rel_err(parity.f32(dX)[rows], dx_ref),
+        "XA": qlora.rel_err(parity.f32(XA), wts["XA"]),
+        "dA": qlora.rel_err(parity.f32(dA), wts["dA"]),
+        "dB": qlora.rel_err(parity.f32(dB), wts["dB"]),
+    }
+    for k, v in errs.items():
+        assert v <= parity.TOL, f"{tag} {k}: {v:.3e}"
+    return errs, H, dX
+
+
+@pytest.mark.parametrize("name", ["q_proj_8b", "proj_70b_dq", "sweep_m1", "sweep_m16",
+                                  "sweep_m128", "sweep_m16384"])
+def test_full_size_workload(name):
+    w = synth.workload(name)
+    inp = synth.make_inputs(w, seed=0)
+    for L, lin in zip(w.linears, inp["linears"]):
+        check_one_linear(lin["X"], lin["dY"], lin, L, f"{name}/{L.name}")
+
+
+def test_full_size_mlp():
+    """The MLP workload: gate/up 4096->14336, SwiGLU, down 14336->4096 on 8192 tokens.  Each
+    linear is checked at full size on its actual input (down's input is the GPU's SwiGLU output;
+    the SwiGLU itself is checked elementwise on the sampled rows)."""
+    w = synth.workload("mlp_8b")
+    inp = synth.make_inputs(w, seed=0)
+    gate, up, down = w.linears
+    lg, lu, ld = inp["linears"]
+    X = inp["X"]
+    rows = synth.sample_rows(w.M).numpy()
+    # Upstream gradients of gate and up: seeded stand-ins with the recipe's spread.
+    _, Hg, _ = check_one_linear(X, _grad_like(w.M, gate.N, 1), lg, gate, "mlp/gate")
+    _, Hu, _ = check_one_linear(X, _grad_like(w.M, up.N, 2), lu, up, "mlp/up")
+    a = linear.swiglu_forward(Hg, Hu)
+    torch.cuda.synchronize()
+    ref_a = qlora.swiglu_forward(parity.f32(Hg)[rows], parity.f32(Hu)[rows])
+    assert qlora.rel_err(parity.f32(a)[rows], ref_a) <= 1e-2
+    check_one_linear(a.cpu(), inp["dY"], ld, down, "mlp/down")
+
+
+def _grad_like(M, N, seed):
+    g = torch.Generator().manual_seed(1000 + seed)
+    return (torch.randn((M, N), generator=g) * 1e-2).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 14336), (14336, 4096)])
+def test_one_hot_products_reproduce_the_weight(K, N):
+    """With one-hot activations each output row of the dequant GEMM is one row (dX) or one
+    column (forward) of deq(W0), exactly: one product by 1.0 accumulated in fp32 and rounded to
+    bf16 is the bf16 weight itself, so every element must equal the oracle's dequantised weight
+    exactly (compared as values: the sign of a zero is left to the tensor core's adder).  Three repeats at a full grid and a 64-step reduction: every pipeline
+    slot is reused many times, so a slot refilled before its reads finished shows up as wrong
+    bits here (the LoRA extension input is zero and contributes nothing)."""
+    from nf4_base_lora_blockwise_b200 import abi
+
+    inp, L = parity.make(4, K, N, 16, seed=K + 3 * N)
+    W0 = inp["linears"][0]["W0"]
+    ref = parity.oracle_pack(W0, False)
+    ref_w = nf4.dequantize(ref["q"], ref["absmax_eff"], N, K)      # [N, K] float32, bf16 values
+    w = linear.nf4_pack(W0.cuda())
+    cw = w.c_struct()
+    r = 16
+    A = torch.zeros((r, K), dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros((N, r), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def one_hot(M, C):
+        t = torch.zeros((M, C), dtype=torch.bfloat16, device="cuda")
+        m = torch.arange(M, device="cuda")
+        t[m, m % C] = 1.0
+        return t
+
+    # dX[m, :] = deq(W0)[m % N, :]
+    dY = one_hot(N, N)
+    zero = torch.zeros((N, r), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        dX = torch.full((N, K), float("nan"), dtype=torch.bfloat16, device="cuda")
+        abi.qlora_nf4_gemm(dY.data_ptr(), cw, 1, A.data_ptr(), zero.data_ptr(), N, r,
+                           dX.data_ptr(), stream)
+        torch.cuda.synchronize()
+        assert linear.device_error() == 0
+        bad = int((parity.f32(dX) != ref_w).sum())
+        assert bad == 0, f"dX: {bad} elements differ from deq(W0) rows"
+    # h[m, :] = deq(W0)[:, m % K]
+    X = one_hot(K, K)
+    zero = torch.zeros((K, r), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        H = torch.full((K, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        abi.qlora_nf4_gemm(X.data_ptr(), cw, 0, B.data_ptr(), zero.data_ptr(), K, r,
+                           H.data_ptr(), stream)
+        torch.cuda.synchronize()
+        assert linear.device_error() == 0
+        bad = int((parity.f32(H) != ref_w.T).sum())
+        assert bad == 0, f"h: {bad} elements differ from deq(W0) columns"
