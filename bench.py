@@ -10,9 +10,13 @@ batch of synthetic tokens (seeded, resident in HBM before timing):
     dYB = dY B, dX = dY deq(W0) + s dYB A, dB, dA          (backward)
 
 run as the six library stages (lora_down, dequant GEMM, lora_down, dequant GEMM (dX),
-lora_grad x 2) with CUDA events between them on the launching stream, so the dominant
-kernel's own duration is measured live.  L2 is flushed before every step, outside the events:
-a 256 MiB write followed by a read of the same buffer, so no dirty line is left to write back.  One JSON line is printed by rank 0.
+lora_grad x 2; the MLP block adds the SwiGLU glue between its three linears).  The step is
+captured once into a CUDA graph with timing events between the stages (recorded by the graph
+on its own stream), and each timed step is one replay, so the dominant kernel's own duration
+is measured live and host launch cost never appears as idle time (--eager launches every stage
+from Python instead).  L2 is flushed before every step, outside the events: a 256 MiB write
+followed by a read of the same buffer, so no dirty line is left to write back.  One JSON line
+is printed by rank 0.
 
 Multi-GPU (torchrun): every rank runs an independent replica on its own batch (the layer's
 data path has no exchange step in one forward+backward); the step time is the max over ranks.
@@ -166,7 +170,7 @@ class LinearState:
                                          p(self.XA), p(self.sXA), ws, wsb, stream)),
             (f"{n}.gemm_fwd",
              lambda: abi.qlora_nf4_gemm(p(self.X), self.cw, 0, p(self.B), p(self.sXA), M, L.r,
-                                        p(self.H), stream)),
+                                        p(self.H), ws, wsb, stream)),
         ]
 
     def bwd_stages(self, stream):
@@ -179,7 +183,7 @@ class LinearState:
                                          p(self.dYB), p(self.sdYB), ws, wsb, stream)),
             (f"{n}.gemm_dx",
              lambda: abi.qlora_nf4_gemm(p(self.dY), self.cw, 1, p(self.A), p(self.sdYB), M, L.r,
-                                        p(self.dX), stream)),
+                                        p(self.dX), ws, wsb, stream)),
             (f"{n}.lora_grad_dB",
              lambda: abi.qlora_lora_grad(p(self.dY), M, L.N, p(self.XA), L.r, self.s,
                                          p(self.dB), 0, ws, wsb, stream)),
@@ -266,8 +270,8 @@ class Step:
 
 
 def run_steps(step, n, stream, flush, record):
-    """Run n steps; per step and per stage, CUDA events on `stream`.  Returns
-    (per-step ms list, {stage: [ms...]})."""
+    """Eager mode: run n steps, each stage launched from Python, CUDA events on `stream`
+    between the stages.  Returns (per-step ms list, {stage: [ms...]})."""
     per_step = []
     per_stage = {}
     calls = step.stages(stream.cuda_stream)
@@ -294,6 +298,41 @@ def run_steps(step, n, stream, flush, record):
         for (name, a), (_, b) in zip(evs[:-1], evs[1:]):
             per_stage.setdefault(name, []).append(a.elapsed_time(b))
     return per_step, per_stage
+
+
+class GraphStep:
+    """The whole step captured once into a CUDA graph, with timing events (recorded by the
+    graph itself) between the stages, so host-side launch cost never shows up as idle time
+    between kernels.  Each replay is preceded by the L2 flush (outside the graph) and
+    followed by a synchronize to read that replay's events."""
+
+    def __init__(self, step):
+        side = torch.cuda.Stream()
+        calls = step.stages(side.cuda_stream)
+        self.names = [name for name, _ in calls]
+        self.evs = [torch.cuda.Event(enable_timing=True, external=True)
+                    for _ in range(len(calls) + 1)]
+        self.graph = torch.cuda.CUDAGraph()
+        n0 = abi.qlora_launch_counter()
+        with torch.cuda.graph(self.graph, stream=side, capture_error_mode="relaxed"):
+            for (_, fn), e in zip(calls, self.evs):
+                e.record()
+                fn()
+            self.evs[-1].record()
+        self.launches_per_step = abi.qlora_launch_counter() - n0
+
+    def run(self, n, flush, record):
+        per_step, per_stage = [], {}
+        for _ in range(n):
+            flush.zero_()
+            flush.max()
+            self.graph.replay()
+            torch.cuda.synchronize()
+            if record:
+                per_step.append(self.evs[0].elapsed_time(self.evs[-1]))
+                for name, a, b in zip(self.names, self.evs[:-1], self.evs[1:]):
+                    per_stage.setdefault(name, []).append(a.elapsed_time(b))
+        return per_step, per_stage
 
 
 def run_e2e(step, steps):
@@ -502,6 +541,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every stage from Python instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -531,6 +572,16 @@ def main():
     run_steps(step, args.warmup, stream, flush, record=False)
     if abi.qlora_device_error() != 0:
         raise SystemExit("device error word set during warm-up")
+    graph = None
+    if not args.eager:
+        try:
+            graph = GraphStep(step)
+            graph.run(3, flush, record=True)
+        except Exception as exc:  # a runtime without timing events in graphs: time eagerly
+            print(f"CUDA graph timing unavailable ({exc}); timing eager launches",
+                  file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
     if not args.no_clocks and rank == 0:
@@ -540,9 +591,13 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     n0 = abi.qlora_launch_counter()
-    per_step, per_stage = run_steps(step, args.steps, stream, flush, record=True)
-    torch.cuda.synchronize()
-    launches = abi.qlora_launch_counter() - n0
+    if graph is not None:
+        per_step, per_stage = graph.run(args.steps, flush, record=True)
+        launches = graph.launches_per_step * args.steps
+    else:
+        per_step, per_stage = run_steps(step, args.steps, stream, flush, record=True)
+        torch.cuda.synchronize()
+        launches = abi.qlora_launch_counter() - n0
     if dist:
         dist.barrier()
     clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
@@ -588,6 +643,7 @@ def main():
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches),
+            "launch_mode": "cuda_graph" if graph is not None else "eager",
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -105,7 +105,8 @@ QLORA_API qlora_status qlora_nf4_pack(const void* W, int N, int K, int double_qu
 QLORA_API qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, qlora_stream_t stream);
 
 /* Scratch bytes the linear entry points need for (M, N, K, r): the scaled rank-r
- * activations and the fixed-order split partials of the rank-r reductions. */
+ * activations, the fixed-order split partials of the rank-r reductions and the stream-K
+ * partial sums of the dequant GEMM (sized for any device of up to 160 SMs).  Needs no GPU. */
 QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
 
 /* Forward.  X [M, K], A [r, K], B [N, r] bf16 device (read); H [M, N] bf16 device (written);
@@ -144,14 +145,18 @@ QLORA_API qlora_status qlora_lora_down(const void* in, int M, int C, const void*
                                        void* scaled, void* ws, size_t ws_bytes,
                                        qlora_stream_t stream);
 
-/* The dequant GEMM with the fused rank-r extension (no workspace):
+/* The dequant GEMM with the fused rank-r extension:
  *   transpose_w = 0: out[M, N] = act[M, K] . deq(W0)^T + ext_act[M, r] . ext_w^T, ext_w = B [N, r]
  *   transpose_w = 1: out[M, K] = act[M, N] . deq(W0)   + ext_act[M, r] . ext_w,   ext_w = A [r, K]
  * act, ext_w, ext_act bf16 device (read); out bf16 device (written).  The scale s is expected
- * to be folded into ext_act already (qlora_lora_down's `scaled` output). */
+ * to be folded into ext_act already (qlora_lora_down's `scaled` output).
+ * ws: device scratch for the partial sums of problems with fewer output tiles (128 output
+ * features x up to 512 tokens) than SMs, which are cut along the reduction so every SM works;
+ * at least qlora_workspace_bytes(M, N, K, r) bytes (may be NULL when that shape needs none). */
 QLORA_API qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
                                       const void* ext_w, const void* ext_act, int M, int r,
-                                      void* out, qlora_stream_t stream);
+                                      void* out, void* ws, size_t ws_bytes,
+                                      qlora_stream_t stream);
 
 /* Rank-r weight gradient: G[c, j] = scale * sum_m big[m, c] small[m, j] with big [M, C] and
  * small [M, r] bf16 device; written fp32 as out [C, r] (out_r_by_c = 0, e.g. dB) or

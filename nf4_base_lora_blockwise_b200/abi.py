@@ -85,7 +85,7 @@ def _lib():
             "qlora_swiglu_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _VP]),
             "qlora_lora_down": (_I, [_VP, _I, _I, _VP, _I, _I, _F, _VP, _VP, _VP, _SZ, _VP]),
             "qlora_nf4_gemm": (_I, [_VP, ctypes.POINTER(Nf4Weight), _I, _VP, _VP, _I, _I, _VP,
-                                    _VP]),
+                                    _VP, _SZ, _VP]),
             "qlora_lora_grad": (_I, [_VP, _I, _I, _VP, _I, _F, _VP, _I, _VP, _SZ, _VP]),
             "qlora_launch_counter": (ctypes.c_uint64, []),
             "qlora_linear_fwd_noalloc": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _I, _I,
@@ -158,9 +158,10 @@ def qlora_lora_down(inp, M, C, w, w_is_r_by_c, r, scale, saved, scaled, ws, ws_b
                                                      stream))
 
 
-def qlora_nf4_gemm(act, weight, transpose_w, ext_w, ext_act, M, r, out, stream):
+def qlora_nf4_gemm(act, weight, transpose_w, ext_w, ext_act, M, r, out, ws, ws_bytes, stream):
     _check("qlora_nf4_gemm", _lib().qlora_nf4_gemm(act, ctypes.byref(weight), int(transpose_w),
-                                                   ext_w, ext_act, M, r, out, stream))
+                                                   ext_w, ext_act, M, r, out, ws, ws_bytes,
+                                                   stream))
 
 
 def qlora_lora_grad(big, M, C, small, r, scale, out, out_r_by_c, ws, ws_bytes, stream):

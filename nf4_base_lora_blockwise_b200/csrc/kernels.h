@@ -39,7 +39,9 @@ struct GemmArgs {
   const uint8_t* absmax_q8;
   const float* absmax_scale;
   __nv_bfloat16* out;
-  int* err;  // device error word
+  int* err;        // device error word
+  float* partial;  // stream-K partial sums [grid][2][tile tokens][128] fp32 (workspace)
+  int streamk;     // set by the launcher
   Codebook cb;
 };
 
@@ -50,12 +52,28 @@ struct GemmMaps {
   CUtensorMap ext_act;  // scaled rank-r activation [M, r] bf16, box {64, bt}
 };
 
+// Work schedule of one launch: whole tiles (one CTA per tile, at most one per SM) or, with
+// fewer tiles than SMs, stream-K over one CTA per SM (up to kGemmMaxCtas) plus a finalize
+// kernel that adds the partial sums of cut tiles.
+constexpr int kGemmMaxCtas = 160;
+struct GemmSchedule {
+  int n_tiles;
+  int streamk;
+  int grid;
+  size_t partial_floats;  // workspace the stream-K partials need
+};
+GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count);
+// Partial-sum bytes any device (at most kGemmMaxCtas SMs) may need for this shape.
+size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile);
+
 int gemm_pick_bt(int M);
 int gemm_pick_halves(int M);
 int gemm_pick_stages(int bt);
 size_t gemm_smem_bytes(int bt, int nh);
-cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, const GemmArgs& args,
-                              cudaStream_t stream);
+// Falls back to whole tiles when stream-K is chosen but `partial` is null or smaller than the
+// schedule needs (partial_floats_avail).  *launched = kernels enqueued (1, or 2 with stream-K).
+cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
+                              size_t partial_floats_avail, cudaStream_t stream, int* launched);
 
 // ------------------------------ rank-r skinny products (mma.sync) --------------------------
 // out[m, j] = sum_c in[m, c] * Wl(j, c); Wl(j, c) = w[j * C + c] (w_is_rc = true, i.e. A [r, C])

@@ -109,18 +109,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int si
   }
 }
 
-// Warp-wide bounded wait: lane 0 polls (so a waiting warp costs one lane's polling, not 32),
-// then every lane takes the completed phase itself with one more try_wait (acquire per thread).
+// Warp-wide bounded wait: lane 0 alone polls the barrier (its try_wait has acquire semantics)
+// and __syncwarp, which orders memory among the warp's lanes, passes that ordering on to the
+// other 31.  One barrier operation per warp instead of 32: with a dozen warps waiting every
+// pipeline step, per-lane polling saturates the shared-memory barrier unit and slows every
+// barrier operation in the CTA, the MMA issuer's included.
 // Must be called by all 32 lanes; returns a warp-uniform result.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int site,
                                                int* err, int tag = 0) {
   bool ok = true;
   if ((threadIdx.x & 31u) == 0u) ok = mbar_wait(bar, parity, site, err, tag);
   ok = __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
-  if (ok) {
-    for (int i = 0; i < 64 && !mbar_try_wait(bar, parity); ++i) {
-    }
-  }
+  __syncwarp();
   return ok;
 }
 

@@ -150,31 +150,41 @@ qlora_status check_weight(const qlora_nf4_weight* W) {
 
 bool rank_ok(int r) { return r >= 8 && r <= 128 && (r % 8) == 0; }
 
+int ext_steps(int r) { return ((r + 15) / 16 * 16 + 63) / 64; }
+
+// Stream-K partial-sum bytes of the forward (rows N, K/64 steps) or dX (rows K, N/64 steps).
+size_t gemm_ws_bytes(int M, int N, int K, int r, bool trans) {
+  return trans ? gemm_partial_bytes_bound(M, K, N / 64 + ext_steps(r))
+               : gemm_partial_bytes_bound(M, N, K / 64 + ext_steps(r));
+}
+
 // ---------------------------------------------------------------------------------------------
 // Workspace layout (each region 256-byte aligned):
-//   [0]  small0  bf16 [M, r]   s*XA (forward) / dYB (backward)
-//   [1]  small1  bf16 [M, r]   s*dYB (backward)
-//   [2]  down    fp32 split partials of the rank-r down-projection
-//   [3]  grad    fp32 split partials of dB / dA (used one after the other)
+//   [0]  small0   bf16 [M, r]   s*XA (forward) / dYB (backward)
+//   [1]  small1   bf16 [M, r]   s*dYB (backward)
+//   [2]  scratch  fp32 partial sums, written and read within one stage: the split partials of
+//                 the rank-r down-projection, the stream-K partials of the dequant GEMM, then
+//                 the split partials of dB and dA (stages run one after another on the stream)
 // ---------------------------------------------------------------------------------------------
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-  size_t small0, small1, down, grad, total;
+  size_t small0, small1, scratch, scratch_bytes, total;
 };
 
 WsLayout ws_layout(int M, int N, int K, int r) {
   WsLayout L;
   const size_t small = align256(static_cast<size_t>(M) * r * 2);
-  const size_t down = align256(4 * std::max(lora_down_plan(M, K, r).partial_floats,
-                                            lora_down_plan(M, N, r).partial_floats));
-  const size_t grad = align256(4 * std::max(lora_grad_plan(M, N, r).partial_floats,
-                                            lora_grad_plan(M, K, r).partial_floats));
+  const size_t down = 4 * std::max(lora_down_plan(M, K, r).partial_floats,
+                                   lora_down_plan(M, N, r).partial_floats);
+  const size_t grad = 4 * std::max(lora_grad_plan(M, N, r).partial_floats,
+                                   lora_grad_plan(M, K, r).partial_floats);
+  const size_t gemm = std::max(gemm_ws_bytes(M, N, K, r, false), gemm_ws_bytes(M, N, K, r, true));
   L.small0 = 0;
   L.small1 = small;
-  L.down = 2 * small;
-  L.grad = L.down + down;
-  L.total = L.grad + grad;
+  L.scratch = 2 * small;
+  L.scratch_bytes = align256(std::max(std::max(down, grad), gemm));
+  L.total = L.scratch + L.scratch_bytes;
   return L;
 }
 
@@ -196,6 +206,8 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, bool trans, void* ou
   a.absmax_scale = W->absmax_scale;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
+  a.partial = nullptr;
+  a.streamk = 0;
   a.cb = codebook();
   return a;
 }
@@ -247,15 +259,20 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
   return QLORA_OK;
 }
 
+// `partial` / `partial_bytes`: scratch for the stream-K partial sums (whole tiles if too small).
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
-                     const void* ext_act, int M, int r, void* out, int* err, cudaStream_t s) {
+                     const void* ext_act, int M, int r, void* out, int* err, void* partial,
+                     size_t partial_bytes, cudaStream_t s) {
   GemmArgs a = gemm_args(W, M, r, trans, out, err);
+  a.partial = static_cast<float*>(partial);
   GemmMaps maps;
   qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, a.bt);
   if (st != QLORA_OK) return st;
-  if (launch_qlora_gemm(trans, maps, a, s) != cudaSuccess) return QLORA_ERR_CUDA;
-  count(1);
-  return QLORA_OK;
+  int launched = 0;
+  const cudaError_t e = launch_qlora_gemm(trans, maps, a, partial ? partial_bytes / 4 : 0, s,
+                                          &launched);
+  count(launched);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int r, float scale,
@@ -389,10 +406,10 @@ qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const vo
 
   // XA = X A^T (saved, bf16) and s * XA (the scaled operand of the fused up-projection).
   st = do_lora_down(X, M, W->K, A, true, r, scale, XA_saved, sxa,
-                    reinterpret_cast<float*>(w8 + L.down), s);
+                    reinterpret_cast<float*>(w8 + L.scratch), s);
   if (st != QLORA_OK) return st;
   // h = X deq(W0)^T + (s XA) B^T.
-  return do_gemm(X, W, false, B, sxa, M, r, H, err, s);
+  return do_gemm(X, W, false, B, sxa, M, r, H, err, w8 + L.scratch, L.scratch_bytes, s);
 }
 
 qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
@@ -417,19 +434,20 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_wei
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   auto* dyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
   auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
-  float* grad_part = reinterpret_cast<float*>(w8 + L.grad);
+  float* scratch = reinterpret_cast<float*>(w8 + L.scratch);
   const float scale = alpha / static_cast<float>(r);
 
   // dYB = dY B (bf16, for dA) and s * dYB (operand of the fused dX up-projection).
-  st = do_lora_down(dY, M, W->N, B, false, r, scale, dyb, sdyb,
-                    reinterpret_cast<float*>(w8 + L.down), s);
+  st = do_lora_down(dY, M, W->N, B, false, r, scale, dyb, sdyb, scratch, s);
   if (st != QLORA_OK) return st;
   // dX = dY deq(W0) + (s dYB) A.
-  if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, r, dX, err, s)) != QLORA_OK) return st;
+  if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, r, dX, err, scratch, L.scratch_bytes, s)) !=
+                QLORA_OK)
+    return st;
   // dB = s dY^T XA  [N, r];  dA = s dYB^T X  [r, K].
-  st = do_lora_grad(dY, M, W->N, XA_saved, r, scale, dB, true, grad_part, s);
+  st = do_lora_grad(dY, M, W->N, XA_saved, r, scale, dB, true, scratch, s);
   if (st != QLORA_OK) return st;
-  return do_lora_grad(X, M, W->K, dyb, r, scale, dA, false, grad_part, s);
+  return do_lora_grad(X, M, W->K, dyb, r, scale, dA, false, scratch, s);
 }
 
 qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_is_r_by_c, int r,
@@ -451,18 +469,21 @@ qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_
 
 qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
                             const void* ext_w, const void* ext_act, int M, int r, void* out,
-                            qlora_stream_t stream) {
+                            void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (!act || !ext_w || !ext_act || !out) return QLORA_ERR_NULL;
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
   if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
   if (!aligned16(act) || !aligned16(ext_w) || !aligned16(ext_act) || !aligned16(out))
     return QLORA_ERR_ALIGN;
+  const size_t need = gemm_ws_bytes(M, W->N, W->K, r, transpose_w != 0);
+  if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
   int dev;
   if ((st = current_device(&dev)) != QLORA_OK) return st;
   int* err;
   if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
-  return do_gemm(act, W, transpose_w != 0, ext_w, ext_act, M, r, out, err,
+  return do_gemm(act, W, transpose_w != 0, ext_w, ext_act, M, r, out, err, ws, ws_bytes,
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -528,7 +549,8 @@ qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, 
   if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
     return QLORA_ERR_ALIGN;
-  // The forward needs s*XA [M, r] bf16 plus the down-projection's split partials.
+  // The forward needs s*XA [M, r] bf16 plus the down-projection's split partials; the GEMM's
+  // stream-K partials use what is left of the scratch (whole tiles if they do not fit).
   const size_t sxa_bytes = align256(static_cast<size_t>(M) * r * 2);
   const size_t need = sxa_bytes + align256(down_ws_bytes(M, W->K, r));
   if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
@@ -546,7 +568,8 @@ qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, 
   st = do_lora_down(X, M, W->K, A, true, r, scale, XA_saved, sxa,
                     reinterpret_cast<float*>(w8 + sxa_bytes), s);
   if (st != QLORA_OK) return st;
-  return do_gemm(X, W, false, B, sxa, M, r, H, err, s);
+  return do_gemm(X, W, false, B, sxa, M, r, H, err, w8 + sxa_bytes,
+                 kNoAllocScratchBytes - sxa_bytes, s);
 }
 
 size_t qlora_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }

@@ -12,11 +12,18 @@
 // than 256 tokens a tile holds two 256-token halves (nh = 2) that share every dequantised
 // weight tile: one dequantised element then feeds 1024 flops.
 //
-// Persistent CTAs (one per SM) walk the tile list.  Three shared-memory rings decouple the
-// stages of a 64-deep reduction step so each one's latency hides behind the others:
-//   Q ring  (2 groups x 4 x 4 KB) TMA -> dequant       packed NF4 codes of the weight tile
+// Persistent CTAs (one per SM) walk the work in one of two modes:
+//   tiles     (enough tiles to fill the GPU): CTA b takes tiles b, b + G, b + 2G, ... whole;
+//   stream-K  (fewer tiles than SMs, i.e. few tokens or few output features): the tiles'
+//             reduction steps, laid end to end, are cut into G equal contiguous ranges, one per
+//             CTA.  A tile cut between CTAs leaves fp32 partial sums in the workspace (two slots
+//             per CTA: the head segment of its range and the tail segment), and a finalize
+//             kernel adds them in step order, so results do not depend on timing.
+// Three shared-memory rings decouple the stages of a 64-deep reduction step so each one's
+// latency hides behind the others:
+//   Q ring  (2 groups x 4..16 x 4 KB) TMA -> dequant   packed NF4 codes of the weight tile
 //   W ring  (2 groups x 2 x 16 KB) dequant -> MMA      bf16 weight operand (never in HBM)
-//   X ring  (bt x 128 B slots)   TMA -> MMA            activation operand, 128B-swizzled
+//   X ring  (2-4 steps)          TMA -> MMA            activation operand, 128B-swizzled
 // TMEM holds two accumulators (ping-pong, epilogue of one tile overlaps the next mainloop)
 // whenever they fit in its 512 columns, else one.
 //
@@ -34,10 +41,18 @@
 //               extension step the owning group TMA-loads the LoRA weight tile (B or A) into its
 //               slot instead.  A waiting warp polls its barrier with one lane only.
 //
+// The MMA thread issues every tensor-core instruction of the CTA and is the pipeline's
+// tightest resource, so it commits to one barrier per step (W empty): the X producer recycles
+// X slots on the W ring's empty barriers instead of X barriers of their own.
+//
 // mbarrier waits test phase parity, which cannot tell phases two apart, and TMA copies may land
 // out of order; so every ring slot has exactly one producer and one consumer that each visit
-// its uses in order: W slots 2g, 2g+1 and Q slots 4g..4g+3 belong to dequant group g (the MMA,
-// resp. the Q producer, is the other side), and the X ring has one producer and one consumer.
+// its uses in order, and a waiter that only observes a barrier must gate its next phase:
+// W slots 2g, 2g+1 and Q slots g*q..g*q+q-1 belong to dequant group g (the MMA, resp. the Q
+// producer, is the other side); the X ring is filled by the X producer and consumed by the MMA
+// thread, and an X slot is refilled only after the W slot of the step DX earlier is released
+// (DX <= 4 steps, the W ring's reuse distance, so that release cannot move on without the new
+// X tile).
 // A slot that threads read with ordinary loads and TMA then refills (the Q ring) needs a
 // generic -> async proxy fence between the reads and the release of the slot; without it the
 // refill was seen to overwrite codes not yet read, at large grids and long reductions.
@@ -60,20 +75,25 @@ constexpr uint32_t kWBytes = 16384;         // 128 rows x 64 bf16
 constexpr uint32_t kQBytes = 4096;          // packed codes of one weight tile step
 constexpr int kRowsW = 128;                 // MMA M
 constexpr uint32_t kSmemLimit = 232448;
-constexpr int kQStages = 8;
 constexpr int kWStages = 2 * kGroups;       // two W slots per group
-constexpr int kQPerGroup = kQStages / kGroups;
+constexpr int kMaxQPerGroup = 16;
+constexpr int kAmAhead = 3;                 // owned steps the block absmax is fetched ahead
 
 struct Plan {
   int bt;        // tokens per half (MMA N)
   int nh;        // halves per tile
-  int sx;        // X half-slots
+  int dx;        // X ring depth in steps (2 or 4)
+  int dxlog;     // log2(dx)
+  int sx;        // X half-slots = dx * nh
   int nacc;      // TMEM accumulators (1 or 2)
+  int qlog;      // log2 of the Q slots per dequant group
   uint32_t acc_cols;  // TMEM columns per half accumulator
   uint32_t x_bytes;   // bytes per X half-slot
   size_t smem;
 };
 
+// Small token tiles leave shared memory for a deeper code ring: with few tokens a step is
+// short and the weight stream is the whole job, so more code tiles stay in flight.
 __host__ __device__ inline Plan make_plan(int bt, int nh) {
   Plan p;
   p.bt = bt;
@@ -81,12 +101,58 @@ __host__ __device__ inline Plan make_plan(int bt, int nh) {
   p.x_bytes = static_cast<uint32_t>(bt) * 128u;
   p.acc_cols = bt <= 16 ? 16u : (bt <= 32 ? 32u : (bt <= 64 ? 64u : (bt <= 128 ? 128u : 256u)));
   p.nacc = (2u * nh * p.acc_cols <= 512u) ? 2 : 1;
-  const uint32_t fixed = 1024u + 512u + kQStages * kQBytes + kWStages * kWBytes;
-  int sx = static_cast<int>((kSmemLimit - fixed) / p.x_bytes);
-  if (sx > 8) sx = 8;
-  p.sx = sx;
-  p.smem = fixed + static_cast<size_t>(sx) * p.x_bytes;
+  p.qlog = bt <= 64 ? 4 : (bt <= 128 ? 3 : 2);
+  // X slots are recycled on the W ring's empty barriers, which allows at most 4 steps of X
+  // in flight.
+  p.dx = nh == 2 ? 2 : 4;
+  p.dxlog = nh == 2 ? 1 : 2;
+  p.sx = p.dx * nh;
+  const uint32_t sq = static_cast<uint32_t>(kGroups) << p.qlog;
+  const uint32_t fixed = 1024u + 1024u + sq * kQBytes + kWStages * kWBytes;
+  p.smem = fixed + static_cast<size_t>(p.sx) * p.x_bytes;
   return p;
+}
+
+// Where the CTA's it-th reduction step lies: tile t and step k within the tile.
+struct StepMap {
+  int total;       // steps per tile
+  int streamk;     // 0: whole tiles b, b + G, ...; 1: contiguous range [g0, g0 + n_steps)
+  long long g0;    // stream-K: first global step of this CTA
+  __device__ __forceinline__ void at(int it, int& t, int& k) const {
+    if (streamk) {
+      const long long g = g0 + it;
+      t = static_cast<int>(g / total);
+      k = static_cast<int>(g - static_cast<long long>(t) * total);
+    } else {
+      const int lt = it / total;
+      t = static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x);
+      k = it - lt * total;
+    }
+  }
+};
+
+// (tile, step) of a CTA-local step index that advances by kGroups at a time, without
+// dividing (every tile has at least 2 steps, so one advance wraps at most once).
+struct StepCursor {
+  int t, k;
+  int row0;  // first weight row (or output feature, dX) of tile t
+  __device__ __forceinline__ void set(const StepMap& m, int it, int row_tiles) {
+    m.at(it, t, k);
+    row0 = (t % row_tiles) * kRowsW;
+  }
+  __device__ __forceinline__ void advance(const StepMap& m, int row_tiles) {
+    k += 2;
+    if (k >= m.total) {
+      k -= m.total;
+      t += m.streamk ? 1 : static_cast<int>(gridDim.x);
+      row0 = (t % row_tiles) * kRowsW;
+    }
+  }
+};
+
+// First global step of stream-K CTA b: floor(b * T / G).
+__host__ __device__ __forceinline__ long long sk_start(long long b, long long T, long long G) {
+  return b * T / G;
 }
 
 // Named barrier among the 256 threads of one dequant group (ids 1, 2).
@@ -109,15 +175,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
   const Plan P = make_plan(args.bt, args.nh);
-  const int bt = P.bt, nh = P.nh, SX = P.sx;
-  constexpr int SW = kWStages, SQ = kQStages;
+  const int bt = P.bt, nh = P.nh, SX = P.sx, DX = P.dx, DXLOG = P.dxlog;
+  const int qper = 1 << P.qlog;          // Q slots per dequant group
+  const int SQ = kGroups * qper;
+  constexpr int SW = kWStages;
   uint8_t* w_ring = smem;                     // SW x 16 KB
   uint8_t* q_ring = w_ring + SW * kWBytes;    // SQ x 4 KB
   uint8_t* x_ring = q_ring + SQ * kQBytes;    // SX x bt*128
   uint64_t* bars = reinterpret_cast<uint64_t*>(x_ring + SX * P.x_bytes);
   uint64_t* xfull = bars;
-  uint64_t* xempty = xfull + SX;
-  uint64_t* wfull = xempty + SX;
+  uint64_t* wfull = xfull + SX;
   uint64_t* wempty = wfull + SW;
   uint64_t* qfull = wempty + SW;
   uint64_t* qempty = qfull + SQ;
@@ -127,9 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   auto WS = [&](int it) { return w_ring + w_slot(it) * kWBytes; };
-  auto XS = [&](int hi) { return x_ring + (hi % SX) * P.x_bytes; };
-  auto QS = [&](int qi) { return q_ring + (qi % SQ) * kQBytes; };
-  auto par = [](int i, int s) { return static_cast<uint32_t>(i / s) & 1u; };
+  auto QS = [&](int qi) { return q_ring + qi * kQBytes; };
+  // X half-slot of step it, half h, and the parity of that use.
+  auto x_slot = [&](int it, int h) { return (it & (DX - 1)) * nh + h; };
+  auto x_par = [&](int it) { return static_cast<uint32_t>(it >> DXLOG) & 1u; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -138,20 +206,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile_tokens = nh * bt;
   const int row_tiles = (args.rows_w + kRowsW - 1) / kRowsW;
   const int n_tiles = row_tiles * ((args.M + tile_tokens - 1) / tile_tokens);
-  const int my_tiles =
-      static_cast<int>(blockIdx.x) < n_tiles ? (n_tiles - 1 - static_cast<int>(blockIdx.x)) /
-                                                       static_cast<int>(gridDim.x) + 1
-                                             : 0;
+
+  // This CTA's reduction steps: whole tiles, or one contiguous stream-K range.
+  StepMap map;
+  map.total = total;
+  map.streamk = args.streamk;
+  int n_steps;
+  if (args.streamk) {
+    const long long T = static_cast<long long>(n_tiles) * total;
+    map.g0 = sk_start(blockIdx.x, T, gridDim.x);
+    n_steps = static_cast<int>(sk_start(blockIdx.x + 1, T, gridDim.x) - map.g0);
+  } else {
+    map.g0 = 0;
+    const int my_tiles = static_cast<int>(blockIdx.x) < n_tiles
+                             ? (n_tiles - 1 - static_cast<int>(blockIdx.x)) /
+                                       static_cast<int>(gridDim.x) + 1
+                             : 0;
+    n_steps = my_tiles * total;
+  }
+  // Segment of the range starting at step it: tile t, steps [k0, k0 + len) of that tile.
+  auto segment = [&](int it, int& t, int& k0, int& len) {
+    map.at(it, t, k0);
+    len = total - k0 < n_steps - it ? total - k0 : n_steps - it;
+  };
+
   const uint32_t tile_cols = static_cast<uint32_t>(nh) * P.acc_cols;
   uint32_t ncols = static_cast<uint32_t>(P.nacc) * tile_cols;
   if (ncols < 32) ncols = 32;
   int* err = args.err;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SX; ++s) {
-      mbar_init(xfull + s, 1);
-      mbar_init(xempty + s, 1);
-    }
+    for (int s = 0; s < SX; ++s) mbar_init(xfull + s, 1);
     for (int s = 0; s < SW; ++s) {
       mbar_init(wfull + s, 1);
       mbar_init(wempty + s, 1);
@@ -181,56 +266,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
       tma_prefetch_desc(&tm_ext_act);
-      int xs = 0;            // ring slot
-      uint32_t xph = 0;      // use parity of that slot
-      int issued = 0;
+      int issued = 0;  // steps whose X tiles were issued
       bool ok = true;
-      for (int lt = 0; ok && lt < my_tiles; ++lt) {
-        const int t = blockIdx.x + lt * gridDim.x;
+      for (int it = 0; ok && it < n_steps;) {
+        int t, k0, len;
+        segment(it, t, k0, len);
         const int tok0 = (t / row_tiles) * tile_tokens;
-        for (int k = 0; ok && k < total; ++k) {
+        for (int k = k0; k < k0 + len; ++k, ++it) {
+          // Step it reuses the X slots of step it - DX: wait until that step's MMAs are done.
+          if (it >= DX &&
+              !mbar_wait(wempty + w_slot(it - DX), w_par(it - DX), kErrWaitEmpty, err, it)) {
+            ok = false;
+            break;
+          }
           for (int h = 0; h < nh; ++h) {
-            if (!mbar_wait(xempty + xs, xph ^ 1u, kErrWaitEmpty, err, issued)) {
-              ok = false;
-              break;
-            }
+            const int xs = x_slot(it, h);
             uint8_t* dst = x_ring + xs * P.x_bytes;
             mbar_arrive_expect_tx(xfull + xs, P.x_bytes);
             if (k < kt)
               tma_load_2d(dst, &tm_act, xfull + xs, k * 64, tok0 + h * bt);
             else
               tma_load_2d(dst, &tm_ext_act, xfull + xs, (k - kt) * 64, tok0 + h * bt);
-            ++issued;
-            if (++xs == SX) {
-              xs = 0;
-              xph ^= 1u;
-            }
           }
+          issued = it + 1;
         }
       }
       // Every issued copy lands before the CTA may exit.
-      for (int j = issued > SX ? issued - SX : 0; j < issued; ++j)
-        mbar_wait(xfull + j % SX, par(j, SX), kErrWaitDrain, err, j);
+      for (int j = issued > DX ? issued - DX : 0; j < issued; ++j)
+        for (int h = 0; h < nh; ++h) mbar_wait(xfull + x_slot(j, h), x_par(j), kErrWaitDrain, err, j);
     }
   } else if (warp == 2) {
     // ------------------------------ Q producer -------------------------------------------
-    // Step it's code tile goes to the four-slot Q ring of its owner group g = it % 2, filled and
-    // consumed strictly in order (slot 4g + (v & 3) for the group's v-th code tile), so each
-    // slot has exactly one producer and one consumer even though TMA copies land out of order.
+    // Step it's code tile goes to the Q ring of its owner group g = it % 2, filled and
+    // consumed strictly in order (slot g * qper + (v % qper) for the group's v-th code tile),
+    // so each slot has exactly one producer and one consumer even though TMA copies land out
+    // of order.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       int vq0 = 0, vq1 = 0;  // per-group code-tile counters (registers, not an array)
       bool ok = true;
-      for (int lt = 0; ok && lt < my_tiles; ++lt) {
-        const int t = blockIdx.x + lt * gridDim.x;
+      for (int it = 0; ok && it < n_steps;) {
+        int t, k0, len;
+        segment(it, t, k0, len);
         const int row0 = (t % row_tiles) * kRowsW;
-        for (int k = 0; k < kt; ++k) {
-          const int it = lt * total + k;
-          const int g = it & 1;
+        const int kq_end = k0 + len < kt ? k0 + len : kt;
+        for (int k = k0; k < kq_end; ++k) {
+          const int step = it + (k - k0);
+          const int g = step & 1;
           const int v = g ? vq1 : vq0;
-          const int slot = kQPerGroup * g + (v % kQPerGroup);
-          const uint32_t u = static_cast<uint32_t>(v / kQPerGroup);
-          if (!mbar_wait(qempty + slot, (u & 1u) ^ 1u, kErrWaitEmpty, err, it)) {
+          const int slot = (g << P.qlog) + (v & (qper - 1));
+          const uint32_t u = static_cast<uint32_t>(v >> P.qlog);
+          if (!mbar_wait(qempty + slot, (u & 1u) ^ 1u, kErrWaitEmpty, err, step)) {
             ok = false;
             break;
           }
@@ -242,13 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             tma_load_2d(QS(slot), &tm_q, qfull + slot, row0 / 2, k * 64);  // [64 rows, 64 B]
         }
+        it += len;
       }
       // Every issued copy lands before the CTA may exit.
       for (int g = 0; g < kGroups; ++g) {
         const int n = g ? vq1 : vq0;
-        for (int v = n > kQPerGroup ? n - kQPerGroup : 0; v < n; ++v)
-          mbar_wait(qfull + kQPerGroup * g + (v % kQPerGroup),
-                    static_cast<uint32_t>(v / kQPerGroup) & 1u, kErrWaitDrain, err, v);
+        for (int v = n > qper ? n - qper : 0; v < n; ++v)
+          mbar_wait(qfull + (g << P.qlog) + (v & (qper - 1)),
+                    static_cast<uint32_t>(v >> P.qlog) & 1u, kErrWaitDrain, err, v);
       }
     }
   } else if (warp == 1) {
@@ -267,24 +354,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t w_slot_step = kWBytes >> 4;
       const uint64_t x_slot_step = P.x_bytes >> 4;
       const uint32_t half_cols = P.acc_cols;
-      int it = 0, xs = 0;
-      uint32_t xph = 0;
+      int it = 0, seg = 0;
       bool ok = true;
-      for (int lt = 0; ok && lt < my_tiles; ++lt) {
-        const int ab = P.nacc == 2 ? (lt & 1) : 0;
-        const int use = P.nacc == 2 ? (lt >> 1) : lt;
+      while (ok && it < n_steps) {
+        int t, k0, len;
+        segment(it, t, k0, len);
+        const int ab = P.nacc == 2 ? (seg & 1) : 0;
+        const int use = P.nacc == 2 ? (seg >> 1) : seg;
         if (!mbar_wait(accempty + ab, (static_cast<uint32_t>(use) & 1u) ^ 1u, kErrWaitAcc, err,
-                       lt))
+                       seg))
           break;
         tc_fence_after();
         const uint32_t dtm = tmem_base + static_cast<uint32_t>(ab) * tile_cols;
-        for (int k = 0; k < total; ++k, ++it) {
+        for (int k = k0; k < k0 + len; ++k, ++it) {
           const int ws = w_slot(it);
+          const int xs = (it & (DX - 1)) * nh;
           bool got = mbar_wait(wfull + ws, w_par(it), kErrWaitDequant, err, it);
-          const int xs1 = xs + 1 == SX ? 0 : xs + 1;
-          const uint32_t xph1 = xs + 1 == SX ? (xph ^ 1u) : xph;
-          if (got) got = mbar_wait(xfull + xs, xph, kErrWaitFull, err, it);
-          if (got && nh == 2) got = mbar_wait(xfull + xs1, xph1, kErrWaitFull, err, it);
+          if (got) got = mbar_wait(xfull + xs, x_par(it), kErrWaitFull, err, it);
+          if (got && nh == 2) got = mbar_wait(xfull + xs + 1, x_par(it), kErrWaitFull, err, it);
           if (!got) {
             ok = false;
             break;
@@ -292,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint64_t ad = wdesc0 + static_cast<uint64_t>(ws) * w_slot_step;
           const uint64_t bd0 = xdesc0 + static_cast<uint64_t>(xs) * x_slot_step;
-          const uint64_t bd1 = xdesc0 + static_cast<uint64_t>(xs1) * x_slot_step;
-          const uint32_t acc0 = k > 0 ? 1u : 0u;
+          const uint64_t bd1 = bd0 + x_slot_step;
+          const uint32_t acc0 = k > k0 ? 1u : 0u;  // the segment's first step starts the sum
           if (k < kt) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -306,59 +393,80 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rem = args.r_pad16 - (k - kt) * 64;
             const int nk = (rem >= 64 ? 64 : rem) / 16;
             for (int j = 0; j < nk; ++j) {
-              umma_f16_ss(dtm, ad + j * w_kstep, bd0 + j * x_kstep, idesc, 1u);
-              if (nh == 2) umma_f16_ss(dtm + half_cols, ad + j * w_kstep, bd1 + j * x_kstep, idesc, 1u);
+              const uint32_t acc = j > 0 ? 1u : acc0;
+              umma_f16_ss(dtm, ad + j * w_kstep, bd0 + j * x_kstep, idesc, acc);
+              if (nh == 2)
+                umma_f16_ss(dtm + half_cols, ad + j * w_kstep, bd1 + j * x_kstep, idesc, acc);
             }
           }
-          umma_commit(xempty + xs);
-          if (nh == 2) umma_commit(xempty + xs1);
-          umma_commit(wempty + ws);
-          if (nh == 2) {
-            xs = xs1 + 1 == SX ? 0 : xs1 + 1;
-            xph = xs1 + 1 == SX ? (xph1 ^ 1u) : xph1;
-          } else {
-            xs = xs1;
-            xph = xph1;
-          }
+          umma_commit(wempty + ws);  // releases the W slot and, DX steps on, the X slots
         }
         if (!ok) break;
         umma_commit(accfull + ab);
+        ++seg;
       }
       umma_commit(drain);
       mbar_wait(drain, 0, kErrWaitDrain, err);  // every MMA retired before teardown
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------ epilogue ---------------------------------------------
+    // A segment that covers its whole tile goes straight to the bf16 output; a cut one goes
+    // as fp32 to this CTA's head (0) or tail (1) partial slot of the workspace.
     const int quad = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    for (int lt = 0; lt < my_tiles; ++lt) {
-      const int t = blockIdx.x + lt * gridDim.x;
-      const int ab = P.nacc == 2 ? (lt & 1) : 0;
-      const int use = P.nacc == 2 ? (lt >> 1) : lt;
+    int seg = 0;
+    for (int it = 0; it < n_steps; ++seg) {
+      int t, k0, len;
+      segment(it, t, k0, len);
+      const bool whole = k0 == 0 && len == total;
+      const int slot = it == 0 ? 0 : 1;
+      it += len;
+      const int ab = P.nacc == 2 ? (seg & 1) : 0;
+      const int use = P.nacc == 2 ? (seg >> 1) : seg;
       bool got = true;
       if (lane == 0)
         got = mbar_wait_sleepy(accfull + ab, static_cast<uint32_t>(use) & 1u, kErrWaitAcc, err,
-                               lt);
+                               seg);
       if (!__shfl_sync(0xFFFFFFFFu, got, 0)) break;
-      for (int i = 0; i < 64 && !mbar_try_wait(accfull + ab, static_cast<uint32_t>(use) & 1u); ++i) {
-      }
+      __syncwarp();  // lane 0's acquire, passed on to the warp
       tc_fence_after();
-      const int row = (t % row_tiles) * kRowsW + quad * 32 + lane;
+      const int row_l = quad * 32 + lane;
+      const int row = (t % row_tiles) * kRowsW + row_l;
       const int tok0 = (t / row_tiles) * tile_tokens;
       const bool row_ok = row < args.rows_w;
-      for (int h = 0; h < nh; ++h) {
-        const uint32_t tb = tmem_base + lane_base + static_cast<uint32_t>(ab) * tile_cols +
-                            static_cast<uint32_t>(h) * P.acc_cols;
-        for (int c8 = 0; c8 < bt / 8; ++c8) {
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(tb + static_cast<uint32_t>(c8 * 8), v);
-          tmem_ld_wait();
+      float* part = args.partial +
+                    ((static_cast<long long>(blockIdx.x) * 2 + slot) * tile_tokens) * kRowsW;
+      // (Two separate loops: a branch inside the drain loop measurably slows the bf16 path.)
+      if (whole) {
+        for (int h = 0; h < nh; ++h) {
+          const uint32_t tb = tmem_base + lane_base + static_cast<uint32_t>(ab) * tile_cols +
+                              static_cast<uint32_t>(h) * P.acc_cols;
+          for (int c8 = 0; c8 < bt / 8; ++c8) {
+            uint32_t v[8];
+            tmem_ld_32x32b_x8(tb + static_cast<uint32_t>(c8 * 8), v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int tok = tok0 + h * bt + c8 * 8 + j;
-            if (row_ok && tok < args.M)
-              args.out[static_cast<long long>(tok) * args.rows_w + row] =
-                  __float2bfloat16_rn(__uint_as_float(v[j]));
+            for (int j = 0; j < 8; ++j) {
+              const int tok = tok0 + h * bt + c8 * 8 + j;
+              if (row_ok && tok < args.M)
+                args.out[static_cast<long long>(tok) * args.rows_w + row] =
+                    __float2bfloat16_rn(__uint_as_float(v[j]));
+            }
+          }
+        }
+      } else {
+        for (int h = 0; h < nh; ++h) {
+          const uint32_t tb = tmem_base + lane_base + static_cast<uint32_t>(ab) * tile_cols +
+                              static_cast<uint32_t>(h) * P.acc_cols;
+          for (int c8 = 0; c8 < bt / 8; ++c8) {
+            uint32_t v[8];
+            tmem_ld_32x32b_x8(tb + static_cast<uint32_t>(c8 * 8), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int tl = h * bt + c8 * 8 + j;
+              part[static_cast<long long>(tl) * kRowsW + row_l] = __uint_as_float(v[j]);
+            }
           }
         }
       }
@@ -397,9 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       seg_kb = kseg;
     }
     const uint32_t c0 = 4u * static_cast<uint32_t>(hf);  // first 16-byte chunk of this half
-    // Effective absmax of this thread's block at reduction step k of tile t (0 outside W0).
-    auto absmax_at = [&](int t, int k) -> float {
-      const int row0 = (t % row_tiles) * kRowsW;
+    // Effective absmax of this thread's block at reduction step k of the tile whose first
+    // row is row0 (0 outside W0).
+    auto absmax_at = [&](int row0, int k) -> float {
       long long blk;
       if (!kTransW) {
         const int n = row0 + seg_row;
@@ -413,28 +521,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       return nf4_block_absmax(args.absmax, args.absmax_q8, args.absmax_scale, args.dq, blk);
     };
 
-    // Steps it = g, g + 2, ... of the CTA's pipeline (tile lt = it / total, k = it % total).
-    // The block absmax is fetched one owned step ahead to hide its latency.  After a failed
-    // wait the group keeps walking its steps (without waiting or writing) so that every
-    // thread still meets the group barrier once per step.
-    const int n_steps = my_tiles * total;
+    // Steps it = g, g + 2, ... of the CTA's range.  The block absmax is fetched kAmAhead owned
+    // steps ahead to hide its latency.  After a failed wait the group keeps walking its steps
+    // (without waiting or writing) so that every thread still meets the group barrier once
+    // per step.
     int vq = 0;  // code tiles this group has consumed
     bool failed = false;
     int last_ext = -1;
     if (tid == 0) tma_prefetch_desc(&tm_ext_w);
     auto absmax_of_step = [&](int it) -> float {
-      const int k = it % total;
-      if (it >= n_steps || k >= kt) return 0.f;
-      return absmax_at(blockIdx.x + (it / total) * gridDim.x, k);
+      if (it >= n_steps) return 0.f;
+      int t, k;
+      map.at(it, t, k);
+      return k < kt ? absmax_at((t % row_tiles) * kRowsW, k) : 0.f;
     };
-    float am = absmax_of_step(g);
-    for (int it = g; it < n_steps; it += kGroups) {
-      const int lt = it / total;
-      const int k = it - lt * total;
-      const float am_next = failed ? 0.f : absmax_of_step(it + kGroups);
+    static_assert(kGroups == 2 && kAmAhead == 3, "the step cursors advance by two steps");
+    float am0 = absmax_of_step(g);
+    float am1 = absmax_of_step(g + kGroups);
+    float am2 = absmax_of_step(g + 2 * kGroups);
+    StepCursor cur, ahead;  // step it, and step it + kAmAhead * kGroups
+    cur.set(map, g, row_tiles);
+    ahead.set(map, g + kAmAhead * kGroups, row_tiles);
+    for (int it = g; it < n_steps;
+         it += kGroups, cur.advance(map, row_tiles), ahead.advance(map, row_tiles)) {
+      const int k = cur.k;
+      const float am_next =
+          (failed || it + kAmAhead * kGroups >= n_steps || ahead.k >= kt)
+              ? 0.f
+              : absmax_at(ahead.row0, ahead.k);
       if (k < kt) {
-        const int qslot = kQPerGroup * g + (vq % kQPerGroup);
-        const uint32_t qpar = static_cast<uint32_t>(vq / kQPerGroup) & 1u;
+        const int qslot = (g << P.qlog) + (vq & (qper - 1));
+        const uint32_t qpar = static_cast<uint32_t>(vq >> P.qlog) & 1u;
         ++vq;
         if (!failed) failed = !mbar_wait_warp(qfull + qslot, qpar, kErrWaitFull, err, it);
         if (!failed) {
@@ -445,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(qempty + qslot);
           Nf4Lut lut;
-          nf4_build_lut(args.cb, am, lut);
+          nf4_build_lut(args.cb, am0, lut);
           const uint4 o0 = nf4_lookup8(lut, q4.x);
           const uint4 o1 = nf4_lookup8(lut, q4.y);
           const uint4 o2 = nf4_lookup8(lut, q4.z);
@@ -462,14 +579,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         group_sync(g);
         if (tid == 0 && !failed) mbar_arrive(wfull + w_slot(it));
-      } else if (tid < 32) {
-        // Extension step: one thread waits for the slot and TMA-loads the LoRA weight tile.
-        if (lane == 0 && !failed) {
-          const int e = k - kt;
-          const int row0 = ((blockIdx.x + lt * gridDim.x) % row_tiles) * kRowsW;
-          if (!mbar_wait(wempty + w_slot(it), w_par(it) ^ 1u, kErrWaitEmpty, err, it)) {
-            failed = true;
-          } else {
+      } else {
+        // Extension step: the lead thread TMA-loads the LoRA weight tile into the W slot.  Every
+        // warp of the group first sees the slot's previous use released and the group syncs:
+        // a warp that skipped this use could otherwise meet the slot's barrier two phases on.
+        if (!failed) failed = !mbar_wait_warp(wempty + w_slot(it), w_par(it) ^ 1u, kErrWaitEmpty,
+                                              err, it);
+        group_sync(g);
+        if (tid == 0 && !failed) {
+          {
+            const int e = k - kt;
+            const int row0 = cur.row0;
             uint64_t* bar = wfull + w_slot(it);
             mbar_arrive_expect_tx(bar, kWBytes);
             if (!kTransW) {
@@ -481,9 +601,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             last_ext = it;
           }
         }
-        failed = __shfl_sync(0xFFFFFFFFu, failed, 0);
       }
-      am = am_next;
+      am0 = am1;
+      am1 = am2;
+      am2 = am_next;
     }
     // After a failure, copies this thread issued must land before the CTA exits.
     if (failed && last_ext >= 0)
@@ -496,6 +617,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, ncols);
   }
+}
+
+// Stream-K finalize.  A tile cut between CTAs b_first..b_last gets the sum of their partials
+// in that (step) order, rounded once to bf16; an uncut tile was written whole.  Grid (chunks of
+// 1024 tile elements, tiles); each thread owns 4 consecutive output features of one token and
+// issues its partial loads four contributors at a time before adding them in order.
+__global__ void __launch_bounds__(256) qlora_gemm_finalize(const float* __restrict__ partial,
+                                                           int M, int rows_w, int tile_tokens,
+                                                           int total, long long T, int G,
+                                                           __nv_bfloat16* __restrict__ out) {
+  const int row_tiles = (rows_w + kRowsW - 1) / kRowsW;
+  const int t = blockIdx.y;
+  const long long gs = static_cast<long long>(t) * total;
+  // CTA holding global step g: the largest b with floor(b T / G) <= g.
+  auto owner = [&](long long g) { return static_cast<int>(((g + 1) * G - 1) / T); };
+  const int b_first = owner(gs);
+  const int b_last = owner(gs + total - 1);
+  if (b_first == b_last) return;
+  const int e = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // element of the tile
+  if (e >= tile_tokens * kRowsW) return;
+  const int tl = e / kRowsW, rl = e - tl * kRowsW;
+  const int tok = (t / row_tiles) * tile_tokens + tl;
+  const int row = (t % row_tiles) * kRowsW + rl;
+  if (tok >= M || row >= rows_w) return;  // rows_w % 64 == 0: the 4 features are all in or out
+  const long long slot_elems = static_cast<long long>(tile_tokens) * kRowsW;
+  const float* base = partial + e;
+  auto slot_ptr = [&](int b) {
+    const int slot = sk_start(b, T, G) >= gs ? 0 : 1;  // tile t heads b's range, or ends it
+    return base + (static_cast<long long>(b) * 2 + slot) * slot_elems;
+  };
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int b = b_first; b <= b_last; b += 4) {
+    float4 p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (b + i <= b_last) p[i] = __ldg(reinterpret_cast<const float4*>(slot_ptr(b + i)));
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (b + i <= b_last) {
+        v.x += p[i].x;
+        v.y += p[i].y;
+        v.z += p[i].z;
+        v.w += p[i].w;
+      }
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(out + static_cast<long long>(tok) * rows_w + row) = pk;
 }
 
 int g_sm_count[64];
@@ -514,8 +686,33 @@ int gemm_pick_stages(int bt) { return make_plan(bt, 1).sx; }
 
 size_t gemm_smem_bytes(int bt, int nh) { return make_plan(bt, nh).smem; }
 
-cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, const GemmArgs& args,
-                              cudaStream_t stream) {
+GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count) {
+  GemmSchedule sc;
+  const int bt = gemm_pick_bt(M), nh = gemm_pick_halves(M);
+  const int tile_tokens = bt * nh;
+  sc.n_tiles = ((rows_w + kRowsW - 1) / kRowsW) * ((M + tile_tokens - 1) / tile_tokens);
+  const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
+  if (sc.n_tiles >= G) {
+    sc.streamk = 0;
+    sc.grid = G;
+  } else {
+    // Fewer tiles than SMs: cut the reduction so every SM streams its share of the weight
+    // (every CTA gets at least one step).
+    const long long T = static_cast<long long>(sc.n_tiles) * steps_per_tile;
+    sc.streamk = 1;
+    sc.grid = T < G ? static_cast<int>(T) : G;
+  }
+  sc.partial_floats = sc.streamk ? static_cast<size_t>(sc.grid) * 2 * tile_tokens * kRowsW : 0;
+  return sc;
+}
+
+size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile) {
+  return 4 * gemm_schedule(M, rows_w, steps_per_tile, kGemmMaxCtas).partial_floats;
+}
+
+cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
+                              size_t partial_floats_avail, cudaStream_t stream, int* launched) {
+  *launched = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -524,25 +721,40 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, const GemmArgs
     e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
   }
+  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, g_sm_count[dev]);
+  if (sc.streamk && (!args.partial || sc.partial_floats > partial_floats_avail)) {
+    // No room for the partial sums: whole tiles, one CTA per tile.
+    sc.streamk = 0;
+    sc.grid = sc.n_tiles;
+  }
+  args.streamk = sc.streamk;
   const size_t smem = gemm_smem_bytes(args.bt, args.nh);
-  const int row_tiles = (args.rows_w + kRowsW - 1) / kRowsW;
-  const int tile_tokens = args.bt * args.nh;
-  const int n_tiles = row_tiles * ((args.M + tile_tokens - 1) / tile_tokens);
-  const int grid = n_tiles < g_sm_count[dev] ? n_tiles : g_sm_count[dev];
   if (!trans_w) {
     e = cudaFuncSetAttribute(qlora_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    qlora_gemm_kernel<false><<<grid, kThreads, smem, stream>>>(maps.act, maps.q, maps.ext_w,
-                                                               maps.ext_act, args);
+    qlora_gemm_kernel<false><<<sc.grid, kThreads, smem, stream>>>(maps.act, maps.q, maps.ext_w,
+                                                                  maps.ext_act, args);
   } else {
     e = cudaFuncSetAttribute(qlora_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    qlora_gemm_kernel<true><<<grid, kThreads, smem, stream>>>(maps.act, maps.q, maps.ext_w,
-                                                              maps.ext_act, args);
+    qlora_gemm_kernel<true><<<sc.grid, kThreads, smem, stream>>>(maps.act, maps.q, maps.ext_w,
+                                                                 maps.ext_act, args);
   }
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  *launched = 1;
+  if (!sc.streamk) return e;
+  const int total = args.kt + args.n_ext;
+  const long long T = static_cast<long long>(sc.n_tiles) * total;
+  const int tile_elems = args.bt * args.nh * kRowsW;
+  const dim3 fgrid((tile_elems / 4 + 255) / 256, sc.n_tiles);
+  qlora_gemm_finalize<<<fgrid, 256, 0, stream>>>(args.partial, args.M, args.rows_w,
+                                                 args.bt * args.nh, total, T, sc.grid, args.out);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) *launched = 2;
+  return e;
 }
 
 }  // namespace qlora

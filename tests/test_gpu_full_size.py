@@ -130,14 +130,18 @@ def _grad_like(M, N, seed):
     return (torch.randn((M, N), generator=g) * 1e-2).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 14336), (14336, 4096)])
-def test_one_hot_products_reproduce_the_weight(K, N):
+@pytest.mark.parametrize("K,N,M", [(4096, 4096, None), (4096, 14336, None), (14336, 4096, None),
+                                   (4096, 14336, 16), (4096, 14336, 1024)])
+def test_one_hot_products_reproduce_the_weight(K, N, M):
     """With one-hot activations each output row of the dequant GEMM is one row (dX) or one
     column (forward) of deq(W0), exactly: one product by 1.0 accumulated in fp32 and rounded to
     bf16 is the bf16 weight itself, so every element must equal the oracle's dequantised weight
-    exactly (compared as values: the sign of a zero is left to the tensor core's adder).  Three repeats at a full grid and a 64-step reduction: every pipeline
-    slot is reused many times, so a slot refilled before its reads finished shows up as wrong
-    bits here (the LoRA extension input is zero and contributes nothing)."""
+    exactly (compared as values: the sign of a zero is left to the tensor core's adder).
+    Three repeats at a full grid: every pipeline slot is reused many times, so a slot refilled
+    before its reads finished shows up as wrong values here (the LoRA extension input is zero
+    and contributes nothing).  M = None takes every row / column of the weight (whole-tile
+    schedule); M = 16 and 1024 tokens give fewer tiles than SMs, i.e. the stream-K schedule,
+    whose cut tiles are summed from partials (exact too: all but one partial are zero)."""
     from nf4_base_lora_blockwise_b200 import abi
 
     inp, L = parity.make(4, K, N, 16, seed=K + 3 * N)
@@ -150,32 +154,34 @@ def test_one_hot_products_reproduce_the_weight(K, N):
     A = torch.zeros((r, K), dtype=torch.bfloat16, device="cuda")
     B = torch.zeros((N, r), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
+    Md, Mf = (N, K) if M is None else (M, M)
+    ws = linear.alloc_workspace(max(Md, Mf), N, K, r, "cuda")
 
-    def one_hot(M, C):
-        t = torch.zeros((M, C), dtype=torch.bfloat16, device="cuda")
-        m = torch.arange(M, device="cuda")
-        t[m, m % C] = 1.0
+    def one_hot(m, C):
+        t = torch.zeros((m, C), dtype=torch.bfloat16, device="cuda")
+        i = torch.arange(m, device="cuda")
+        t[i, i % C] = 1.0
         return t
 
     # dX[m, :] = deq(W0)[m % N, :]
-    dY = one_hot(N, N)
-    zero = torch.zeros((N, r), dtype=torch.bfloat16, device="cuda")
+    dY = one_hot(Md, N)
+    zero = torch.zeros((Md, r), dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
-        dX = torch.full((N, K), float("nan"), dtype=torch.bfloat16, device="cuda")
-        abi.qlora_nf4_gemm(dY.data_ptr(), cw, 1, A.data_ptr(), zero.data_ptr(), N, r,
-                           dX.data_ptr(), stream)
+        dX = torch.full((Md, K), float("nan"), dtype=torch.bfloat16, device="cuda")
+        abi.qlora_nf4_gemm(dY.data_ptr(), cw, 1, A.data_ptr(), zero.data_ptr(), Md, r,
+                           dX.data_ptr(), ws.data_ptr(), ws.numel(), stream)
         torch.cuda.synchronize()
         assert linear.device_error() == 0
-        bad = int((parity.f32(dX) != ref_w).sum())
+        bad = int((parity.f32(dX) != ref_w[np.arange(Md) % N]).sum())
         assert bad == 0, f"dX: {bad} elements differ from deq(W0) rows"
     # h[m, :] = deq(W0)[:, m % K]
-    X = one_hot(K, K)
-    zero = torch.zeros((K, r), dtype=torch.bfloat16, device="cuda")
+    X = one_hot(Mf, K)
+    zero = torch.zeros((Mf, r), dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
-        H = torch.full((K, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-        abi.qlora_nf4_gemm(X.data_ptr(), cw, 0, B.data_ptr(), zero.data_ptr(), K, r,
-                           H.data_ptr(), stream)
+        H = torch.full((Mf, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        abi.qlora_nf4_gemm(X.data_ptr(), cw, 0, B.data_ptr(), zero.data_ptr(), Mf, r,
+                           H.data_ptr(), ws.data_ptr(), ws.numel(), stream)
         torch.cuda.synchronize()
         assert linear.device_error() == 0
-        bad = int((parity.f32(H) != ref_w.T).sum())
+        bad = int((parity.f32(H) != ref_w.T[np.arange(Mf) % K]).sum())
         assert bad == 0, f"h: {bad} elements differ from deq(W0) columns"
