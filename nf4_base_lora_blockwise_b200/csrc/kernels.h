@@ -75,6 +75,26 @@ size_t gemm_smem_bytes(int bt, int nh);
 cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
                               size_t partial_floats_avail, cudaStream_t stream, int* launched);
 
+// ------------------------------ few-token forward (mma.sync, register-direct) ---------------
+// h[M, N] = X[M, K] . deq(W0)^T + ext_act[M, r] . ext_w[N, r]^T for M <= 32: stream-K over
+// (128-row tile, 64-block) units with fp32 partial slots and a fixed-order finalize.
+struct GemvPlan {
+  int tt;                 // token tiles of 8
+  long long units;
+  int grid;
+  int max_seg;            // row tiles a CTA's range can touch
+  size_t partial_floats;
+  size_t smem;
+};
+constexpr int kGemvMaxTokens = 32;
+GemvPlan gemv_plan(int M, int N, int K, int sm_count);
+cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const float* absmax,
+                                const uint8_t* absmax_q8, const float* absmax_scale, int dq, int M,
+                                int N, int K, const __nv_bfloat16* ext_act,
+                                const __nv_bfloat16* ext_w, int r, __nv_bfloat16* out,
+                                float* partial, size_t partial_floats, const Codebook& cb,
+                                cudaStream_t stream);
+
 // ------------------------------ rank-r skinny products (mma.sync) --------------------------
 // out[m, j] = sum_c in[m, c] * Wl(j, c); Wl(j, c) = w[j * C + c] (w_is_rc = true, i.e. A [r, C])
 // or w[c * r + j] (w_is_rc = false, i.e. B [C, r]).  Writes bf16 RN(v) to `saved` (if not

@@ -154,6 +154,7 @@ int ext_steps(int r) { return ((r + 15) / 16 * 16 + 63) / 64; }
 
 // Stream-K partial-sum bytes of the forward (rows N, K/64 steps) or dX (rows K, N/64 steps).
 size_t gemm_ws_bytes(int M, int N, int K, int r, bool trans) {
+  if (!trans && M <= kGemvMaxTokens) return 4 * gemv_plan(M, N, K, kGemmMaxCtas).partial_floats;
   return trans ? gemm_partial_bytes_bound(M, K, N / 64 + ext_steps(r))
                : gemm_partial_bytes_bound(M, N, K / 64 + ext_steps(r));
 }
@@ -263,6 +264,20 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
                      const void* ext_act, int M, int r, void* out, int* err, void* partial,
                      size_t partial_bytes, cudaStream_t s) {
+  if (!trans && M <= kGemvMaxTokens && partial) {
+    // Few tokens: the register-direct kernel streams the weight without the tcgen05 rings.
+    const cudaError_t e = launch_nf4_gemv_fwd(
+        static_cast<const __nv_bfloat16*>(act), W->q, W->absmax, W->absmax_q8, W->absmax_scale,
+        W->double_quant ? 1 : 0, M, W->N, W->K, static_cast<const __nv_bfloat16*>(ext_act),
+        static_cast<const __nv_bfloat16*>(ext_w), r, static_cast<__nv_bfloat16*>(out),
+        static_cast<float*>(partial), partial_bytes / 4, codebook(), s);
+    if (e == cudaSuccess) {
+      count(2);
+      return QLORA_OK;
+    }
+    if (e != cudaErrorInvalidValue) return QLORA_ERR_CUDA;
+    (void)cudaGetLastError();  // scratch too small for its partials: use the tcgen05 kernel
+  }
   GemmArgs a = gemm_args(W, M, r, trans, out, err);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;

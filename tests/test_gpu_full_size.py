@@ -141,7 +141,8 @@ def test_one_hot_products_reproduce_the_weight(K, N, M):
     before its reads finished shows up as wrong values here (the LoRA extension input is zero
     and contributes nothing).  M = None takes every row / column of the weight (whole-tile
     schedule); M = 16 and 1024 tokens give fewer tiles than SMs, i.e. the stream-K schedule,
-    whose cut tiles are summed from partials (exact too: all but one partial are zero)."""
+    whose cut tiles are summed from partials (exact too: all but one partial are zero).  The
+    forward at M = 16 runs the few-token kernel, exact up to the weight's bf16 rounding."""
     from nf4_base_lora_blockwise_b200 import abi
 
     inp, L = parity.make(4, K, N, 16, seed=K + 3 * N)
@@ -183,5 +184,15 @@ def test_one_hot_products_reproduce_the_weight(K, N, M):
                            H.data_ptr(), ws.data_ptr(), ws.numel(), stream)
         torch.cuda.synchronize()
         assert linear.device_error() == 0
-        bad = int((parity.f32(H) != ref_w.T[np.arange(Mf) % K]).sum())
+        ref_h = ref_w.T[np.arange(Mf) % K]
+        if M is not None and M <= 32:
+            # The few-token forward applies the block scale after the products: the weight
+            # enters as bf16(c) * absmax, rounded once more to bf16 here, instead of
+            # bf16(c * absmax).  bf16 rounds within 2^-8 relative, so the two paths agree
+            # within 3 * 2^-8 relative (exact zeros stay zero).
+            err = np.abs(parity.f32(H) - ref_h)
+            bound = 3.0 * 2.0 ** -8 * np.abs(ref_h)
+            bad = int((err > bound).sum())
+        else:
+            bad = int((parity.f32(H) != ref_h).sum())
         assert bad == 0, f"h: {bad} elements differ from deq(W0) columns"
