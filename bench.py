@@ -531,6 +531,22 @@ def workload_config(w):
 
 
 # ----------------------------------------------------------------------------------------------
+# Replicas: every rank times its own copy of the step; the job's time is the slowest rank's
+# ----------------------------------------------------------------------------------------------
+def max_over_ranks(ms, dist, device):
+    """The largest of the ranks' device-timed milliseconds (this rank's alone without dist)."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, M, steps, total_ms):
+    """Whole-job throughput: every rank processed M tokens per step, in the slowest rank's time."""
+    return world * M * steps / (total_ms * 1e-3)
+
+
+# ----------------------------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -604,20 +620,12 @@ def main():
     if abi.qlora_device_error() != 0:
         raise SystemExit("device error word set during the timed region")
 
-    total_ms = sum(per_step)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    tokens = world * w.M * args.steps
-    value = tokens / (total_ms * 1e-3)
+    total_ms = max_over_ranks(sum(per_step), dist, dev)
+    value = job_tokens_per_s(world, w.M, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     e2e_ms, h2d, d2h = run_e2e(step, args.e2e_steps)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * w.M / (float(te.item()) * 1e-3)
+    e2e_value = job_tokens_per_s(world, w.M, 1, max_over_ranks(e2e_ms, dist, dev))
 
     if rank == 0:
         peaks = _peaks()
