@@ -97,7 +97,7 @@ def check_one_linear(X_cpu, dY_cpu, lin, L, tag):
 
 
 @pytest.mark.parametrize("name", ["q_proj_8b", "proj_70b_dq", "sweep_m1", "sweep_m16",
-                                  "sweep_m128", "sweep_m16384"])
+                                  "sweep_m128", "sweep_m1024", "sweep_m16384"])
 def test_full_size_workload(name):
     w = synth.workload(name)
     inp = synth.make_inputs(w, seed=0)
