@@ -23,6 +23,7 @@ data path has no exchange step in one forward+backward); the step time is the ma
 """
 
 import argparse
+import copy
 import json
 import math
 import os
@@ -160,6 +161,14 @@ class LinearState:
         self.dB = torch.empty((L.N, L.r), dtype=torch.float32, device=dev)
         self.ws = linear.alloc_workspace(M, L.N, L.K, L.r, dev)
 
+    def twin(self):
+        """The same linear (weights shared) with its own activation, output and scratch
+        buffers, so two steps can be in flight at once."""
+        t = copy.copy(self)
+        for name in ("X", "dY", "H", "XA", "sXA", "dYB", "sdYB", "dX", "dA", "dB", "ws"):
+            setattr(t, name, torch.empty_like(getattr(self, name)))
+        return t
+
     def fwd_stages(self, stream):
         M, L, p = self.M, self.L, lambda t: t.data_ptr()
         ws, wsb = p(self.ws), self.ws.numel()
@@ -222,6 +231,23 @@ class Step:
         self.states = [sg, su, sd]
         self.glue = (sg, su, sd, dg, du)
         self.inputs = [(sg, "X"), (sd, "dY")]
+
+    def twin(self):
+        """A second set of step buffers over the same weights (see LinearState.twin)."""
+        t = copy.copy(self)
+        if self.glue is None:
+            t.states = [st.twin() for st in self.states]
+            t.inputs = [(st, "X") for st in t.states] + [(st, "dY") for st in t.states]
+            return t
+        sg, su, sd, dg, du = (x.twin() if isinstance(x, LinearState) else torch.empty_like(x)
+                              for x in self.glue)
+        t.a = torch.empty_like(self.a)
+        su.X = sg.X
+        sg.dY, su.dY, sd.X = dg, du, t.a
+        t.states = [sg, su, sd]
+        t.glue = (sg, su, sd, dg, du)
+        t.inputs = [(sg, "X"), (sd, "dY")]
+        return t
 
     def stages(self, stream):
         if self.glue is None:
@@ -337,29 +363,52 @@ class GraphStep:
 
 def run_e2e(step, steps):
     """The same metric through the public entry points (qlora_linear_fwd / qlora_linear_bwd, and
-    the SwiGLU glue for the MLP block) with host buffers: each step copies the step's inputs
-    from pinned host memory, runs the layer(s), and copies every result back."""
-    ins = [(st, attr, getattr(st, attr).cpu().pin_memory()) for st, attr in step.inputs]
-    outs = [(t, torch.empty_like(t, device="cpu").pin_memory()) for t in step.outputs()]
-    h2d = sum(h.numel() * h.element_size() for _, _, h in ins)
-    d2h = sum(h.numel() * h.element_size() for _, h in outs)
+    the SwiGLU glue for the MLP block) with host buffers.  Every step copies its inputs from
+    pinned host memory, runs the layer(s) and copies every result back.  Two buffer sets and
+    three streams (copy in, compute, copy out) overlap one step's transfers with the other
+    step's compute, as a training loop feeding the layer from the host would; the time is the
+    whole pipeline's, from the first input copy to the last result copy."""
+    sets = [step, step.twin()]
+    host_in = [getattr(st, attr).cpu().pin_memory() for st, attr in step.inputs]
+    host_out = [[torch.empty_like(t, device="cpu").pin_memory() for t in s.outputs()]
+                for s in sets]
+    h2d = sum(h.numel() * h.element_size() for h in host_in)
+    d2h = sum(h.numel() * h.element_size() for h in host_out[0])
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in sets]
+    ev_comp = [torch.cuda.Event() for _ in sets]
+    ev_out = [torch.cuda.Event() for _ in sets]
 
-    def one():
-        for st, attr, h in ins:
-            getattr(st, attr).copy_(h, non_blocking=True)
-        step.e2e()
-        for t, h in outs:
-            h.copy_(t, non_blocking=True)
+    def one(i):
+        b = i % 2
+        S = sets[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[b])  # step i-2 has finished reading these inputs
+            for (st, attr), h in zip(S.inputs, host_in):
+                getattr(st, attr).copy_(h, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            if i >= 2:
+                s_comp.wait_event(ev_out[b])  # step i-2's results have left these buffers
+            S.e2e()
+            ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            for t, h in zip(S.outputs(), host_out[b]):
+                h.copy_(t, non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(3):
+        one(i)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    a.record(s_in)
+    for i in range(3, 3 + steps):
+        one(i)
+    b.record(s_out)
     torch.cuda.synchronize()
     return a.elapsed_time(b) / steps, h2d, d2h
 
