@@ -205,6 +205,9 @@ __global__ void __launch_bounds__(kThreadsSk) lora_down_kernel(
     cp_async_commit();
   }
   cp_async_wait0();
+  // Let the finalize kernel (launched as a programmatic dependent) be scheduled now; it
+  // still waits for this whole grid's results before reading them.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int r_lo = m0 + warp * 16 + (lane >> 2);
 #pragma unroll
@@ -237,6 +240,7 @@ constexpr int kMaxSplit = 16;
 __global__ void lora_down_finalize(const float* __restrict__ partial, int split, long long n,
                                    float scale, __nv_bfloat16* __restrict__ saved,
                                    __nv_bfloat16* __restrict__ scaled) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the split kernel's partials are done
   const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i4 >= n) return;
   float4 p[kMaxSplit];
@@ -333,6 +337,9 @@ __global__ void __launch_bounds__(kThreadsSk) lora_grad_kernel(
     cp_async_commit();
   }
   cp_async_wait0();
+  // Let the finalize kernel (launched as a programmatic dependent) be scheduled now; it
+  // still waits for this whole grid's results before reading them.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int c_lo = c0 + warp * 16 + (lane >> 2);
 #pragma unroll
@@ -363,6 +370,7 @@ __global__ void __launch_bounds__(kThreadsSk) lora_grad_kernel(
 // Each thread owns 4 consecutive outputs and issues all of its partial loads first.
 __global__ void lora_grad_finalize(const float* __restrict__ partial, int split, int C, int R,
                                    float scale, float* __restrict__ out, int out_cr) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the split kernel's partials are done
   const long long n = static_cast<long long>(C) * R;
   const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i4 >= n) return;
@@ -391,6 +399,25 @@ __global__ void lora_grad_finalize(const float* __restrict__ partial, int split,
     }
   *reinterpret_cast<float4*>(out + i4) =
       make_float4(scale * v.x, scale * v.y, scale * v.z, scale * v.w);
+}
+
+// Launches a 256-thread finalize kernel as a programmatic dependent of the kernel before it on
+// the stream: it may be scheduled while that kernel's last CTAs run and waits for its results
+// with griddepcontrol.wait.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), unsigned blocks, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
 }
 
 int clamp_split(int want, int maxv) { return want < 1 ? 1 : (want > maxv ? maxv : want); }
@@ -481,9 +508,9 @@ cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_b
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.split == 1) return e;
   const long long n = static_cast<long long>(M) * r;
-  lora_down_finalize<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
-      partial, plan.split, n, scale, saved, scaled);
-  return cudaGetLastError();
+  return launch_dependent(lora_down_finalize, static_cast<unsigned>((n / 4 + 255) / 256),
+                          stream, static_cast<const float*>(partial), plan.split, n, scale,
+                          saved, scaled);
 }
 #undef QLORA_DOWN_CASE
 
@@ -524,9 +551,9 @@ cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.split == 1) return e;
   const long long n = static_cast<long long>(C) * r;
-  lora_grad_finalize<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
-      partial, plan.split, C, r, scale, out, out_cr ? 1 : 0);
-  return cudaGetLastError();
+  return launch_dependent(lora_grad_finalize, static_cast<unsigned>((n / 4 + 255) / 256),
+                          stream, static_cast<const float*>(partial), plan.split, C, r, scale,
+                          out, out_cr ? 1 : 0);
 }
 #undef QLORA_GRAD_CASE
 
