@@ -112,7 +112,11 @@ QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
 /* Forward.  X [M, K], A [r, K], B [N, r] bf16 device (read); H [M, N] bf16 device (written);
  * XA_saved [M, r] bf16 device (written: X A^T rounded to bf16, kept for the backward).
  * ws: device scratch of at least qlora_workspace_bytes(M, N, K, r) bytes.
- * alpha: LoRA alpha; s = alpha / r.  r must be a multiple of 8 in [8, 128]. */
+ * alpha: LoRA alpha; s = alpha / r.  r must be a multiple of 8 in [8, 128].
+ * For M <= 32 the base product applies each block's absmax to the block's 64-deep partial sum
+ * (the weight enters as bf16(code value) * absmax rather than bf16(code value * absmax)); the
+ * two agree within one bf16 rounding of the weight.  Larger M and dX use the dequantised
+ * bf16 weight exactly as qlora_nf4_dequant returns it. */
 QLORA_API qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
                               const void* B, int M, int r, float alpha, void* H, void* XA_saved,
                               void* ws, size_t ws_bytes, qlora_stream_t stream);
