@@ -67,11 +67,15 @@ def weight_stream_bytes(L):
     return nk // 2 + 4 * (nk // 64)
 
 
-def gemm_work(L, M, trans):
-    """(flops, min HBM bytes) of one dequant GEMM launch (forward or dX)."""
+def gemm_work(L, M, trans, n_groups=1):
+    """(flops, min HBM bytes) of one dequant GEMM launch (forward or dX).  With n adapters
+    packed along W0's rows, every output row of the forward takes r extension columns and the
+    dX extension runs over all n r."""
     red, rows = (L.N, L.K) if trans else (L.K, L.N)
-    flops = 2.0 * M * L.N * L.K + 2.0 * M * rows * L.r
-    byts = weight_stream_bytes(L) + 2 * M * red + 2 * M * rows + 2 * M * L.r + 2 * rows * L.r
+    r_row = L.r * n_groups if trans else L.r
+    flops = 2.0 * M * L.N * L.K + 2.0 * M * rows * r_row
+    byts = (weight_stream_bytes(L) + 2 * M * red + 2 * M * rows + 2 * M * L.r * n_groups
+            + 2 * rows * r_row)
     return flops, byts
 
 
@@ -141,10 +145,14 @@ class ClockSampler:
 class LinearState:
     """Device buffers of one QLoRA linear on M tokens, and its timed stages: forward
     (lora_down, dequant GEMM) and backward (lora_down, dequant GEMM for dX, lora_grad x 2).
-    X and dY may be buffers shared with other stages (the MLP block chains them)."""
+    X and dY may be buffers shared with other stages (the MLP block chains them).  With
+    `groups` (adapter row counts) the linear is a packed-adapter layer: L.N is the stacked
+    weight's rows, L.r each adapter's rank, A [n r, K] and B [N, r] stacked by adapter."""
 
-    def __init__(self, L, M, X, dY, W0, A, B, dev):
+    def __init__(self, L, M, X, dY, W0, A, B, dev, groups=None):
         self.L, self.M = L, M
+        self.groups = list(groups) if groups else None
+        self.R = L.r * (len(self.groups) if self.groups else 1)  # packed rank columns
         self.X, self.dY = X.to(dev), dY.to(dev)
         self.A, self.B = A.to(dev), B.to(dev)
         self.w = linear.nf4_pack(W0.to(dev), double_quant=L.double_quant)
@@ -152,14 +160,14 @@ class LinearState:
         self.s = L.alpha / L.r
         bf = dict(dtype=torch.bfloat16, device=dev)
         self.H = torch.empty((M, L.N), **bf)
-        self.XA = torch.empty((M, L.r), **bf)
-        self.sXA = torch.empty((M, L.r), **bf)
-        self.dYB = torch.empty((M, L.r), **bf)
-        self.sdYB = torch.empty((M, L.r), **bf)
+        self.XA = torch.empty((M, self.R), **bf)
+        self.sXA = torch.empty((M, self.R), **bf)
+        self.dYB = torch.empty((M, self.R), **bf)
+        self.sdYB = torch.empty((M, self.R), **bf)
         self.dX = torch.empty((M, L.K), **bf)
-        self.dA = torch.empty((L.r, L.K), dtype=torch.float32, device=dev)
+        self.dA = torch.empty((self.R, L.K), dtype=torch.float32, device=dev)
         self.dB = torch.empty((L.N, L.r), dtype=torch.float32, device=dev)
-        self.ws = linear.alloc_workspace(M, L.N, L.K, L.r, dev)
+        self.ws = linear.alloc_workspace(M, L.N, L.K, self.R, dev)
 
     def twin(self):
         """The same linear (weights shared) with its own activation, output and scratch
@@ -170,45 +178,89 @@ class LinearState:
         return t
 
     def fwd_stages(self, stream):
-        M, L, p = self.M, self.L, lambda t: t.data_ptr()
+        M, L, R, g, p = self.M, self.L, self.R, self.groups, lambda t: t.data_ptr()
         ws, wsb = p(self.ws), self.ws.numel()
         n = L.name
         return [
             (f"{n}.lora_down_fwd",
-             lambda: abi.qlora_lora_down(p(self.X), M, L.K, p(self.A), 1, L.r, self.s,
+             lambda: abi.qlora_lora_down(p(self.X), M, L.K, p(self.A), 1, R, None, self.s,
                                          p(self.XA), p(self.sXA), ws, wsb, stream)),
             (f"{n}.gemm_fwd",
              lambda: abi.qlora_nf4_gemm(p(self.X), self.cw, 0, p(self.B), p(self.sXA), M, L.r,
-                                        p(self.H), ws, wsb, stream)),
+                                        g, p(self.H), ws, wsb, stream)),
         ]
 
     def bwd_stages(self, stream):
-        M, L, p = self.M, self.L, lambda t: t.data_ptr()
+        M, L, R, g, p = self.M, self.L, self.R, self.groups, lambda t: t.data_ptr()
         ws, wsb = p(self.ws), self.ws.numel()
         n = L.name
         return [
             (f"{n}.lora_down_bwd",
-             lambda: abi.qlora_lora_down(p(self.dY), M, L.N, p(self.B), 0, L.r, self.s,
+             lambda: abi.qlora_lora_down(p(self.dY), M, L.N, p(self.B), 0, R, g, self.s,
                                          p(self.dYB), p(self.sdYB), ws, wsb, stream)),
             (f"{n}.gemm_dx",
-             lambda: abi.qlora_nf4_gemm(p(self.dY), self.cw, 1, p(self.A), p(self.sdYB), M, L.r,
-                                        p(self.dX), ws, wsb, stream)),
+             lambda: abi.qlora_nf4_gemm(p(self.dY), self.cw, 1, p(self.A), p(self.sdYB), M, R,
+                                        None, p(self.dX), ws, wsb, stream)),
             (f"{n}.lora_grad_dB",
-             lambda: abi.qlora_lora_grad(p(self.dY), M, L.N, p(self.XA), L.r, self.s,
+             lambda: abi.qlora_lora_grad(p(self.dY), M, L.N, p(self.XA), L.r, g, self.s,
                                          p(self.dB), 0, ws, wsb, stream)),
             (f"{n}.lora_grad_dA",
-             lambda: abi.qlora_lora_grad(p(self.X), M, L.K, p(self.dYB), L.r, self.s,
+             lambda: abi.qlora_lora_grad(p(self.X), M, L.K, p(self.dYB), R, None, self.s,
                                          p(self.dA), 1, ws, wsb, stream)),
         ]
+
+    def forward(self):
+        """The layer's forward through the public Python entry points."""
+        if self.groups:
+            linear.grouped_forward(self.X, self.w, self.A, self.B, self.groups, self.L.alpha,
+                                   H=self.H, XA=self.XA, ws=self.ws)
+        else:
+            linear.forward(self.X, self.w, self.A, self.B, self.L.alpha, H=self.H, XA=self.XA,
+                           ws=self.ws)
+
+    def backward(self):
+        if self.groups:
+            linear.grouped_backward(self.dY, self.X, self.w, self.A, self.B, self.XA,
+                                    self.groups, self.L.alpha, dX=self.dX, dA=self.dA,
+                                    dB=self.dB, ws=self.ws)
+        else:
+            linear.backward(self.dY, self.X, self.w, self.A, self.B, self.XA, self.L.alpha,
+                            dX=self.dX, dA=self.dA, dB=self.dB, ws=self.ws)
 
 
 class Step:
     """One step of a workload: its linears' states and the ordered (name, call) stages."""
 
-    def __init__(self, w, dev, seed):
+    def __init__(self, w, dev, seed, unpacked=False):
         self.w = w
+        self.share_x = False
         inp = synth.make_inputs(w, seed=seed)
         bf = dict(dtype=torch.bfloat16, device=dev)
+        if w.grouped:
+            # Adapters sharing X: one packed-adapter layer (stacked W0, A, B), or, unpacked,
+            # one layer per adapter on the same X with its own column block of dY.
+            Ls, lins = w.linears, inp["linears"]
+            Ns = [L.N for L in Ls]
+            self.glue = None
+            if unpacked:
+                edges = np.cumsum([0] + Ns)
+                self.states = [LinearState(L, w.M, inp["X"],
+                                           inp["dY"][:, edges[i]:edges[i + 1]].contiguous(),
+                                           d["W0"], d["A"], d["B"], dev)
+                               for i, (L, d) in enumerate(zip(Ls, lins))]
+                self.share_x = True
+                for st in self.states[1:]:
+                    st.X = self.states[0].X
+            else:
+                L0 = Ls[0]
+                Lp = synth.LinearShape("+".join(L.name for L in Ls), L0.K, sum(Ns), L0.r,
+                                       L0.alpha, L0.w_std, L0.double_quant)
+                self.states = [LinearState(Lp, w.M, inp["X"], inp["dY"],
+                                           torch.cat([d["W0"] for d in lins]),
+                                           torch.cat([d["A"] for d in lins]),
+                                           torch.cat([d["B"] for d in lins]), dev, groups=Ns)]
+            self.inputs = self._inputs(self.states)
+            return
         if not w.mlp:
             self.states = [LinearState(L, w.M, d["X"], d["dY"], d["W0"], d["A"], d["B"], dev)
                            for L, d in zip(w.linears, inp["linears"])]
@@ -237,7 +289,10 @@ class Step:
         t = copy.copy(self)
         if self.glue is None:
             t.states = [st.twin() for st in self.states]
-            t.inputs = [(st, "X") for st in t.states] + [(st, "dY") for st in t.states]
+            if self.share_x:
+                for st in t.states[1:]:
+                    st.X = t.states[0].X
+            t.inputs = t._inputs(t.states)
             return t
         sg, su, sd, dg, du = (x.twin() if isinstance(x, LinearState) else torch.empty_like(x)
                               for x in self.glue)
@@ -248,6 +303,10 @@ class Step:
         t.glue = (sg, su, sd, dg, du)
         t.inputs = [(sg, "X"), (sd, "dY")]
         return t
+
+    def _inputs(self, states):
+        xs = states[:1] if self.share_x else states
+        return [(st, "X") for st in xs] + [(st, "dY") for st in states]
 
     def stages(self, stream):
         if self.glue is None:
@@ -271,9 +330,8 @@ class Step:
         SwiGLU glue), on the device buffers already holding this step's inputs."""
         if self.glue is None:
             for st in self.states:
-                linear.forward(st.X, st.w, st.A, st.B, st.L.alpha, H=st.H, XA=st.XA, ws=st.ws)
-                linear.backward(st.dY, st.X, st.w, st.A, st.B, st.XA, st.L.alpha, dX=st.dX,
-                                dA=st.dA, dB=st.dB, ws=st.ws)
+                st.forward()
+                st.backward()
             return
         sg, su, sd, dg, du = self.glue
         for st in (sg, su):
@@ -443,14 +501,16 @@ def roofline(step, per_stage, peaks, workload):
         flops, byts = 0.0, (3 if stage == "fwd" else 5) * 2 * n
     else:
         st = next(s for s in step.states if s.L.name == lin_name)
+        M, L, R = st.M, st.L, st.R  # R: packed rank columns (r for a single adapter)
         if stage.startswith("gemm"):
-            flops, byts = gemm_work(st.L, st.M, stage == "gemm_dx")
+            flops, byts = gemm_work(L, M, stage == "gemm_dx", R // L.r)
         elif stage.startswith("lora_down"):
-            C = st.L.K if stage.endswith("fwd") else st.L.N
-            flops, byts = 2.0 * st.M * C * st.L.r, 2 * st.M * C + 4 * st.M * st.L.r
+            # X A^T: every input column feeds R outputs; dY B: each feeds its adapter's r.
+            C, per = (L.K, R) if stage.endswith("fwd") else (L.N, L.r)
+            flops, byts = 2.0 * M * C * per, 2 * M * C + 4 * M * R
         else:
-            C = st.L.N if stage.endswith("dB") else st.L.K
-            flops, byts = 2.0 * st.M * C * st.L.r, 2 * st.M * C + 4 * C * st.L.r
+            C, per = (L.N, L.r) if stage.endswith("dB") else (L.K, R)
+            flops, byts = 2.0 * M * C * per, 2 * M * C + 2 * M * R + 4 * C * per
     ai = flops / byts
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if stage.startswith("gemm") and ai >= ridge:
@@ -494,13 +554,19 @@ def oracle_prepare(w, seed):
 
 def oracle_rows(w, prep, n):
     """Seconds the fp64 oracle takes for forward + backward on the first n token rows of the
-    workload (for the MLP block: gate/up, SwiGLU, down, and back)."""
+    workload (for the MLP block: gate/up, SwiGLU, down, and back; for packed adapters the
+    packed layer)."""
     from oracle import qlora  # test infrastructure: only here and in the reference arm
     inp, Wds, _ = prep
     f64 = lambda t: t.float().numpy().astype(np.float64)
     lora = [(f64(d["A"]), f64(d["B"])) for d in inp["linears"]]
     t0 = time.perf_counter()
-    if not w.mlp:
+    if w.grouped:
+        X, dY = f64(inp["X"][:n]), f64(inp["dY"][:n])
+        As, Bs = [A for A, _ in lora], [B for _, B in lora]
+        qlora.grouped_forward(X, Wds, As, Bs, w.linears[0].alpha)
+        qlora.grouped_backward(dY, X, Wds, As, Bs, w.linears[0].alpha)
+    elif not w.mlp:
         for L, d, Wd, (A, B) in zip(w.linears, inp["linears"], Wds, lora):
             X, dY = f64(d["X"][:n]), f64(d["dY"][:n])
             qlora.forward(X, Wd, A, B, L.alpha)
@@ -571,11 +637,14 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w):
+def workload_config(w, unpacked=False):
     c = {"workload": w.name, "M": w.M,
          "linears": [{"name": L.name, "K": L.K, "N": L.N, "r": L.r, "alpha": L.alpha,
                       "absmax": "double-quant" if L.double_quant else "fp32"} for L in w.linears],
          "l2": "flushed before every step (256 MiB write + read, outside the events)", "parallelism": "replicas"}
+    if w.grouped:
+        c["adapters"] = ("unpacked: one layer per adapter on the shared input" if unpacked else
+                         "packed: one stacked NF4 weight, adapters along its rows, shared input")
     return c
 
 
@@ -608,6 +677,8 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="launch every stage from Python instead of replaying a CUDA graph")
+    ap.add_argument("--unpacked", action="store_true",
+                    help="adapters sharing an input (qkv_8b) run as separate layers")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -629,7 +700,7 @@ def main():
                                 device_id=dev)
 
     w = synth.workload(args.workload)
-    step = Step(w, dev, seed=rank)
+    step = Step(w, dev, seed=rank, unpacked=args.unpacked)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
@@ -692,7 +763,7 @@ def main():
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) W0 packed to NF4, random LoRA)",
-            "config": workload_config(w),
+            "config": workload_config(w, args.unpacked),
             "tflops": round(tflops, 2),
             "tflops_frac_of_peak": round(tflops / peaks["bf16_tflops"], 4),
             "stages_ms": {k: round(statistics.mean(v), 5) for k, v in per_stage.items()},

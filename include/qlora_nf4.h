@@ -129,6 +129,37 @@ QLORA_API qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlo
                               float alpha, void* dX, float* dA, float* dB, void* ws,
                               size_t ws_bytes, qlora_stream_t stream);
 
+/* ---- Several adapters packed into one launch sequence. ----
+ * n adapters share the input X and own consecutive row ranges of one stacked base weight:
+ * q/k/v projections, or gate/up ("Speed Up Fine-Tuning 2x with Unsloth on Llama and Mistral",
+ * "How it works internally", item 3: several LoRA adapters packed into a single tensor;
+ * "Unsloth vs QLoRA vs Liger-Kernel", section 5, step 2: adapters on q/k/v/o/gate/up/down).
+ * Adapter g has N_g = group_rows[g] output rows (host array of n_groups ints) and rank r; all
+ * share alpha, so s = alpha / r.  Layouts (bf16 unless noted, all device):
+ *   W        NF4 [N, K], N = sum N_g: the adapters' base weights stacked by rows (pack the
+ *            stacked bf16 weight with qlora_nf4_pack);
+ *   A        [n r, K]: A_0, A_1, ... stacked by rows;      B  [N, r]: B_0, B_1, ... by rows;
+ *   H, dY    [M, N]: adapter g's outputs in columns [sum_{i<g} N_i, sum_{i<=g} N_i);
+ *   XA_saved [M, n r]: X A_g^T in columns [g r, (g + 1) r);
+ *   dA       [n r, K] fp32 (rows of A_g at g r);          dB [N, r] fp32 (rows of B_g).
+ * The results equal n separate qlora_linear_fwd / qlora_linear_bwd calls on the slices, with
+ * dX their sum; X is read once for all adapters' down-projections, and each large product is
+ * one launch over all adapters' rows.  Requirements: 1 <= n_groups <= 8; r and n r multiples
+ * of 8 in [8, 128]; every N_g a multiple of 128 (of 64 when n_groups = 1); sum N_g = W->N.
+ * Violations return QLORA_ERR_SHAPE (QLORA_ERR_NULL for a NULL group_rows). */
+QLORA_API size_t qlora_grouped_workspace_bytes(int M, int N, int K, int r, int n_groups);
+
+QLORA_API qlora_status qlora_grouped_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
+                               const void* B, const int* group_rows, int n_groups, int M, int r,
+                               float alpha, void* H, void* XA_saved, void* ws, size_t ws_bytes,
+                               qlora_stream_t stream);
+
+QLORA_API qlora_status qlora_grouped_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
+                               const void* A, const void* B, const void* XA_saved,
+                               const int* group_rows, int n_groups, int M, int r, float alpha,
+                               void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                               qlora_stream_t stream);
+
 /* SwiGLU glue for the MLP workload: a = g * sigmoid(g) * u (elementwise, n elements, bf16
  * device), and its exact backward dg = da*u*sig(g)*(1 + g*(1 - sig(g))), du = da*g*sig(g).
  * Computed in fp32, rounded to bf16.  ("Unsloth vs QLoRA vs Liger-Kernel", section 2: the
@@ -140,34 +171,44 @@ QLORA_API qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void
 
 /* ---- The stages the two linear entry points are composed of (same validation rules). ---- */
 
-/* Rank-r down-projection: out = in . Wl^T with in [M, C] bf16 and Wl given either as
+/* The stage calls take an optional adapter split, `group_rows` (host array of n_groups row
+ * counts, with the rules of the packed-adapter entry points) or NULL for a single adapter.
+ *
+ * Rank-r down-projection: out = in . Wl^T with in [M, C] bf16 and Wl given either as
  * w [r, C] (w_is_r_by_c = 1, the LoRA A) or as w [C, r] (w_is_r_by_c = 0, the LoRA B).
  * Writes bf16(out) to `saved` [M, r] (may be NULL) and bf16(scale * out) to `scaled` [M, r].
+ * With group_rows (w_is_r_by_c = 0 only): r = n r_g output columns, w = B [C, r_g] stacked by
+ * adapter, and Wl is block-diagonal: rows of adapter g feed columns g r_g .. g r_g + r_g - 1.
  * ws: device scratch of at least qlora_workspace_bytes(M, C, C, r) bytes. */
 QLORA_API qlora_status qlora_lora_down(const void* in, int M, int C, const void* w,
-                                       int w_is_r_by_c, int r, float scale, void* saved,
-                                       void* scaled, void* ws, size_t ws_bytes,
-                                       qlora_stream_t stream);
+                                       int w_is_r_by_c, int r, const int* group_rows,
+                                       int n_groups, float scale, void* saved, void* scaled,
+                                       void* ws, size_t ws_bytes, qlora_stream_t stream);
 
 /* The dequant GEMM with the fused rank-r extension:
  *   transpose_w = 0: out[M, N] = act[M, K] . deq(W0)^T + ext_act[M, r] . ext_w^T, ext_w = B [N, r]
  *   transpose_w = 1: out[M, K] = act[M, N] . deq(W0)   + ext_act[M, r] . ext_w,   ext_w = A [r, K]
  * act, ext_w, ext_act bf16 device (read); out bf16 device (written).  The scale s is expected
  * to be folded into ext_act already (qlora_lora_down's `scaled` output).
+ * With group_rows (transpose_w = 0 only): ext_act is [M, n r] and output row n of adapter g
+ * takes ext_act's columns g r .. g r + r - 1; ext_w = B [N, r] stacked by adapter.
  * ws: device scratch for the partial sums of problems with fewer output tiles (128 output
  * features x up to 512 tokens) than SMs, which are cut along the reduction so every SM works;
  * at least qlora_workspace_bytes(M, N, K, r) bytes (may be NULL when that shape needs none). */
 QLORA_API qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
                                       const void* ext_w, const void* ext_act, int M, int r,
-                                      void* out, void* ws, size_t ws_bytes,
-                                      qlora_stream_t stream);
+                                      const int* group_rows, int n_groups, void* out, void* ws,
+                                      size_t ws_bytes, qlora_stream_t stream);
 
 /* Rank-r weight gradient: G[c, j] = scale * sum_m big[m, c] small[m, j] with big [M, C] and
  * small [M, r] bf16 device; written fp32 as out [C, r] (out_r_by_c = 0, e.g. dB) or
- * out [r, C] (out_r_by_c = 1, e.g. dA).  ws: at least qlora_workspace_bytes(M, C, C, r). */
+ * out [r, C] (out_r_by_c = 1, e.g. dA).  With group_rows (adapters along big's columns):
+ * small is [M, n r] and column c of adapter g uses small[m, g r + j].
+ * ws: at least qlora_workspace_bytes(M, C, C, r). */
 QLORA_API qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, int r,
-                                       float scale, float* out, int out_r_by_c, void* ws,
-                                       size_t ws_bytes, qlora_stream_t stream);
+                                       const int* group_rows, int n_groups, float scale,
+                                       float* out, int out_r_by_c, void* ws, size_t ws_bytes,
+                                       qlora_stream_t stream);
 
 /* Number of kernels this library has launched in this process so far (all devices). */
 QLORA_API uint64_t qlora_launch_counter(void);

@@ -29,6 +29,9 @@ EXPORTS = (
     "qlora_linear_fwd_noalloc",
     "qlora_noalloc_scratch_bytes",
     "qlora_device_error",
+    "qlora_grouped_workspace_bytes",
+    "qlora_grouped_fwd",
+    "qlora_grouped_bwd",
 )
 
 STATUS = {
@@ -83,15 +86,24 @@ def _lib():
                                       _F, _VP, _VP, _VP, _VP, _SZ, _VP]),
             "qlora_swiglu_fwd": (_I, [_VP, _VP, _VP, _I64, _VP]),
             "qlora_swiglu_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _VP]),
-            "qlora_lora_down": (_I, [_VP, _I, _I, _VP, _I, _I, _F, _VP, _VP, _VP, _SZ, _VP]),
-            "qlora_nf4_gemm": (_I, [_VP, ctypes.POINTER(Nf4Weight), _I, _VP, _VP, _I, _I, _VP,
-                                    _VP, _SZ, _VP]),
-            "qlora_lora_grad": (_I, [_VP, _I, _I, _VP, _I, _F, _VP, _I, _VP, _SZ, _VP]),
+            "qlora_lora_down": (_I, [_VP, _I, _I, _VP, _I, _I, ctypes.POINTER(_I), _I, _F, _VP,
+                                     _VP, _VP, _SZ, _VP]),
+            "qlora_nf4_gemm": (_I, [_VP, ctypes.POINTER(Nf4Weight), _I, _VP, _VP, _I, _I,
+                                    ctypes.POINTER(_I), _I, _VP, _VP, _SZ, _VP]),
+            "qlora_lora_grad": (_I, [_VP, _I, _I, _VP, _I, ctypes.POINTER(_I), _I, _F, _VP, _I,
+                                     _VP, _SZ, _VP]),
             "qlora_launch_counter": (ctypes.c_uint64, []),
             "qlora_linear_fwd_noalloc": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _I, _I,
                                               _F, _VP, _VP, _VP]),
             "qlora_noalloc_scratch_bytes": (_SZ, []),
             "qlora_device_error": (_I, [ctypes.POINTER(ctypes.c_int)]),
+            "qlora_grouped_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+            "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
+                                       ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
+                                       _VP]),
+            "qlora_grouped_bwd": (_I, [_VP, _VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _VP,
+                                       ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _VP,
+                                       _SZ, _VP]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -144,6 +156,31 @@ def qlora_linear_bwd(dY, X, weight, A, B, XA_saved, M, r, alpha, dX, dA, dB, ws,
                                                        ws, ws_bytes, stream))
 
 
+def _int_array(values):
+    values = [int(v) for v in values]
+    return (_I * max(len(values), 1))(*values), len(values)
+
+
+def qlora_grouped_workspace_bytes(M, N, K, r, n_groups):
+    return int(_lib().qlora_grouped_workspace_bytes(M, N, K, r, n_groups))
+
+
+def qlora_grouped_fwd(X, weight, A, B, group_rows, M, r, alpha, H, XA_saved, ws, ws_bytes,
+                      stream):
+    rows, n = _int_array(group_rows)
+    _check("qlora_grouped_fwd", _lib().qlora_grouped_fwd(X, ctypes.byref(weight), A, B, rows, n,
+                                                         M, r, float(alpha), H, XA_saved, ws,
+                                                         ws_bytes, stream))
+
+
+def qlora_grouped_bwd(dY, X, weight, A, B, XA_saved, group_rows, M, r, alpha, dX, dA, dB, ws,
+                      ws_bytes, stream):
+    rows, n = _int_array(group_rows)
+    _check("qlora_grouped_bwd", _lib().qlora_grouped_bwd(dY, X, ctypes.byref(weight), A, B,
+                                                         XA_saved, rows, n, M, r, float(alpha),
+                                                         dX, dA, dB, ws, ws_bytes, stream))
+
+
 def qlora_swiglu_fwd(g, u, a, n, stream):
     _check("qlora_swiglu_fwd", _lib().qlora_swiglu_fwd(g, u, a, n, stream))
 
@@ -152,21 +189,34 @@ def qlora_swiglu_bwd(g, u, da, dg, du, n, stream):
     _check("qlora_swiglu_bwd", _lib().qlora_swiglu_bwd(g, u, da, dg, du, n, stream))
 
 
-def qlora_lora_down(inp, M, C, w, w_is_r_by_c, r, scale, saved, scaled, ws, ws_bytes, stream):
-    _check("qlora_lora_down", _lib().qlora_lora_down(inp, M, C, w, int(w_is_r_by_c), r,
+def _groups(group_rows):
+    """(int array or None, n) for an optional list of adapter row counts."""
+    if group_rows is None:
+        return None, 0
+    return _int_array(group_rows)
+
+
+def qlora_lora_down(inp, M, C, w, w_is_r_by_c, r, group_rows, scale, saved, scaled, ws, ws_bytes,
+                    stream):
+    rows, n = _groups(group_rows)
+    _check("qlora_lora_down", _lib().qlora_lora_down(inp, M, C, w, int(w_is_r_by_c), r, rows, n,
                                                      float(scale), saved, scaled, ws, ws_bytes,
                                                      stream))
 
 
-def qlora_nf4_gemm(act, weight, transpose_w, ext_w, ext_act, M, r, out, ws, ws_bytes, stream):
+def qlora_nf4_gemm(act, weight, transpose_w, ext_w, ext_act, M, r, group_rows, out, ws, ws_bytes,
+                   stream):
+    rows, n = _groups(group_rows)
     _check("qlora_nf4_gemm", _lib().qlora_nf4_gemm(act, ctypes.byref(weight), int(transpose_w),
-                                                   ext_w, ext_act, M, r, out, ws, ws_bytes,
-                                                   stream))
+                                                   ext_w, ext_act, M, r, rows, n, out, ws,
+                                                   ws_bytes, stream))
 
 
-def qlora_lora_grad(big, M, C, small, r, scale, out, out_r_by_c, ws, ws_bytes, stream):
-    _check("qlora_lora_grad", _lib().qlora_lora_grad(big, M, C, small, r, float(scale), out,
-                                                     int(out_r_by_c), ws, ws_bytes, stream))
+def qlora_lora_grad(big, M, C, small, r, group_rows, scale, out, out_r_by_c, ws, ws_bytes,
+                    stream):
+    rows, n = _groups(group_rows)
+    _check("qlora_lora_grad", _lib().qlora_lora_grad(big, M, C, small, r, rows, n, float(scale),
+                                                     out, int(out_r_by_c), ws, ws_bytes, stream))
 
 
 def qlora_launch_counter():

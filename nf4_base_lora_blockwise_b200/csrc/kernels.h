@@ -11,6 +11,30 @@
 
 namespace qlora {
 
+// ------------------------------ adapters packed along the output rows -----------------------
+// A stacked base weight [sum N_g, K] whose rows are split into n adapters (q/k/v, gate/up):
+// adapter g owns rows [end[g-1], end[g]) and columns [g r, (g + 1) r) of the packed rank-r
+// activations ([M, n r]: X A_cat^T, dY B_bd).  Every end is a multiple of 128, so no 128-row
+// tile of any kernel straddles two adapters.  n = 1 is the plain single-adapter layer.
+constexpr int kMaxGroups = 8;
+struct RowGroups {
+  int n;
+  int end[kMaxGroups];
+};
+// Adapter owning `row` (static indices only, so a kernel parameter stays in the constant bank).
+__host__ __device__ __forceinline__ int row_group(const RowGroups& g, int row) {
+  int i = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxGroups - 1; ++j) i += (j + 1 < g.n && row >= g.end[j]) ? 1 : 0;
+  return i;
+}
+inline RowGroups single_group(int rows) {
+  RowGroups g = {};
+  g.n = 1;
+  g.end[0] = rows;
+  return g;
+}
+
 // ------------------------------ NF4 pack / dequant -----------------------------------------
 cudaError_t launch_nf4_pack(const __nv_bfloat16* W, int N, int K, int dq, uint8_t* q,
                             float* absmax, uint8_t* absmax_q8, float* absmax_scale,
@@ -42,6 +66,7 @@ struct GemmArgs {
   int* err;        // device error word
   float* partial;  // stream-K partial sums [grid][2][tile tokens][128] fp32 (workspace)
   int streamk;     // set by the launcher
+  RowGroups groups;  // forward: the adapter of each row tile selects its slice of ext_act
   Codebook cb;
 };
 
@@ -49,7 +74,7 @@ struct GemmMaps {
   CUtensorMap act;      // [M, red] bf16, box {64, bt}, 128B swizzle
   CUtensorMap q;        // [N, K/2] u8
   CUtensorMap ext_w;    // B_lora [N, r] (fwd) or A_lora [r, K] (dX), bf16
-  CUtensorMap ext_act;  // scaled rank-r activation [M, r] bf16, box {64, bt}
+  CUtensorMap ext_act;  // scaled rank-r activation [M, n, r] bf16 (n adapters), box {64, 1, bt}
 };
 
 // Work schedule of one launch: whole tiles (one CTA per tile, at most one per SM) or, with
@@ -76,8 +101,9 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
                               size_t partial_floats_avail, cudaStream_t stream, int* launched);
 
 // ------------------------------ few-token forward (mma.sync, register-direct) ---------------
-// h[M, N] = X[M, K] . deq(W0)^T + ext_act[M, r] . ext_w[N, r]^T for M <= 32: stream-K over
-// (128-row tile, 64-block) units with fp32 partial slots and a fixed-order finalize.
+// h[M, N] = X[M, K] . deq(W0)^T + ext_act[M, g(n), r] . ext_w[N, r]^T for M <= 32 (g(n) the
+// adapter of row n): stream-K over (128-row tile, 64-block) units with fp32 partial slots and
+// a fixed-order finalize.
 struct GemvPlan {
   int tt;                 // token tiles of 8
   long long units;
@@ -91,34 +117,38 @@ GemvPlan gemv_plan(int M, int N, int K, int sm_count);
 cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const float* absmax,
                                 const uint8_t* absmax_q8, const float* absmax_scale, int dq, int M,
                                 int N, int K, const __nv_bfloat16* ext_act,
-                                const __nv_bfloat16* ext_w, int r, __nv_bfloat16* out,
-                                float* partial, size_t partial_floats, const Codebook& cb,
-                                cudaStream_t stream);
+                                const __nv_bfloat16* ext_w, int r, const RowGroups& groups,
+                                __nv_bfloat16* out, float* partial, size_t partial_floats,
+                                const Codebook& cb, cudaStream_t stream);
 
 // ------------------------------ rank-r skinny products (mma.sync) --------------------------
 // out[m, j] = sum_c in[m, c] * Wl(j, c); Wl(j, c) = w[j * C + c] (w_is_rc = true, i.e. A [r, C])
 // or w[c * r + j] (w_is_rc = false, i.e. B [C, r]).  Writes bf16 RN(v) to `saved` (if not
 // null) and bf16 RN(scale * v) to `scaled`.  `partial` is fp32 scratch [split, M, r].
+// With w_is_rc = false and groups.n > 1, r = n r_g and w is B_cat [C, r_g]: Wl is the
+// block-diagonal matrix with Wl(g r_g + j, c) = w[c * r_g + j] for the rows c of adapter g and
+// zero elsewhere; the zero blocks are neither loaded nor multiplied.
 struct DownPlan {
   int split;
   size_t partial_floats;
 };
 DownPlan lora_down_plan(int M, int C, int r);
 cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_bfloat16* w,
-                             bool w_is_rc, int r, float scale, __nv_bfloat16* saved,
-                             __nv_bfloat16* scaled, float* partial, const DownPlan& plan,
-                             cudaStream_t stream);
+                             bool w_is_rc, int r, const RowGroups& groups, float scale,
+                             __nv_bfloat16* saved, __nv_bfloat16* scaled, float* partial,
+                             const DownPlan& plan, cudaStream_t stream);
 
-// G[c, j] = scale * sum_m big[m, c] * small[m, j]; written as out[c * r + j] (out_cr) or
-// out[j * C + c].  `partial` is fp32 scratch [split, C, r].
+// G[c, j] = scale * sum_m big[m, c] * small[m, g(c) r + j]; written as out[c * r + j] (out_cr)
+// or out[j * C + c].  small is [M, groups.n r]; g(c) is the adapter of column c (0 for
+// groups.n = 1).  `partial` is fp32 scratch [split, C, r].
 struct GradPlan {
   int split;
   size_t partial_floats;
 };
 GradPlan lora_grad_plan(int M, int C, int r);
 cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_bfloat16* small,
-                             int r, float scale, float* out, bool out_cr, float* partial,
-                             const GradPlan& plan, cudaStream_t stream);
+                             int r, const RowGroups& groups, float scale, float* out, bool out_cr,
+                             float* partial, const GradPlan& plan, cudaStream_t stream);
 
 // ------------------------------ SwiGLU ------------------------------------------------------
 cudaError_t launch_swiglu_fwd(const __nv_bfloat16* g, const __nv_bfloat16* u, __nv_bfloat16* a,

@@ -5,6 +5,10 @@
 //   lora_down:  out[M, r] = in[M, C] . Wl^T      XA = X A^T (forward, kept for the backward)
 //                                                dYB = dY B (backward)
 //   lora_grad:  G[C, r]   = s in[M, C]^T . small[M, r]   dB = s dY^T XA,  dA = s (dYB^T X)
+// With n adapters packed along the rows of B (q/k/v sharing X), dY B takes the block-diagonal
+// B (adapter g's rows feed columns g r_g .. g r_g + r_g - 1 only) and dB takes, for adapter
+// g's rows, the columns g r_g .. of XA.  Every 64-row step and 128-column tile lies in one
+// adapter, so the zero blocks are skipped, not multiplied.
 // ("Unsloth vs QLoRA vs Liger-Kernel", section 1 forward formula, section 2 hand-derived
 // backward.)  Long reductions are split across CTAs into fixed-order fp32 partials that a
 // second kernel sums in order, so results are deterministic run to run.
@@ -132,8 +136,8 @@ __device__ __forceinline__ void load_b_frags(uint32_t (&b)[NT][2], const __nv_bf
 template <int NT, bool kWrc>
 __global__ void __launch_bounds__(kThreadsSk) lora_down_kernel(
     const __nv_bfloat16* __restrict__ in, int M, int C, const __nv_bfloat16* __restrict__ w,
-    float scale, __nv_bfloat16* __restrict__ saved, __nv_bfloat16* __restrict__ scaled,
-    float* __restrict__ partial, int split) {
+    int rg, const RowGroups groups, float scale, __nv_bfloat16* __restrict__ saved,
+    __nv_bfloat16* __restrict__ scaled, float* __restrict__ partial, int split) {
   constexpr int R = NT * 8;
   constexpr int S = stages_for(R);
   constexpr int kInLd = kBC + kPad;
@@ -167,11 +171,14 @@ __global__ void __launch_bounds__(kThreadsSk) lora_down_kernel(
         cp_async16(&s_w[buf][j * kWLd + ch * 8], w + static_cast<long long>(j) * C + c0 + ch * 8,
                    true);
       }
-    } else {  // B [C, r]: rows c, r contiguous
+    } else {  // B [C, rg]: rows c, rg contiguous, placed in columns g rg .. of the R-wide tile
+      const int jg = row_group(groups, c0) * rg;
       for (int i = tid; i < kBC * (R / 8); i += kThreadsSk) {
         const int c = i / (R / 8), ch = i % (R / 8);
-        cp_async16(&s_w[buf][c * kWLd + ch * 8], w + static_cast<long long>(c0 + c) * R + ch * 8,
-                   true);
+        const int j = ch * 8 - jg;
+        const bool ok = j >= 0 && j < rg;  // other adapters' columns: zero-filled
+        cp_async16(&s_w[buf][c * kWLd + ch * 8],
+                   w + static_cast<long long>(c0 + c) * rg + (ok ? j : 0), ok);
       }
     }
   };
@@ -190,6 +197,9 @@ __global__ void __launch_bounds__(kThreadsSk) lora_down_kernel(
     cp_async_wait_n(S - 2);
     __syncthreads();
     const int buf = i % S;
+    // n8 column tiles this step feeds: all of them, or (B of one adapter) that adapter's.
+    const int t_lo = kWrc ? 0 : row_group(groups, (sb + i) * kBC) * (rg / 8);
+    const int t_hi = kWrc ? NT : t_lo + rg / 8;
 #pragma unroll
     for (int kk = 0; kk < kBC / 16; ++kk) {
       uint32_t a[4];
@@ -197,7 +207,8 @@ __global__ void __launch_bounds__(kThreadsSk) lora_down_kernel(
       uint32_t b[NT][2];
       load_b_frags<NT, !kWrc>(b, s_w[buf], kWLd, kk * 16, lane);
 #pragma unroll
-      for (int t = 0; t < NT; ++t) mma16816(acc[t], a, b[t][0], b[t][1]);
+      for (int t = 0; t < NT; ++t)
+        if (t >= t_lo && t < t_hi) mma16816(acc[t], a, b[t][0], b[t][1]);
     }
     // Refill the slot consumed one iteration ago (every warp has passed this iteration's
     // barrier, so none still reads it).
@@ -272,7 +283,8 @@ __global__ void lora_down_finalize(const float* __restrict__ partial, int split,
 template <int NT>
 __global__ void __launch_bounds__(kThreadsSk) lora_grad_kernel(
     const __nv_bfloat16* __restrict__ big, int M, int C, const __nv_bfloat16* __restrict__ small,
-    float scale, float* __restrict__ out, int out_cr, float* __restrict__ partial, int split) {
+    const RowGroups groups, float scale, float* __restrict__ out, int out_cr,
+    float* __restrict__ partial, int split) {
   constexpr int R = NT * 8;
   constexpr int S = stages_for(R);
   constexpr int kBigLd = kGC + kPad;
@@ -284,6 +296,9 @@ __global__ void __launch_bounds__(kThreadsSk) lora_grad_kernel(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c0 = blockIdx.x * kGC;
+  // small is [M, n R]; the tile's columns of `big` belong to one adapter, whose R columns it reads.
+  const int ld_small = groups.n * R;
+  const int j0 = row_group(groups, c0) * R;
   const int steps = (M + kGM - 1) / kGM;
   const int sb = static_cast<int>((static_cast<long long>(steps) * blockIdx.y) / split);
   const int se = static_cast<int>((static_cast<long long>(steps) * (blockIdx.y + 1)) / split);
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(kThreadsSk) lora_grad_kernel(
       const int m = mb + row;
       const bool ok = m < M;
       cp_async16(&s_sm[buf][row * kSmLd + ch * 8],
-                 small + static_cast<long long>(ok ? m : 0) * R + ch * 8, ok);
+                 small + static_cast<long long>(ok ? m : 0) * ld_small + j0 + ch * 8, ok);
     }
   };
 
@@ -468,20 +483,20 @@ GradPlan lora_grad_plan(int M, int C, int r) {
     if (w_is_rc) {                                                                          \
       e = launch_dyn(lora_down_kernel<NTV, true>, grid, smem, stream);                      \
       if (e != cudaSuccess) return e;                                                       \
-      lora_down_kernel<NTV, true><<<grid, kThreadsSk, smem, stream>>>(in, M, C, w, scale, saved,   \
-                                                               scaled, partial, plan.split); \
+      lora_down_kernel<NTV, true><<<grid, kThreadsSk, smem, stream>>>(                     \
+          in, M, C, w, r, groups, scale, saved, scaled, partial, plan.split);               \
     } else {                                                                                \
       e = launch_dyn(lora_down_kernel<NTV, false>, grid, smem, stream);                     \
       if (e != cudaSuccess) return e;                                                       \
-      lora_down_kernel<NTV, false><<<grid, kThreadsSk, smem, stream>>>(in, M, C, w, scale, saved,  \
-                                                                scaled, partial, plan.split); \
+      lora_down_kernel<NTV, false><<<grid, kThreadsSk, smem, stream>>>(                    \
+          in, M, C, w, r / groups.n, groups, scale, saved, scaled, partial, plan.split);    \
     }                                                                                       \
     break;
 
 cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_bfloat16* w,
-                             bool w_is_rc, int r, float scale, __nv_bfloat16* saved,
-                             __nv_bfloat16* scaled, float* partial, const DownPlan& plan,
-                             cudaStream_t stream) {
+                             bool w_is_rc, int r, const RowGroups& groups, float scale,
+                             __nv_bfloat16* saved, __nv_bfloat16* scaled, float* partial,
+                             const DownPlan& plan, cudaStream_t stream) {
   dim3 grid((M + kBM - 1) / kBM, plan.split);
   const size_t smem = down_smem(r, w_is_rc);
   cudaError_t e = cudaSuccess;
@@ -518,13 +533,13 @@ cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_b
   case NTV:                                                                                \
     e = launch_dyn(lora_grad_kernel<NTV>, grid, smem, stream);                             \
     if (e != cudaSuccess) return e;                                                        \
-    lora_grad_kernel<NTV><<<grid, kThreadsSk, smem, stream>>>(big, M, C, small, scale, out,       \
-                                                       out_cr ? 1 : 0, partial, plan.split); \
+    lora_grad_kernel<NTV><<<grid, kThreadsSk, smem, stream>>>(                            \
+        big, M, C, small, groups, scale, out, out_cr ? 1 : 0, partial, plan.split);        \
     break;
 
 cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_bfloat16* small,
-                             int r, float scale, float* out, bool out_cr, float* partial,
-                             const GradPlan& plan, cudaStream_t stream) {
+                             int r, const RowGroups& groups, float scale, float* out, bool out_cr,
+                             float* partial, const GradPlan& plan, cudaStream_t stream) {
   dim3 grid((C + kGC - 1) / kGC, plan.split);
   const size_t smem = grad_smem(r);
   cudaError_t e = cudaSuccess;

@@ -282,13 +282,13 @@ __global__ void __launch_bounds__(kGvThreads, 2)
 }
 
 // h[tok, row] = bf16( sum of the row tile's partial slots, in CTA order
-//                    + sum_j ext_act[tok, j] * ext_w[row, j] )
+//                    + sum_j ext_act[tok, g, j] * ext_w[row, j] ),  g = the row tile's adapter
 // Grid (row tiles, tokens), one row per thread.  Thread 0 finds the CTAs whose ranges cover
 // the row tile (one 64-bit division each) and shares them through shared memory.
 __global__ void __launch_bounds__(kGvRows) nf4_gemv_finalize(
     const float* __restrict__ partial, int M, int N, int K, long long U, int G, int max_seg,
     int Mp, const __nv_bfloat16* __restrict__ ext_act, const __nv_bfloat16* __restrict__ ext_w,
-    int r, __nv_bfloat16* __restrict__ out) {
+    int r, const RowGroups groups, __nv_bfloat16* __restrict__ out) {
   __shared__ int s_first, s_last, s_seg0;
   const int KB = K / 64;
   const int rt = blockIdx.x, tok = blockIdx.y;
@@ -321,7 +321,8 @@ __global__ void __launch_bounds__(kGvRows) nf4_gemv_finalize(
       if (b + i <= b_last) v += p[i];
   }
   float e = 0.f;
-  const __nv_bfloat16* ea = ext_act + static_cast<long long>(tok) * r;
+  const __nv_bfloat16* ea = ext_act + static_cast<long long>(tok) * groups.n * r +
+                            row_group(groups, rt * kGvRows) * r;
   const __nv_bfloat16* ew = ext_w + static_cast<long long>(row) * r;
   for (int j = 0; j < r; j += 8) {
     const uint4 a4 = *reinterpret_cast<const uint4*>(ea + j);
@@ -362,9 +363,9 @@ GemvPlan gemv_plan(int M, int N, int K, int sm_count) {
 cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const float* absmax,
                                 const uint8_t* absmax_q8, const float* absmax_scale, int dq, int M,
                                 int N, int K, const __nv_bfloat16* ext_act,
-                                const __nv_bfloat16* ext_w, int r, __nv_bfloat16* out,
-                                float* partial, size_t partial_floats, const Codebook& cb,
-                                cudaStream_t stream) {
+                                const __nv_bfloat16* ext_w, int r, const RowGroups& groups,
+                                __nv_bfloat16* out, float* partial, size_t partial_floats,
+                                const Codebook& cb, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -401,8 +402,8 @@ cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const 
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  nf4_gemv_finalize<<<dim3((N + kGvRows - 1) / kGvRows, M), kGvRows, 0, stream>>>(partial, M, N, K, p.units, p.grid, p.max_seg,
-                                               8 * p.tt, ext_act, ext_w, r, out);
+  nf4_gemv_finalize<<<dim3((N + kGvRows - 1) / kGvRows, M), kGvRows, 0, stream>>>(
+      partial, M, N, K, p.units, p.grid, p.max_seg, 8 * p.tt, ext_act, ext_w, r, groups, out);
   return cudaGetLastError();
 }
 

@@ -131,6 +131,23 @@ qlora_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* 
   return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// 3-D row-major bf16 tensor [d2, d1, d0] (d0 contiguous), pitches p1 = d0 * 2 and p2 = d1 * p1
+// bytes, box {b0, 1, b2}, 128-byte swizzle.
+qlora_status encode_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                            uint64_t d2, uint32_t b0, uint32_t b2) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn;
+  qlora_status st = encoder(&fn);
+  if (st != QLORA_OK) return st;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, 1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 qlora_status check_weight(const qlora_nf4_weight* W) {
@@ -149,6 +166,23 @@ qlora_status check_weight(const qlora_nf4_weight* W) {
 }
 
 bool rank_ok(int r) { return r >= 8 && r <= 128 && (r % 8) == 0; }
+
+// Adapters packed along W0's rows: n in [1, kMaxGroups], n r a valid rank, every adapter's row
+// count a positive multiple of 128 (any multiple of 64 for n = 1), summing to N.
+qlora_status make_groups(const int* rows, int n, int N, int r, RowGroups* g) {
+  if (!rows) return QLORA_ERR_NULL;
+  if (n < 1 || n > kMaxGroups || !rank_ok(r) || !rank_ok(n * r)) return QLORA_ERR_SHAPE;
+  *g = RowGroups{};
+  g->n = n;
+  long long end = 0;
+  for (int i = 0; i < n; ++i) {
+    if (rows[i] < 64 || rows[i] % (n == 1 ? 64 : 128)) return QLORA_ERR_SHAPE;
+    end += rows[i];
+    if (end > N) return QLORA_ERR_SHAPE;
+    g->end[i] = static_cast<int>(end);
+  }
+  return end == N ? QLORA_OK : QLORA_ERR_SHAPE;
+}
 
 int ext_steps(int r) { return ((r + 15) / 16 * 16 + 63) / 64; }
 
@@ -189,7 +223,8 @@ WsLayout ws_layout(int M, int N, int K, int r) {
   return L;
 }
 
-GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, bool trans, void* out, int* err) {
+GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& groups, bool trans,
+                   void* out, int* err) {
   GemmArgs a;
   a.M = M;
   a.rows_w = trans ? W->K : W->N;
@@ -209,13 +244,16 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, bool trans, void* ou
   a.err = err;
   a.partial = nullptr;
   a.streamk = 0;
+  a.groups = groups;
   a.cb = codebook();
   return a;
 }
 
-// Maps for the dequant GEMM.  act: [M, red] bf16; ext_act: [M, r] bf16 (scaled rank-r term).
+// Maps for the dequant GEMM.  act: [M, red] bf16; ext_act: [M, n, r] bf16 (scaled rank-r
+// term of n adapters; n = 1 for dX, whose extension runs over all n r columns at once).
 qlora_status gemm_maps(GemmMaps* m, const qlora_nf4_weight* W, bool trans, const void* act,
-                       const void* ext_w, const void* ext_act, int M, int r, int bt) {
+                       const void* ext_w, const void* ext_act, int M, int r, int n_groups,
+                       int bt) {
   const uint64_t red = trans ? W->N : W->K;
   qlora_status st;
   st = encode_2d(&m->act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, red, M, red * 2, 64, bt,
@@ -235,8 +273,7 @@ qlora_status gemm_maps(GemmMaps* m, const qlora_nf4_weight* W, bool trans, const
     st = encode_2d(&m->ext_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ext_w, W->K, r, W->K * 2, 64, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != QLORA_OK) return st;
-  return encode_2d(&m->ext_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ext_act, r, M, r * 2, 64, bt,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode_3d_bf16(&m->ext_act, ext_act, r, trans ? 1 : n_groups, M, 64, bt);
 }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
@@ -247,12 +284,13 @@ void count(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_o
 // ---------------------------------------------------------------------------------------------
 // Stage bodies (validated by their callers).
 // ---------------------------------------------------------------------------------------------
+// groups: the adapters packed along the rows of B (w_rc = false); r is then n r_g.
 qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc, int r,
-                          float scale, void* saved, void* scaled, float* partial,
-                          cudaStream_t s) {
+                          const RowGroups& groups, float scale, void* saved, void* scaled,
+                          float* partial, cudaStream_t s) {
   const DownPlan dp = lora_down_plan(M, C, r);
   cudaError_t e = launch_lora_down(static_cast<const __nv_bfloat16*>(in), M, C,
-                                   static_cast<const __nv_bfloat16*>(w), w_rc, r, scale,
+                                   static_cast<const __nv_bfloat16*>(w), w_rc, r, groups, scale,
                                    static_cast<__nv_bfloat16*>(saved),
                                    static_cast<__nv_bfloat16*>(scaled), partial, dp, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
@@ -261,15 +299,16 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
 }
 
 // `partial` / `partial_bytes`: scratch for the stream-K partial sums (whole tiles if too small).
+// groups (forward only): adapters packed along W0's rows, each with r columns of ext_act.
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
-                     const void* ext_act, int M, int r, void* out, int* err, void* partial,
-                     size_t partial_bytes, cudaStream_t s) {
+                     const void* ext_act, int M, int r, const RowGroups& groups, void* out,
+                     int* err, void* partial, size_t partial_bytes, cudaStream_t s) {
   if (!trans && M <= kGemvMaxTokens && partial) {
     // Few tokens: the register-direct kernel streams the weight without the tcgen05 rings.
     const cudaError_t e = launch_nf4_gemv_fwd(
         static_cast<const __nv_bfloat16*>(act), W->q, W->absmax, W->absmax_q8, W->absmax_scale,
         W->double_quant ? 1 : 0, M, W->N, W->K, static_cast<const __nv_bfloat16*>(ext_act),
-        static_cast<const __nv_bfloat16*>(ext_w), r, static_cast<__nv_bfloat16*>(out),
+        static_cast<const __nv_bfloat16*>(ext_w), r, groups, static_cast<__nv_bfloat16*>(out),
         static_cast<float*>(partial), partial_bytes / 4, codebook(), s);
     if (e == cudaSuccess) {
       count(2);
@@ -278,10 +317,10 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
     if (e != cudaErrorInvalidValue) return QLORA_ERR_CUDA;
     (void)cudaGetLastError();  // scratch too small for its partials: use the tcgen05 kernel
   }
-  GemmArgs a = gemm_args(W, M, r, trans, out, err);
+  GemmArgs a = gemm_args(W, M, r, groups, trans, out, err);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;
-  qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, a.bt);
+  qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, groups.n, a.bt);
   if (st != QLORA_OK) return st;
   int launched = 0;
   const cudaError_t e = launch_qlora_gemm(trans, maps, a, partial ? partial_bytes / 4 : 0, s,
@@ -290,11 +329,13 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int r, float scale,
-                          float* out, bool out_cr, float* partial, cudaStream_t s) {
+// groups: the adapters packed along the columns of `big`; small is then [M, n r].
+qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int r,
+                          const RowGroups& groups, float scale, float* out, bool out_cr,
+                          float* partial, cudaStream_t s) {
   const GradPlan gp = lora_grad_plan(M, C, r);
   cudaError_t e = launch_lora_grad(static_cast<const __nv_bfloat16*>(big), M, C,
-                                   static_cast<const __nv_bfloat16*>(small), r, scale, out,
+                                   static_cast<const __nv_bfloat16*>(small), r, groups, scale, out,
                                    out_cr, partial, gp, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   count(gp.split > 1 ? 2 : 1);
@@ -303,6 +344,78 @@ qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int 
 
 size_t down_ws_bytes(int M, int C, int r) { return 4 * lora_down_plan(M, C, r).partial_floats; }
 size_t grad_ws_bytes(int M, int C, int r) { return 4 * lora_grad_plan(M, C, r).partial_floats; }
+
+// ---------------------------------------------------------------------------------------------
+// The layer over n adapters packed along W0's rows (n = 1: a single adapter).  W is
+// [N = sum N_g, K]; A [n r, K] stacks A_g; B [N, r] stacks B_g; XA_saved, dA and the packed
+// rank-r operands are [M, n r] / [n r, K]; dB is [N, r]; s = alpha / r for every adapter.
+// The caller has checked W and built `g`.
+// ---------------------------------------------------------------------------------------------
+qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A, const void* B,
+                        const RowGroups& g, int M, int r, float alpha, void* H, void* XA_saved,
+                        void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (!X || !A || !B || !H || !XA_saved) return QLORA_ERR_NULL;
+  const int R = g.n * r;
+  if (M < 1 || !rank_ok(r) || !rank_ok(R)) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
+    return QLORA_ERR_ALIGN;
+  const WsLayout L = ws_layout(M, W->N, W->K, R);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
+  const float scale = alpha / static_cast<float>(r);
+
+  // XA = X A^T [M, n r] (saved, bf16) and s * XA: every adapter's down-projection in one pass
+  // over X.
+  st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa,
+                    reinterpret_cast<float*>(w8 + L.scratch), s);
+  if (st != QLORA_OK) return st;
+  // h = X deq(W0)^T + (s XA_g) B_g^T for the rows of each adapter g, in one launch.
+  return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s);
+}
+
+qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W, const void* A,
+                        const void* B, const void* XA_saved, const RowGroups& g, int M, int r,
+                        float alpha, void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                        cudaStream_t s) {
+  if (!dY || !X || !A || !B || !XA_saved || !dA || !dB) return QLORA_ERR_NULL;
+  const int R = g.n * r;
+  if (M < 1 || !rank_ok(r) || !rank_ok(R)) return QLORA_ERR_SHAPE;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) ||
+      !aligned16(XA_saved) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)))
+    return QLORA_ERR_ALIGN;
+  const WsLayout L = ws_layout(M, W->N, W->K, R);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  auto* dyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
+  auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
+  float* scratch = reinterpret_cast<float*>(w8 + L.scratch);
+  const float scale = alpha / static_cast<float>(r);
+
+  // dYB = dY B_bd [M, n r] (bf16, for dA) and s * dYB, B_bd the block-diagonal of the B_g.
+  st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, scratch, s);
+  if (st != QLORA_OK) return st;
+  // dX = dY deq(W0) + (s dYB) A: one extension over all n r columns sums the adapters' terms.
+  if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
+                          L.scratch_bytes, s)) != QLORA_OK)
+    return st;
+  // dB_g = s dY_g^T XA_g  [N, r];  dA = s dYB^T X  [n r, K].
+  st = do_lora_grad(dY, M, W->N, XA_saved, r, g, scale, dB, true, scratch, s);
+  if (st != QLORA_OK) return st;
+  return do_lora_grad(X, M, W->K, dyb, R, single_group(W->K), scale, dA, false, scratch, s);
+}
 
 }  // namespace
 }  // namespace qlora
@@ -401,75 +514,65 @@ size_t qlora_workspace_bytes(int M, int N, int K, int r) {
 qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
                               const void* B, int M, int r, float alpha, void* H, void* XA_saved,
                               void* ws, size_t ws_bytes, qlora_stream_t stream) {
-  if (!X || !A || !B || !H || !XA_saved) return QLORA_ERR_NULL;
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
-    return QLORA_ERR_ALIGN;
-  const WsLayout L = ws_layout(M, W->N, W->K, r);
-  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
-  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
-  int dev;
-  if ((st = current_device(&dev)) != QLORA_OK) return st;
-  int* err;
-  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
-  const float scale = alpha / static_cast<float>(r);
-
-  // XA = X A^T (saved, bf16) and s * XA (the scaled operand of the fused up-projection).
-  st = do_lora_down(X, M, W->K, A, true, r, scale, XA_saved, sxa,
-                    reinterpret_cast<float*>(w8 + L.scratch), s);
-  if (st != QLORA_OK) return st;
-  // h = X deq(W0)^T + (s XA) B^T.
-  return do_gemm(X, W, false, B, sxa, M, r, H, err, w8 + L.scratch, L.scratch_bytes, s);
+  return linear_fwd(X, W, A, B, single_group(W->N), M, r, alpha, H, XA_saved, ws, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
                               const void* A, const void* B, const void* XA_saved, int M, int r,
                               float alpha, void* dX, float* dA, float* dB, void* ws,
                               size_t ws_bytes, qlora_stream_t stream) {
-  if (!dY || !X || !A || !B || !XA_saved || !dA || !dB) return QLORA_ERR_NULL;
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
-  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) ||
-      !aligned16(XA_saved) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)))
-    return QLORA_ERR_ALIGN;
-  const WsLayout L = ws_layout(M, W->N, W->K, r);
-  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
-  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
-  int dev;
-  if ((st = current_device(&dev)) != QLORA_OK) return st;
-  int* err;
-  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  auto* dyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
-  auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
-  float* scratch = reinterpret_cast<float*>(w8 + L.scratch);
-  const float scale = alpha / static_cast<float>(r);
+  return linear_bwd(dY, X, W, A, B, XA_saved, single_group(W->N), M, r, alpha, dX, dA, dB, ws,
+                    ws_bytes, static_cast<cudaStream_t>(stream));
+}
 
-  // dYB = dY B (bf16, for dA) and s * dYB (operand of the fused dX up-projection).
-  st = do_lora_down(dY, M, W->N, B, false, r, scale, dyb, sdyb, scratch, s);
+size_t qlora_grouped_workspace_bytes(int M, int N, int K, int r, int n_groups) {
+  if (M < 1 || N < 64 || K < 64 || n_groups < 1 || n_groups > kMaxGroups || !rank_ok(r) ||
+      !rank_ok(n_groups * r))
+    return 0;
+  return ws_layout(M, N, K, n_groups * r).total;
+}
+
+qlora_status qlora_grouped_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
+                               const void* B, const int* group_rows, int n_groups, int M, int r,
+                               float alpha, void* H, void* XA_saved, void* ws, size_t ws_bytes,
+                               qlora_stream_t stream) {
+  qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  // dX = dY deq(W0) + (s dYB) A.
-  if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, r, dX, err, scratch, L.scratch_bytes, s)) !=
-                QLORA_OK)
-    return st;
-  // dB = s dY^T XA  [N, r];  dA = s dYB^T X  [r, K].
-  st = do_lora_grad(dY, M, W->N, XA_saved, r, scale, dB, true, scratch, s);
+  RowGroups g;
+  if ((st = make_groups(group_rows, n_groups, W->N, r, &g)) != QLORA_OK) return st;
+  return linear_fwd(X, W, A, B, g, M, r, alpha, H, XA_saved, ws, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_grouped_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
+                               const void* A, const void* B, const void* XA_saved,
+                               const int* group_rows, int n_groups, int M, int r, float alpha,
+                               void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                               qlora_stream_t stream) {
+  qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  return do_lora_grad(X, M, W->K, dyb, r, scale, dA, false, scratch, s);
+  RowGroups g;
+  if ((st = make_groups(group_rows, n_groups, W->N, r, &g)) != QLORA_OK) return st;
+  return linear_bwd(dY, X, W, A, B, XA_saved, g, M, r, alpha, dX, dA, dB, ws, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_is_r_by_c, int r,
-                             float scale, void* saved, void* scaled, void* ws, size_t ws_bytes,
-                             qlora_stream_t stream) {
+                             const int* group_rows, int n_groups, float scale, void* saved,
+                             void* scaled, void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (!in || !w || !scaled) return QLORA_ERR_NULL;
   if (M < 1 || C < 64 || (C % 64) || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  RowGroups g = single_group(C);
+  if (group_rows) {  // B of n adapters [C, r / n], block-diagonal over the output columns
+    if (w_is_r_by_c || n_groups < 1 || r % n_groups) return QLORA_ERR_SHAPE;
+    const qlora_status gs = make_groups(group_rows, n_groups, C, r / n_groups, &g);
+    if (gs != QLORA_OK) return gs;
+  }
   if (!aligned16(in) || !aligned16(w) || !aligned16(scaled) || (saved && !aligned16(saved)))
     return QLORA_ERR_ALIGN;
   const size_t need = down_ws_bytes(M, C, r);
@@ -478,35 +581,46 @@ qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_
   int dev;
   qlora_status st = current_device(&dev);
   if (st != QLORA_OK) return st;
-  return do_lora_down(in, M, C, w, w_is_r_by_c != 0, r, scale, saved, scaled,
+  return do_lora_down(in, M, C, w, w_is_r_by_c != 0, r, g, scale, saved, scaled,
                       static_cast<float*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
-                            const void* ext_w, const void* ext_act, int M, int r, void* out,
-                            void* ws, size_t ws_bytes, qlora_stream_t stream) {
+                            const void* ext_w, const void* ext_act, int M, int r,
+                            const int* group_rows, int n_groups, void* out, void* ws,
+                            size_t ws_bytes, qlora_stream_t stream) {
   if (!act || !ext_w || !ext_act || !out) return QLORA_ERR_NULL;
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
   if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  RowGroups g = single_group(transpose_w ? W->K : W->N);
+  if (group_rows) {  // forward only: adapters along W0's rows, ext_act [M, n, r]
+    if (transpose_w) return QLORA_ERR_SHAPE;
+    if ((st = make_groups(group_rows, n_groups, W->N, r, &g)) != QLORA_OK) return st;
+  }
   if (!aligned16(act) || !aligned16(ext_w) || !aligned16(ext_act) || !aligned16(out))
     return QLORA_ERR_ALIGN;
-  const size_t need = gemm_ws_bytes(M, W->N, W->K, r, transpose_w != 0);
+  const size_t need = gemm_ws_bytes(M, W->N, W->K, g.n * r, transpose_w != 0);
   if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
   int dev;
   if ((st = current_device(&dev)) != QLORA_OK) return st;
   int* err;
   if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
-  return do_gemm(act, W, transpose_w != 0, ext_w, ext_act, M, r, out, err, ws, ws_bytes,
+  return do_gemm(act, W, transpose_w != 0, ext_w, ext_act, M, r, g, out, err, ws, ws_bytes,
                  static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, int r,
-                             float scale, float* out, int out_r_by_c, void* ws, size_t ws_bytes,
-                             qlora_stream_t stream) {
+                             const int* group_rows, int n_groups, float scale, float* out,
+                             int out_r_by_c, void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (!big || !small || !out) return QLORA_ERR_NULL;
   if (M < 1 || C < 64 || (C % 64) || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  RowGroups g = single_group(C);
+  if (group_rows) {  // adapters along big's columns, small [M, n r]
+    const qlora_status gs = make_groups(group_rows, n_groups, C, r, &g);
+    if (gs != QLORA_OK) return gs;
+  }
   if (!aligned16(big) || !aligned16(small) || !aligned16(out)) return QLORA_ERR_ALIGN;
   const size_t need = grad_ws_bytes(M, C, r);
   if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
@@ -514,8 +628,8 @@ qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, i
   int dev;
   qlora_status st = current_device(&dev);
   if (st != QLORA_OK) return st;
-  return do_lora_grad(big, M, C, small, r, scale, out, out_r_by_c == 0, static_cast<float*>(ws),
-                      static_cast<cudaStream_t>(stream));
+  return do_lora_grad(big, M, C, small, r, g, scale, out, out_r_by_c == 0,
+                      static_cast<float*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 uint64_t qlora_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
@@ -580,10 +694,10 @@ qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, 
   auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8);
   const float scale = alpha / static_cast<float>(r);
   // Both scratch regions are written in full before they are read: nothing needs clearing.
-  st = do_lora_down(X, M, W->K, A, true, r, scale, XA_saved, sxa,
+  st = do_lora_down(X, M, W->K, A, true, r, single_group(W->K), scale, XA_saved, sxa,
                     reinterpret_cast<float*>(w8 + sxa_bytes), s);
   if (st != QLORA_OK) return st;
-  return do_gemm(X, W, false, B, sxa, M, r, H, err, w8 + sxa_bytes,
+  return do_gemm(X, W, false, B, sxa, M, r, single_group(W->N), H, err, w8 + sxa_bytes,
                  kNoAllocScratchBytes - sxa_bytes, s);
 }
 

@@ -8,7 +8,11 @@
 //   dX       dX[M, K] = dY[M, N] . deq(W0)  + (s dYB)[M, r] . A
 // A tile is computed transposed, out^T[128 weight rows, nh x bt tokens]: the weight is the MMA's
 // A operand (M = 128 rows of W0 for the forward, 128 input features for dX) and the tokens are
-// the MMA's N (bt = 16..256), so small token counts still fill a full 128-row MMA.  With more
+// the MMA's N (bt = 16..256), so small token counts still fill a full 128-row MMA.  With
+// several adapters packed along W0's rows (q/k/v sharing X), a forward row tile takes the
+// extension operand's columns of its own adapter, (s XA)[M, g, 0..r), so one launch computes
+// every adapter's output ("Speed Up Fine-Tuning 2x with Unsloth", "How it works internally",
+// item 3: several LoRA adapters packed into one tensor).  With more
 // than 256 tokens a tile holds two 256-token halves (nh = 2) that share every dequantised
 // weight tile: one dequantised element then feeds 1024 flops.
 //
@@ -271,7 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; ok && it < n_steps;) {
         int t, k0, len;
         segment(it, t, k0, len);
-        const int tok0 = (t / row_tiles) * tile_tokens;
+        const int tq = t / row_tiles;
+        const int tok0 = tq * tile_tokens;
+        // Forward: the tile's adapter picks its r columns of the packed [M, n, r] operand.
+        const int eg = kTransW ? 0 : row_group(args.groups, (t - tq * row_tiles) * kRowsW);
         for (int k = k0; k < k0 + len; ++k, ++it) {
           // Step it reuses the X slots of step it - DX: wait until that step's MMAs are done.
           if (it >= DX &&
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k < kt)
               tma_load_2d(dst, &tm_act, xfull + xs, k * 64, tok0 + h * bt);
             else
-              tma_load_2d(dst, &tm_ext_act, xfull + xs, (k - kt) * 64, tok0 + h * bt);
+              tma_load_3d(dst, &tm_ext_act, xfull + xs, (k - kt) * 64, eg, tok0 + h * bt);
           }
           issued = it + 1;
         }

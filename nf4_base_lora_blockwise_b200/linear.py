@@ -118,6 +118,60 @@ def backward(dY, X, w: NF4Weight, A, B, XA, alpha, need_dx=True, dX=None, dA=Non
     return (dX if need_dx else None), dA, dB
 
 
+def grouped_workspace_bytes(M, N, K, r, n_groups):
+    return abi.qlora_grouped_workspace_bytes(M, N, K, r, n_groups)
+
+
+def alloc_grouped_workspace(M, N, K, r, n_groups, device):
+    n = grouped_workspace_bytes(M, N, K, r, n_groups)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def grouped_forward(X, w: NF4Weight, A, B, group_rows, alpha, H=None, XA=None, ws=None):
+    """Adapters packed along W0's rows (qlora_grouped_fwd).  w: NF4 [sum N_g, K]; A [n r, K];
+    B [sum N_g, r].  Returns (H [M, sum N_g], XA_saved [M, n r])."""
+    M = X.shape[0]
+    n = len(group_rows)
+    r = A.shape[0] // n
+    _need(X, torch.bfloat16, (M, w.K), "X")
+    _need(A, torch.bfloat16, (n * r, w.K), "A")
+    _need(B, torch.bfloat16, (w.N, r), "B")
+    if H is None:
+        H = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    if XA is None:
+        XA = torch.empty((M, n * r), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = alloc_grouped_workspace(M, w.N, w.K, r, n, X.device)
+    abi.qlora_grouped_fwd(X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(), group_rows, M,
+                          r, alpha, H.data_ptr(), XA.data_ptr(), ws.data_ptr(), ws.numel(),
+                          _stream())
+    return H, XA
+
+
+def grouped_backward(dY, X, w: NF4Weight, A, B, XA, group_rows, alpha, need_dx=True, dX=None,
+                     dA=None, dB=None, ws=None):
+    """Backward of grouped_forward.  Returns (dX or None, dA fp32 [n r, K], dB fp32 [N, r])."""
+    M = X.shape[0]
+    n = len(group_rows)
+    r = A.shape[0] // n
+    _need(dY, torch.bfloat16, (M, w.N), "dY")
+    _need(X, torch.bfloat16, (M, w.K), "X")
+    _need(XA, torch.bfloat16, (M, n * r), "XA")
+    dev = X.device
+    if need_dx and dX is None:
+        dX = torch.empty((M, w.K), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((n * r, w.K), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((w.N, r), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_grouped_workspace(M, w.N, w.K, r, n, dev)
+    abi.qlora_grouped_bwd(dY.data_ptr(), X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(),
+                          XA.data_ptr(), group_rows, M, r, alpha, _ptr(dX) if need_dx else None,
+                          dA.data_ptr(), dB.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
+    return (dX if need_dx else None), dA, dB
+
+
 def swiglu_forward(g, u, a=None):
     if a is None:
         a = torch.empty_like(g)

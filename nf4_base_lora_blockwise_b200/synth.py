@@ -6,8 +6,9 @@ oracle take their inputs from here.
 
 Recipe: one ``torch.Generator`` (CPU) seeded with ``seed`` draws, in this order: for a single
 linear (or independent projections, one after the other) X, W0, A, B, dY; for the MLP
-workload X, then W0, A, B of gate, up and down, then dY.  Values are drawn in fp32 and cast to bf16 (round to nearest
-even).  "N(0, s)" means standard deviation s.  The LoRA down-projection A is either uniform
+workload X, then W0, A, B of gate, up and down, then dY; for a packed-adapter workload (q/k/v
+sharing X) X, then W0, A, B of each adapter, then dY over all adapters' outputs.  Values are
+drawn in fp32 and cast to bf16 (round to nearest even).  "N(0, s)" means standard deviation s.  The LoRA down-projection A is either uniform
 on (-a, a) with a = 1/sqrt(in) ("Kaiming-uniform" with torch's nn.Linear default slope
 sqrt(5)), or the explicit bound of the tiny workload.  B is N(0, 0.01) -- non-zero, so the
 LoRA path contributes to h and to dX.
@@ -43,6 +44,7 @@ class Workload:
     b_std: float = 0.01
     mlp: bool = False             # gate/up -> SwiGLU -> down
     notes: str = ""
+    grouped: bool = False         # the linears share X and run as one packed-adapter layer
 
 
 def _lin(name, K, N, r, alpha, w_std=0.02, dq=False):
@@ -66,6 +68,13 @@ WORKLOADS = {
                              _lin("down_proj", 28672, 8192, 64, 16.0, 0.015, True))),
 }
 
+# Llama-3-8B attention projections q 4096 -> 4096, k and v 4096 -> 1024 (grouped-query), each
+# with its own r 16, alpha 32 adapter, sharing the 4096-token input: one packed-adapter layer.
+WORKLOADS["qkv_8b"] = Workload("qkv_8b", 4096, (_lin("q_proj", 4096, 4096, 16, 32.0),
+                                                _lin("k_proj", 4096, 1024, 16, 32.0),
+                                                _lin("v_proj", 4096, 1024, 16, 32.0)),
+                               grouped=True)
+
 # Token-count sweep on 4096 -> 14336, r 16, alpha 32.
 SWEEP_M = (1, 16, 128, 1024, 16384)
 for _m in SWEEP_M:
@@ -78,7 +87,7 @@ def workload(name, M=None):
     w = WORKLOADS[name]
     if M is not None and M != w.M:
         w = Workload(w.name, M, w.linears, w.x_std, w.dy_std, w.a_bound, w.b_std, w.mlp,
-                     w.notes)
+                     w.notes, w.grouped)
     return w
 
 
@@ -95,7 +104,8 @@ def make_inputs(w, seed=0):
     """Draw the inputs of workload ``w`` on the CPU as bf16 tensors.
 
     MLP workload: X [M, K_gate], then W0, A, B of gate, up and down, then dY [M, N_down] (the
-    gradient at the down output).  Other workloads: for each linear, X [M, K], W0, A, B, then
+    gradient at the down output).  Packed-adapter workload: X [M, K], then W0, A, B of each
+    adapter, then dY [M, sum N] (adapter g's gradient in its own column range).  Other workloads: for each linear, X [M, K], W0, A, B, then
     dY [M, N] -- independent projections, each with its own activations.
 
     Returns ``{"X", "dY", "linears": [{"W0", "A", "B", "X", "dY"}]}``; the top-level X and dY
@@ -112,6 +122,12 @@ def make_inputs(w, seed=0):
         return {"W0": W0, "A": A, "B": B}
 
     lins = []
+    if w.grouped:
+        X = _normal(gen, (w.M, w.linears[0].K), w.x_std)
+        for L in w.linears:
+            lins.append(draw_weights(L))
+        dY = _normal(gen, (w.M, sum(L.N for L in w.linears)), w.dy_std)
+        return {"X": X, "linears": lins, "dY": dY}
     if w.mlp:
         X = _normal(gen, (w.M, w.linears[0].K), w.x_std)
         for L in w.linears:
@@ -132,6 +148,16 @@ def make_linear(M, K, N, r, alpha=None, seed=0, x_std=1.0, w_std=0.02, a_bound=0
     """Inputs of one ad-hoc linear (used by parity tests on ragged / edge shapes)."""
     w = Workload("adhoc", M, (_lin("linear", K, N, r, alpha if alpha else 2.0 * r, w_std),),
                  x_std=x_std, dy_std=dy_std, a_bound=a_bound, b_std=b_std)
+    return make_inputs(w, seed)
+
+
+def make_grouped(M, K, Ns, r, alpha=None, seed=0, x_std=1.0, w_std=0.02, a_bound=0.0,
+                 b_std=0.01, dy_std=1e-2):
+    """Inputs of an ad-hoc packed-adapter layer: adapters with out-features Ns share X [M, K]."""
+    lins = tuple(_lin(f"adapter{i}", K, N, r, alpha if alpha else 2.0 * r, w_std)
+                 for i, N in enumerate(Ns))
+    w = Workload("adhoc_grouped", M, lins, x_std=x_std, dy_std=dy_std, a_bound=a_bound,
+                 b_std=b_std, grouped=True)
     return make_inputs(w, seed)
 
 

@@ -89,6 +89,58 @@ def backward_dx_rows(dY, Wdeq, A, B, alpha, rows):
 
 
 # --------------------------------------------------------------------------------------
+# Several adapters packed into one layer ("Speed Up Fine-Tuning 2x with Unsloth on Llama and
+# Mistral", "How it works internally", item 3: several LoRA adapters packed into one tensor;
+# "Unsloth vs QLoRA vs Liger-Kernel", section 5, step 2: adapters on q/k/v and gate/up, which
+# read the same input).  The pages give no formula beyond the single layer, so the packed
+# layer is read as exactly that: n independent layers (W0_g, A_g, B_g) on one X, each with
+# s = alpha / r, whose outputs sit side by side in columns and whose input gradients add.
+# The lists below hold the adapters in order; packed tensors stack them (H, dY, XA_saved by
+# columns; A, dA, B, dB by rows).
+# --------------------------------------------------------------------------------------
+def split_cols(T, widths):
+    """Column blocks of T of the given widths, in order."""
+    T = _f64(T)
+    edges = np.cumsum([0] + list(widths))
+    assert edges[-1] == T.shape[1]
+    return [T[:, edges[i]:edges[i + 1]] for i in range(len(widths))]
+
+
+def grouped_forward(X, Wdeqs, As, Bs, alpha):
+    """Return (H, XA_saved): each adapter's forward, outputs placed side by side."""
+    outs = [forward(X, Wd, A, B, alpha) for Wd, A, B in zip(Wdeqs, As, Bs)]
+    return (np.concatenate([h for h, _ in outs], axis=1),
+            np.concatenate([xa for _, xa in outs], axis=1))
+
+
+def grouped_forward_rows(X, Wdeqs, As, Bs, alpha, rows):
+    return grouped_forward(_f64(X)[np.asarray(rows)], Wdeqs, As, Bs, alpha)[0]
+
+
+def grouped_backward_weights(dY, X, As, Bs, alpha):
+    """dA (adapters' dA_g stacked by rows) and dB (dB_g stacked by rows); adapter g takes its
+    own column block of dY."""
+    dYs = split_cols(dY, [B.shape[0] for B in Bs])
+    parts = [backward_weights(dYg, X, A, B, alpha) for dYg, A, B in zip(dYs, As, Bs)]
+    return {"dA": np.concatenate([p["dA"] for p in parts], axis=0),
+            "dB": np.concatenate([p["dB"] for p in parts], axis=0)}
+
+
+def grouped_backward_dx_rows(dY, Wdeqs, As, Bs, alpha, rows):
+    """dX on the given rows: the sum over adapters of each one's input gradient."""
+    dYs = split_cols(dY, [B.shape[0] for B in Bs])
+    return sum(backward_dx_rows(dYg, Wd, A, B, alpha, rows)
+               for dYg, Wd, A, B in zip(dYs, Wdeqs, As, Bs))
+
+
+def grouped_backward(dY, X, Wdeqs, As, Bs, alpha):
+    """All gradients of the packed layer over every row: dict(dX, dA, dB)."""
+    out = grouped_backward_weights(dY, X, As, Bs, alpha)
+    out["dX"] = grouped_backward_dx_rows(dY, Wdeqs, As, Bs, alpha, np.arange(_f64(X).shape[0]))
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # SwiGLU glue between gate/up and down in the MLP workload ("Unsloth vs QLoRA vs
 # Liger-Kernel", section 2 names the MLP SwiGLU among the hand-differentiated ops; the pages
 # print no formula).  a = silu(g) * u with silu(g) = g * sigmoid(g).

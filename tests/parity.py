@@ -139,3 +139,65 @@ def make(M, K, N, r, alpha=None, seed=0, **kw):
     inp = synth.make_linear(M, K, N, r, alpha=alpha, seed=seed, **kw)
     L = synth.LinearShape("linear", K, N, r, alpha if alpha else 2.0 * r)
     return inp, L
+
+
+# ------------------------------------------------------------------------------------------
+# Packed adapters (one stacked NF4 weight, adapters along its rows, sharing X)
+# ------------------------------------------------------------------------------------------
+def stacked(inp):
+    """W0, A, B of every adapter stacked by rows (CPU bf16)."""
+    lins = inp["linears"]
+    return (torch.cat([l["W0"] for l in lins]), torch.cat([l["A"] for l in lins]),
+            torch.cat([l["B"] for l in lins]))
+
+
+def run_grouped(inp, Ns, alpha, dq=False, need_dx=True):
+    """GPU pack of the stacked weight + grouped forward + backward; CPU tensors out."""
+    W0, A, B = stacked(inp)
+    X, dY = inp["X"].cuda(), inp["dY"].cuda()
+    A, B = A.cuda(), B.cuda()
+    w = linear.nf4_pack(W0.cuda(), double_quant=dq)
+    H, XA = linear.grouped_forward(X, w, A, B, list(Ns), alpha)
+    dX, dA, dB = linear.grouped_backward(dY, X, w, A, B, XA, list(Ns), alpha, need_dx=need_dx)
+    torch.cuda.synchronize()
+    code = linear.device_error()
+    assert code == 0, f"device error word set: {code}"
+    return {"w": w, "H": H, "XA": XA, "dX": dX, "dA": dA, "dB": dB}
+
+
+def check_grouped(inp, Ns, alpha, got, rows=None, dq=False):
+    """The packed layer against the oracle: the stacked weight is quantised as one tensor and
+    its dequantised rows split by adapter.  Returns the error dict."""
+    W0, _, _ = stacked(inp)
+    ref, Wd = oracle_deq(W0, dq)
+    edges = np.cumsum([0] + list(Ns))
+    Wds = [Wd[edges[i]:edges[i + 1]] for i in range(len(Ns))]
+    As = [f32(l["A"]) for l in inp["linears"]]
+    Bs = [f32(l["B"]) for l in inp["linears"]]
+    X, dY = f32(inp["X"]), f32(inp["dY"])
+    M = X.shape[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    errs = {}
+    errs["h"] = qlora.rel_err(f32(got["H"])[rows],
+                              qlora.grouped_forward_rows(X, Wds, As, Bs, alpha, rows))
+    errs["XA"] = qlora.rel_err(f32(got["XA"]), np.concatenate([qlora.lora_down(X, A) for A in As],
+                                                              axis=1))
+    wts = qlora.grouped_backward_weights(dY, X, As, Bs, alpha)
+    errs["dA"] = qlora.rel_err(f32(got["dA"]), wts["dA"])
+    errs["dB"] = qlora.rel_err(f32(got["dB"]), wts["dB"])
+    # Per adapter too: a small adapter's error must not hide under a large one's scale.
+    r = As[0].shape[0]
+    for i in range(len(Ns)):
+        errs[f"dA{i}"] = qlora.rel_err(f32(got["dA"])[i * r:(i + 1) * r],
+                                       wts["dA"][i * r:(i + 1) * r])
+        errs[f"dB{i}"] = qlora.rel_err(f32(got["dB"])[edges[i]:edges[i + 1]],
+                                       wts["dB"][edges[i]:edges[i + 1]])
+        errs[f"h{i}"] = qlora.rel_err(
+            f32(got["H"])[rows][:, edges[i]:edges[i + 1]],
+            qlora.forward_rows(X, Wds[i], As[i], Bs[i], alpha, rows))
+    if got["dX"] is not None:
+        errs["dX"] = qlora.rel_err(f32(got["dX"])[rows],
+                                   qlora.grouped_backward_dx_rows(dY, Wds, As, Bs, alpha, rows))
+    for k, v in errs.items():
+        assert v <= TOL, f"{k}: max|err|/max|ref| = {v:.3e} > {TOL}"
+    return errs

@@ -88,3 +88,35 @@ def test_workspace_bytes(lib):
     big = lib.qlora_workspace_bytes(4096, 4096, 4096, 16)
     assert 0 < small < big
     assert big >= 2 * 4096 * 16 * 2                    # the two bf16 rank-r activations
+
+
+def _gfwd(lib, rows, N=None, r=16, ws_bytes=1 << 30):
+    N = sum(rows) if N is None else N
+    W = _w(N=N)
+    arr = (ctypes.c_int * max(len(rows), 1))(*rows)
+    return lib.qlora_grouped_fwd(FAKE, ctypes.byref(W), FAKE, FAKE, arr if rows else None,
+                                 len(rows), 64, r, 32.0, FAKE, FAKE, FAKE, ws_bytes, None)
+
+
+def test_grouped_validation_codes(lib):
+    """Packed adapters: 1..8 adapters, each a multiple of 128 rows (of 64 for one adapter),
+    summing to W's rows, with n r a valid rank."""
+    assert _gfwd(lib, [], N=256) == 1                   # no group array
+    assert _gfwd(lib, [128] * 9) == 2                   # more than 8 adapters
+    assert _gfwd(lib, [256, 192]) == 2                  # 192 rows: not a multiple of 128
+    assert _gfwd(lib, [256, 128], N=512) == 2           # rows do not sum to N
+    assert _gfwd(lib, [128, 128], r=72) == 2            # n r = 144 > 128
+    assert _gfwd(lib, [128, 128], r=12) == 2
+    assert _gfwd(lib, [256, 128], ws_bytes=16) == 5     # valid groups, workspace too small
+    assert _gfwd(lib, [192], ws_bytes=16) == 5          # one adapter: multiples of 64 suffice
+    W = _w(N=384)
+    arr = (ctypes.c_int * 2)(256, 128)
+    assert lib.qlora_grouped_bwd(FAKE, FAKE, ctypes.byref(W), FAKE, FAKE, FAKE, arr, 2, 64, 16,
+                                 32.0, FAKE, FAKE, None, FAKE, 1 << 30, None) == 1  # dB NULL
+    assert lib.qlora_grouped_workspace_bytes(64, 384, 256, 16, 9) == 0
+    assert lib.qlora_grouped_workspace_bytes(64, 384, 256, 72, 2) == 0
+    # The packed rank sizes the workspace: n adapters of rank r need what rank n r needs.
+    assert (lib.qlora_grouped_workspace_bytes(4096, 6144, 4096, 16, 3)
+            == lib.qlora_workspace_bytes(4096, 6144, 4096, 48))
+    assert (lib.qlora_grouped_workspace_bytes(64, 512, 256, 16, 1)
+            == lib.qlora_workspace_bytes(64, 512, 256, 16))

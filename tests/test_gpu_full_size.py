@@ -125,6 +125,53 @@ def test_full_size_mlp():
     check_one_linear(a.cpu(), inp["dY"], ld, down, "mlp/down")
 
 
+def test_full_size_packed_qkv():
+    """The packed-adapter workload: q 4096->4096, k and v 4096->1024 on one stacked NF4 weight
+    with their own r 16 adapters, sharing 4096 tokens, in the grouped launch sequence.  Codes
+    and absmax of the stacked weight bit-exact on sampled rows; h and dX on the sampled token
+    rows, per adapter; XA, dA and dB in full, per adapter."""
+    w = synth.workload("qkv_8b")
+    inp = synth.make_inputs(w, seed=0)
+    Ns = [L.N for L in w.linears]
+    L0 = w.linears[0]
+    W0 = torch.cat([d["W0"] for d in inp["linears"]])
+    A = torch.cat([d["A"] for d in inp["linears"]])
+    B = torch.cat([d["B"] for d in inp["linears"]])
+    X, dY = inp["X"].cuda(), inp["dY"].cuda()
+    wg = linear.nf4_pack(W0.cuda())
+    H, XA = linear.grouped_forward(X, wg, A.cuda(), B.cuda(), Ns, L0.alpha)
+    dX, dA, dB = linear.grouped_backward(dY, X, wg, A.cuda(), B.cuda(), XA, Ns, L0.alpha)
+    torch.cuda.synchronize()
+    assert linear.device_error() == 0
+    full = parity.oracle_pack(W0, False)
+    parity.check_pack(wg, parity.subset(full, _weight_rows(sum(Ns))), False)
+    del wg
+    Wd = parity.oracle_dequant(full)
+    del full
+    rows = synth.sample_rows(w.M).numpy()
+    Xf, dYf = parity.f32(inp["X"]), parity.f32(inp["dY"])
+    Xr, dYr = Xf[rows].astype(np.float64), dYf[rows].astype(np.float64)
+    s = L0.alpha / L0.r
+    edges = np.cumsum([0] + Ns)
+    r = L0.r
+    dx_ref = np.zeros((len(rows), L0.K))
+    errs = {}
+    for g, d in enumerate(inp["linears"]):
+        a, b = edges[g], edges[g + 1]
+        Ag = parity.f32(d["A"]).astype(np.float64)
+        Bg = parity.f32(d["B"]).astype(np.float64)
+        h_ref = _rows_matmul(Xr, Wd[a:b]) + s * ((Xr @ Ag.T) @ Bg.T)
+        errs[f"h{g}"] = qlora.rel_err(parity.f32(H)[rows][:, a:b], h_ref)
+        dx_ref += _rows_matmul_t(dYr[:, a:b], Wd[a:b]) + s * ((dYr[:, a:b] @ Bg) @ Ag)
+        wts = qlora.backward_weights(dYf[:, a:b], Xf, Ag, Bg, L0.alpha)
+        errs[f"XA{g}"] = qlora.rel_err(parity.f32(XA)[:, g * r:(g + 1) * r], wts["XA"])
+        errs[f"dA{g}"] = qlora.rel_err(parity.f32(dA)[g * r:(g + 1) * r], wts["dA"])
+        errs[f"dB{g}"] = qlora.rel_err(parity.f32(dB)[a:b], wts["dB"])
+    errs["dX"] = qlora.rel_err(parity.f32(dX)[rows], dx_ref)
+    for k, v in errs.items():
+        assert v <= parity.TOL, f"qkv_8b {k}: {v:.3e}"
+
+
 def _grad_like(M, N, seed):
     g = torch.Generator().manual_seed(1000 + seed)
     return (torch.randn((M, N), generator=g) * 1e-2).to(torch.bfloat16)
@@ -169,7 +216,7 @@ def test_one_hot_products_reproduce_the_weight(K, N, M):
     zero = torch.zeros((Md, r), dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
         dX = torch.full((Md, K), float("nan"), dtype=torch.bfloat16, device="cuda")
-        abi.qlora_nf4_gemm(dY.data_ptr(), cw, 1, A.data_ptr(), zero.data_ptr(), Md, r,
+        abi.qlora_nf4_gemm(dY.data_ptr(), cw, 1, A.data_ptr(), zero.data_ptr(), Md, r, None,
                            dX.data_ptr(), ws.data_ptr(), ws.numel(), stream)
         torch.cuda.synchronize()
         assert linear.device_error() == 0
@@ -180,7 +227,7 @@ def test_one_hot_products_reproduce_the_weight(K, N, M):
     zero = torch.zeros((Mf, r), dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
         H = torch.full((Mf, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-        abi.qlora_nf4_gemm(X.data_ptr(), cw, 0, B.data_ptr(), zero.data_ptr(), Mf, r,
+        abi.qlora_nf4_gemm(X.data_ptr(), cw, 0, B.data_ptr(), zero.data_ptr(), Mf, r, None,
                            H.data_ptr(), ws.data_ptr(), ws.numel(), stream)
         torch.cuda.synchronize()
         assert linear.device_error() == 0
