@@ -55,7 +55,6 @@ struct GemmArgs {
   int r_pad16;     // r rounded up to a multiple of 16
   int bt;          // tokens per half tile = MMA N
   int nh;          // token halves per tile (1 or 2)
-  int stages;
   int kblocks;     // K / 64 = absmax blocks per row of W0
   int N;           // rows of W0
   int dq;
@@ -91,9 +90,15 @@ GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count);
 // Partial-sum bytes any device (at most kGemmMaxCtas SMs) may need for this shape.
 size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile);
 
-int gemm_pick_bt(int M);
-int gemm_pick_halves(int M);
-int gemm_pick_stages(int bt);
+// Token tile: bt tokens per MMA (N) and nh halves per tile.  Up to 256 tokens: one half of
+// M rounded up to 16.  More: two halves of 256, or, when whole tiles fill the GPU, the
+// narrower bt (multiple of 16, >= 128) that a cost model of the busiest CTA favours.
+struct GemmTile {
+  int bt;
+  int nh;
+};
+GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count);
+cudaError_t gemm_device_sms(int* sms);  // SMs of the current device (cached)
 size_t gemm_smem_bytes(int bt, int nh);
 // Falls back to whole tiles when stream-K is chosen but `partial` is null or smaller than the
 // schedule needs (partial_floats_avail).  *launched = kernels enqueued (1, or 2 with stream-K).

@@ -224,16 +224,16 @@ WsLayout ws_layout(int M, int N, int K, int r) {
 }
 
 GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& groups, bool trans,
-                   void* out, int* err) {
+                   void* out, int* err, int sms) {
   GemmArgs a;
   a.M = M;
   a.rows_w = trans ? W->K : W->N;
   a.kt = (trans ? W->N : W->K) / 64;
   a.r_pad16 = (r + 15) / 16 * 16;
   a.n_ext = (a.r_pad16 + 63) / 64;
-  a.bt = gemm_pick_bt(M);
-  a.nh = gemm_pick_halves(M);
-  a.stages = gemm_pick_stages(a.bt);
+  const GemmTile tl = gemm_pick_tile(M, a.rows_w, a.kt + a.n_ext, sms);
+  a.bt = tl.bt;
+  a.nh = tl.nh;
   a.kblocks = W->K / 64;
   a.N = W->N;
   a.dq = W->double_quant ? 1 : 0;
@@ -317,7 +317,9 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
     if (e != cudaErrorInvalidValue) return QLORA_ERR_CUDA;
     (void)cudaGetLastError();  // scratch too small for its partials: use the tcgen05 kernel
   }
-  GemmArgs a = gemm_args(W, M, r, groups, trans, out, err);
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;
   qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, groups.n, a.bt);

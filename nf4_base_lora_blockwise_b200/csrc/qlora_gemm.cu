@@ -681,22 +681,77 @@ int g_sm_count[64];
 
 }  // namespace
 
-int gemm_pick_bt(int M) {
-  if (M >= 256) return 256;
-  const int b = (M + 15) / 16 * 16;
-  return b < 16 ? 16 : b;
+namespace {
+
+// Relative duration (cycles of the busiest CTA) of a whole-tile schedule with token tiles of
+// nh x bt, from the kernel's per-step profile at 512-token tiles: besides ~2.12 tensor cycles
+// per token, the MMA thread spends ~745 cycles per 64-deep step on barriers, descriptors and
+// the commit; and when one accumulator fills TMEM (more than 256 token columns) the epilogue's
+// drain, ~37 cycles per token column, is exposed at every tile switch instead of overlapping
+// the next tile's mainloop.
+double whole_tile_cycles(int M, int rows_w, int steps, int G, int bt, int nh) {
+  const int tt = bt * nh;
+  const long long tiles =
+      static_cast<long long>((rows_w + kRowsW - 1) / kRowsW) * ((M + tt - 1) / tt);
+  const long long rounds = (tiles + G - 1) / G;
+  const double step = 745.0 + 2.12 * tt;
+  const double drain = 37.0 * tt;
+  const bool exposed = make_plan(bt, nh).nacc == 1;
+  return static_cast<double>(rounds) * (steps * step + (exposed ? drain : 0.0)) +
+         (exposed ? 0.0 : drain);
 }
 
-int gemm_pick_halves(int M) { return M > 256 ? 2 : 1; }
+}  // namespace
 
-int gemm_pick_stages(int bt) { return make_plan(bt, 1).sx; }
+GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count) {
+  GemmTile t;
+  if (M <= 256) {  // one half: as many tokens as there are, in steps of 16
+    t.bt = M < 16 ? 16 : (M + 15) / 16 * 16;
+    t.nh = 1;
+    return t;
+  }
+  t.bt = 256;
+  t.nh = 2;
+  const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
+  const long long tiles =
+      static_cast<long long>((rows_w + kRowsW - 1) / kRowsW) * ((M + 511) / 512);
+  if (tiles < G) return t;  // stream-K over the widest tiles
+  // Whole tiles: the last round of tiles is usually part-full, so narrower token tiles can
+  // shorten the busiest CTA's work at the same number of rounds.  Keep 512 tokens unless the
+  // model gives at least 2 %.
+  const double wide = whole_tile_cycles(M, rows_w, steps_per_tile, G, 256, 2);
+  double best = wide;
+  int best_bt = 256;
+  for (int bt = 240; bt >= 128; bt -= 16) {
+    const double c = whole_tile_cycles(M, rows_w, steps_per_tile, G, bt, 2);
+    if (c < best) {
+      best = c;
+      best_bt = bt;
+    }
+  }
+  if (best <= 0.98 * wide) t.bt = best_bt;
+  return t;
+}
+
+cudaError_t gemm_device_sms(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (g_sm_count[dev] == 0) {
+    e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  *sms = g_sm_count[dev];
+  return cudaSuccess;
+}
 
 size_t gemm_smem_bytes(int bt, int nh) { return make_plan(bt, nh).smem; }
 
 GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count) {
   GemmSchedule sc;
-  const int bt = gemm_pick_bt(M), nh = gemm_pick_halves(M);
-  const int tile_tokens = bt * nh;
+  const GemmTile tl = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count);
+  const int tile_tokens = tl.bt * tl.nh;
   sc.n_tiles = ((rows_w + kRowsW - 1) / kRowsW) * ((M + tile_tokens - 1) / tile_tokens);
   const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
   if (sc.n_tiles >= G) {
@@ -720,15 +775,13 @@ size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile) {
 cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
                               size_t partial_floats_avail, cudaStream_t stream, int* launched) {
   *launched = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  int sms = 0;
+  cudaError_t e = gemm_device_sms(&sms);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (g_sm_count[dev] == 0) {
-    e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-  }
-  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, g_sm_count[dev]);
+  // The caller's tile (TMA boxes, smem plan) must be the one the schedule assumes.
+  const GemmTile tl = gemm_pick_tile(args.M, args.rows_w, args.kt + args.n_ext, sms);
+  if (tl.bt != args.bt || tl.nh != args.nh) return cudaErrorInvalidValue;
+  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, sms);
   if (sc.streamk && (!args.partial || sc.partial_floats > partial_floats_avail)) {
     // No room for the partial sums: whole tiles, one CTA per tile.
     sc.streamk = 0;
