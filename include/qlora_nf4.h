@@ -110,7 +110,10 @@ QLORA_API qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, ql
 QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
 
 /* Forward.  X [M, K], A [r, K], B [N, r] bf16 device (read); H [M, N] bf16 device (written);
- * XA_saved [M, r] bf16 device (written: X A^T rounded to bf16, kept for the backward).
+ * XA_saved [M, r] bf16 device (written: X A^T rounded to bf16, kept for the backward), or
+ * NULL to keep nothing and let the backward recompute it ("What is Unsloth? Faster LLM
+ * Fine-Tuning Explained", "How does Unsloth make fine-tuning faster?": recompute instead of
+ * store).
  * ws: device scratch of at least qlora_workspace_bytes(M, N, K, r) bytes.
  * alpha: LoRA alpha; s = alpha / r.  r must be a multiple of 8 in [8, 128].
  * For M <= 32 the base product applies each block's absmax to the block's 64-deep partial sum
@@ -121,7 +124,9 @@ QLORA_API qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W
                               const void* B, int M, int r, float alpha, void* H, void* XA_saved,
                               void* ws, size_t ws_bytes, qlora_stream_t stream);
 
-/* Backward.  dY [M, N], X [M, K], A, B, XA_saved [M, r] bf16 device (read).
+/* Backward.  dY [M, N], X [M, K], A, B, XA_saved [M, r] bf16 device (read).  XA_saved may be
+ * NULL: X A^T is then recomputed from X (one more pass over X), bit-identical to the value the
+ * forward would have saved, so the results do not change.
  * dX [M, K] bf16 device (written; may be NULL to skip the dX GEMM).
  * dA [r, K] and dB [N, r] fp32 device (overwritten).  ws as for the forward. */
 QLORA_API qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
@@ -140,7 +145,7 @@ QLORA_API qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlo
  *            stacked bf16 weight with qlora_nf4_pack);
  *   A        [n r, K]: A_0, A_1, ... stacked by rows;      B  [N, r]: B_0, B_1, ... by rows;
  *   H, dY    [M, N]: adapter g's outputs in columns [sum_{i<g} N_i, sum_{i<=g} N_i);
- *   XA_saved [M, n r]: X A_g^T in columns [g r, (g + 1) r);
+ *   XA_saved [M, n r]: X A_g^T in columns [g r, (g + 1) r) (NULL: recomputed, as for one);
  *   dA       [n r, K] fp32 (rows of A_g at g r);          dB [N, r] fp32 (rows of B_g).
  * The results equal n separate qlora_linear_fwd / qlora_linear_bwd calls on the slices, with
  * dX their sum; X is read once for all adapters' down-projections, and each large product is

@@ -356,10 +356,11 @@ size_t grad_ws_bytes(int M, int C, int r) { return 4 * lora_grad_plan(M, C, r).p
 qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A, const void* B,
                         const RowGroups& g, int M, int r, float alpha, void* H, void* XA_saved,
                         void* ws, size_t ws_bytes, cudaStream_t s) {
-  if (!X || !A || !B || !H || !XA_saved) return QLORA_ERR_NULL;
+  if (!X || !A || !B || !H) return QLORA_ERR_NULL;
   const int R = g.n * r;
   if (M < 1 || !rank_ok(r) || !rank_ok(R)) return QLORA_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) ||
+      (XA_saved && !aligned16(XA_saved)))
     return QLORA_ERR_ALIGN;
   const WsLayout L = ws_layout(M, W->N, W->K, R);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
@@ -373,8 +374,8 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
   auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
   const float scale = alpha / static_cast<float>(r);
 
-  // XA = X A^T [M, n r] (saved, bf16) and s * XA: every adapter's down-projection in one pass
-  // over X.
+  // XA = X A^T [M, n r] (saved in bf16 unless XA_saved is NULL) and s * XA: every adapter's
+  // down-projection in one pass over X.
   st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa,
                     reinterpret_cast<float*>(w8 + L.scratch), s);
   if (st != QLORA_OK) return st;
@@ -386,11 +387,12 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
                         const void* B, const void* XA_saved, const RowGroups& g, int M, int r,
                         float alpha, void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
                         cudaStream_t s) {
-  if (!dY || !X || !A || !B || !XA_saved || !dA || !dB) return QLORA_ERR_NULL;
+  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_NULL;
   const int R = g.n * r;
   if (M < 1 || !rank_ok(r) || !rank_ok(R)) return QLORA_ERR_SHAPE;
   if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) ||
-      !aligned16(XA_saved) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)))
+      (XA_saved && !aligned16(XA_saved)) || !aligned16(dA) || !aligned16(dB) ||
+      (dX && !aligned16(dX)))
     return QLORA_ERR_ALIGN;
   const WsLayout L = ws_layout(M, W->N, W->K, R);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
@@ -406,6 +408,14 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
   float* scratch = reinterpret_cast<float*>(w8 + L.scratch);
   const float scale = alpha / static_cast<float>(r);
 
+  // Without a saved XA, recompute it from X (the forward's own kernel on the same inputs, so
+  // bit for bit the value it would have saved) and take dB first, while small0 holds it.
+  if (!XA_saved) {
+    st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, dyb, sdyb, scratch, s);
+    if (st != QLORA_OK) return st;
+    st = do_lora_grad(dY, M, W->N, dyb, r, g, scale, dB, true, scratch, s);
+    if (st != QLORA_OK) return st;
+  }
   // dYB = dY B_bd [M, n r] (bf16, for dA) and s * dYB, B_bd the block-diagonal of the B_g.
   st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, scratch, s);
   if (st != QLORA_OK) return st;
@@ -414,8 +424,10 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
                           L.scratch_bytes, s)) != QLORA_OK)
     return st;
   // dB_g = s dY_g^T XA_g  [N, r];  dA = s dYB^T X  [n r, K].
-  st = do_lora_grad(dY, M, W->N, XA_saved, r, g, scale, dB, true, scratch, s);
-  if (st != QLORA_OK) return st;
+  if (XA_saved) {
+    st = do_lora_grad(dY, M, W->N, XA_saved, r, g, scale, dB, true, scratch, s);
+    if (st != QLORA_OK) return st;
+  }
   return do_lora_grad(X, M, W->K, dyb, R, single_group(W->K), scale, dA, false, scratch, s);
 }
 
@@ -674,11 +686,12 @@ qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void* da, void
 qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, const void* A,
                                       const void* B, int M, int r, float alpha, void* H,
                                       void* XA_saved, qlora_stream_t stream) {
-  if (!X || !A || !B || !H || !XA_saved) return QLORA_ERR_NULL;
+  if (!X || !A || !B || !H) return QLORA_ERR_NULL;
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
   if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !aligned16(XA_saved))
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) ||
+      (XA_saved && !aligned16(XA_saved)))
     return QLORA_ERR_ALIGN;
   // The forward needs s*XA [M, r] bf16 plus the down-projection's split partials; the GEMM's
   // stream-K partials use what is left of the scratch (whole tiles if they do not fit).

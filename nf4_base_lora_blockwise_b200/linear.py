@@ -77,8 +77,9 @@ def alloc_workspace(M, N, K, r, device):
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
-def forward(X, w: NF4Weight, A, B, alpha, H=None, XA=None, ws=None):
-    """h = X deq(W0)^T + (alpha/r) (X A^T) B^T.  Returns (h, XA_saved)."""
+def forward(X, w: NF4Weight, A, B, alpha, H=None, XA=None, ws=None, save_xa=True):
+    """h = X deq(W0)^T + (alpha/r) (X A^T) B^T.  Returns (h, XA_saved), XA_saved None when
+    save_xa is False (the backward then recomputes it)."""
     M, K = X.shape
     r = A.shape[0]
     _need(X, torch.bfloat16, (M, w.K), "X")
@@ -86,23 +87,26 @@ def forward(X, w: NF4Weight, A, B, alpha, H=None, XA=None, ws=None):
     _need(B, torch.bfloat16, (w.N, r), "B")
     if H is None:
         H = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
-    if XA is None:
+    if XA is None and save_xa:
         XA = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
         ws = alloc_workspace(M, w.N, w.K, r, X.device)
     abi.qlora_linear_fwd(X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(), M, r, alpha,
-                         H.data_ptr(), XA.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
-    return H, XA
+                         H.data_ptr(), _ptr(XA) if save_xa else None, ws.data_ptr(), ws.numel(),
+                         _stream())
+    return H, (XA if save_xa else None)
 
 
 def backward(dY, X, w: NF4Weight, A, B, XA, alpha, need_dx=True, dX=None, dA=None, dB=None,
              ws=None):
-    """Hand-derived gradients.  Returns (dX or None, dA fp32 [r, K], dB fp32 [N, r])."""
+    """Hand-derived gradients.  Returns (dX or None, dA fp32 [r, K], dB fp32 [N, r]).  XA None:
+    recomputed from X."""
     M = X.shape[0]
     r = A.shape[0]
     _need(dY, torch.bfloat16, (M, w.N), "dY")
     _need(X, torch.bfloat16, (M, w.K), "X")
-    _need(XA, torch.bfloat16, (M, r), "XA")
+    if XA is not None:
+        _need(XA, torch.bfloat16, (M, r), "XA")
     dev = X.device
     if need_dx and dX is None:
         dX = torch.empty((M, w.K), dtype=torch.bfloat16, device=dev)
@@ -113,7 +117,7 @@ def backward(dY, X, w: NF4Weight, A, B, XA, alpha, need_dx=True, dX=None, dA=Non
     if ws is None:
         ws = alloc_workspace(M, w.N, w.K, r, dev)
     abi.qlora_linear_bwd(dY.data_ptr(), X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(),
-                         XA.data_ptr(), M, r, alpha, _ptr(dX) if need_dx else None,
+                         _ptr(XA), M, r, alpha, _ptr(dX) if need_dx else None,
                          dA.data_ptr(), dB.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
     return (dX if need_dx else None), dA, dB
 
@@ -127,9 +131,10 @@ def alloc_grouped_workspace(M, N, K, r, n_groups, device):
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
-def grouped_forward(X, w: NF4Weight, A, B, group_rows, alpha, H=None, XA=None, ws=None):
+def grouped_forward(X, w: NF4Weight, A, B, group_rows, alpha, H=None, XA=None, ws=None,
+                    save_xa=True):
     """Adapters packed along W0's rows (qlora_grouped_fwd).  w: NF4 [sum N_g, K]; A [n r, K];
-    B [sum N_g, r].  Returns (H [M, sum N_g], XA_saved [M, n r])."""
+    B [sum N_g, r].  Returns (H [M, sum N_g], XA_saved [M, n r] or None)."""
     M = X.shape[0]
     n = len(group_rows)
     r = A.shape[0] // n
@@ -138,14 +143,14 @@ def grouped_forward(X, w: NF4Weight, A, B, group_rows, alpha, H=None, XA=None, w
     _need(B, torch.bfloat16, (w.N, r), "B")
     if H is None:
         H = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
-    if XA is None:
+    if XA is None and save_xa:
         XA = torch.empty((M, n * r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
         ws = alloc_grouped_workspace(M, w.N, w.K, r, n, X.device)
     abi.qlora_grouped_fwd(X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(), group_rows, M,
-                          r, alpha, H.data_ptr(), XA.data_ptr(), ws.data_ptr(), ws.numel(),
-                          _stream())
-    return H, XA
+                          r, alpha, H.data_ptr(), _ptr(XA) if save_xa else None, ws.data_ptr(),
+                          ws.numel(), _stream())
+    return H, (XA if save_xa else None)
 
 
 def grouped_backward(dY, X, w: NF4Weight, A, B, XA, group_rows, alpha, need_dx=True, dX=None,
@@ -156,7 +161,8 @@ def grouped_backward(dY, X, w: NF4Weight, A, B, XA, group_rows, alpha, need_dx=T
     r = A.shape[0] // n
     _need(dY, torch.bfloat16, (M, w.N), "dY")
     _need(X, torch.bfloat16, (M, w.K), "X")
-    _need(XA, torch.bfloat16, (M, n * r), "XA")
+    if XA is not None:
+        _need(XA, torch.bfloat16, (M, n * r), "XA")
     dev = X.device
     if need_dx and dX is None:
         dX = torch.empty((M, w.K), dtype=torch.bfloat16, device=dev)
@@ -167,7 +173,7 @@ def grouped_backward(dY, X, w: NF4Weight, A, B, XA, group_rows, alpha, need_dx=T
     if ws is None:
         ws = alloc_grouped_workspace(M, w.N, w.K, r, n, dev)
     abi.qlora_grouped_bwd(dY.data_ptr(), X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(),
-                          XA.data_ptr(), group_rows, M, r, alpha, _ptr(dX) if need_dx else None,
+                          _ptr(XA), group_rows, M, r, alpha, _ptr(dX) if need_dx else None,
                           dA.data_ptr(), dB.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
     return (dX if need_dx else None), dA, dB
 

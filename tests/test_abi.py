@@ -120,3 +120,18 @@ def test_grouped_validation_codes(lib):
             == lib.qlora_workspace_bytes(4096, 6144, 4096, 48))
     assert (lib.qlora_grouped_workspace_bytes(64, 512, 256, 16, 1)
             == lib.qlora_workspace_bytes(64, 512, 256, 16))
+
+
+def test_xa_saved_may_be_null(lib):
+    """Recompute instead of store: a NULL XA_saved passes validation in the forward, the
+    backward and the packed entry points (the workspace check answers next)."""
+    W = _w()
+    assert lib.qlora_linear_fwd(FAKE, ctypes.byref(W), FAKE, FAKE, 64, 16, 32.0, FAKE, None,
+                                FAKE, 16, None) == 5
+    assert lib.qlora_linear_bwd(FAKE, FAKE, ctypes.byref(W), FAKE, FAKE, None, 64, 16, 32.0,
+                                FAKE, FAKE, FAKE, FAKE, 16, None) == 5
+    arr = (ctypes.c_int * 1)(128)
+    assert lib.qlora_grouped_bwd(FAKE, FAKE, ctypes.byref(W), FAKE, FAKE, None, arr, 1, 64, 16,
+                                 32.0, FAKE, FAKE, FAKE, FAKE, 16, None) == 5
+    assert lib.qlora_linear_fwd(FAKE, ctypes.byref(W), FAKE, FAKE, 64, 16, 32.0, FAKE, FAKE + 8,
+                                FAKE, 1 << 30, None) == 3

@@ -87,3 +87,21 @@ def test_grouped_no_dx_and_deterministic():
     assert c["dX"] is None
     for k in ("H", "XA", "dA", "dB"):
         assert torch.equal(a[k], c[k]), k
+
+
+def test_grouped_recompute_xa_is_bit_identical():
+    Ns = (256, 128, 128)
+    inp = synth.make_grouped(300, 512, Ns, 16, seed=14, dy_std=1.0)
+    W0, A, B = parity.stacked(inp)
+    X, dY, A, B = inp["X"].cuda(), inp["dY"].cuda(), A.cuda(), B.cuda()
+    w = linear.nf4_pack(W0.cuda())
+    H, XA = linear.grouped_forward(X, w, A, B, list(Ns), 32.0)
+    H2, none = linear.grouped_forward(X, w, A, B, list(Ns), 32.0, save_xa=False)
+    assert none is None
+    saved = linear.grouped_backward(dY, X, w, A, B, XA, list(Ns), 32.0)
+    recomputed = linear.grouped_backward(dY, X, w, A, B, None, list(Ns), 32.0)
+    torch.cuda.synchronize()
+    assert linear.device_error() == 0
+    assert torch.equal(H, H2)
+    for a, b, k in zip(saved, recomputed, ("dX", "dA", "dB")):
+        assert torch.equal(a, b), k

@@ -136,3 +136,23 @@ def test_swiglu_parity():
     rg, ru = qlora.swiglu_backward(fg, fu, fd)
     assert qlora.rel_err(parity.f32(dg), rg) <= 1e-2
     assert qlora.rel_err(parity.f32(du), ru) <= 1e-2
+
+
+@pytest.mark.parametrize("M,K,N,r", [(300, 512, 384, 16), (9, 256, 256, 16), (2048, 256, 2048, 16)])
+def test_recompute_xa_is_bit_identical(M, K, N, r):
+    """Recompute instead of store: with no saved XA the backward recomputes X A^T with the
+    forward's own kernel, so every gradient equals the saving path's bit for bit."""
+    inp, L = parity.make(M, K, N, r, seed=M + 5, dy_std=1.0)
+    lin = inp["linears"][0]
+    X, dY, A, B = (inp["X"].cuda(), inp["dY"].cuda(), lin["A"].cuda(), lin["B"].cuda())
+    w = linear.nf4_pack(lin["W0"].cuda())
+    H, XA = linear.forward(X, w, A, B, L.alpha)
+    H2, none = linear.forward(X, w, A, B, L.alpha, save_xa=False)
+    assert none is None
+    saved = linear.backward(dY, X, w, A, B, XA, L.alpha)
+    recomputed = linear.backward(dY, X, w, A, B, None, L.alpha)
+    torch.cuda.synchronize()
+    assert linear.device_error() == 0
+    assert torch.equal(H, H2)
+    for a, b, k in zip(saved, recomputed, ("dX", "dA", "dB")):
+        assert torch.equal(a, b), k
