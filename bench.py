@@ -234,6 +234,7 @@ class Step:
     def __init__(self, w, dev, seed, unpacked=False):
         self.w = w
         self.share_x = False
+        self.pglue = None
         inp = synth.make_inputs(w, seed=seed)
         bf = dict(dtype=torch.bfloat16, device=dev)
         if w.grouped:
@@ -267,12 +268,29 @@ class Step:
             self.inputs = [(st, "X") for st in self.states] + [(st, "dY") for st in self.states]
             self.glue = None
             return
-        # MLP block: gate/up on the shared input X, SwiGLU, down; the backward runs down, the
-        # SwiGLU backward, then up and gate on their output gradients dg, du.
         gate, up, down = w.linears
         lg, lu, ld = inp["linears"]
-        X = inp["X"].to(dev)
         I = gate.N
+        if not unpacked:
+            # MLP block with gate and up packed into one layer on the shared X: its output
+            # [M, 2I] feeds the packed SwiGLU, whose backward writes the layer's upstream
+            # gradient [M, 2I]; the layer's dX is then the block's input gradient (gate's and
+            # up's contributions summed by the one dX GEMM).
+            Lgu = synth.LinearShape("gate_proj+up_proj", gate.K, 2 * I, gate.r, gate.alpha,
+                                    gate.w_std, gate.double_quant)
+            self.a = torch.empty((w.M, I), **bf)
+            sgu = LinearState(Lgu, w.M, inp["X"], torch.empty((w.M, 2 * I), **bf),
+                              torch.cat([lg["W0"], lu["W0"]]), torch.cat([lg["A"], lu["A"]]),
+                              torch.cat([lg["B"], lu["B"]]), dev, groups=[I, I])
+            sd = LinearState(down, w.M, self.a, inp["dY"], ld["W0"], ld["A"], ld["B"], dev)
+            self.states = [sgu, sd]
+            self.pglue = (sgu, sd)
+            self.glue = None
+            self.inputs = [(sgu, "X"), (sd, "dY")]
+            return
+        # MLP block: gate/up on the shared input X, SwiGLU, down; the backward runs down, the
+        # SwiGLU backward, then up and gate on their output gradients dg, du.
+        X = inp["X"].to(dev)
         dg = torch.empty((w.M, I), **bf)
         du = torch.empty((w.M, I), **bf)
         self.a = torch.empty((w.M, I), **bf)
@@ -287,6 +305,14 @@ class Step:
     def twin(self):
         """A second set of step buffers over the same weights (see LinearState.twin)."""
         t = copy.copy(self)
+        if self.pglue is not None:
+            sgu, sd = (st.twin() for st in self.pglue)
+            t.a = torch.empty_like(self.a)
+            sd.X = t.a
+            t.states = [sgu, sd]
+            t.pglue = (sgu, sd)
+            t.inputs = [(sgu, "X"), (sd, "dY")]
+            return t
         if self.glue is None:
             t.states = [st.twin() for st in self.states]
             if self.share_x:
@@ -309,6 +335,17 @@ class Step:
         return [(st, "X") for st in xs] + [(st, "dY") for st in states]
 
     def stages(self, stream):
+        p = lambda t: t.data_ptr()
+        if self.pglue is not None:
+            sgu, sd = self.pglue
+            M, I = self.a.shape
+            return (sgu.fwd_stages(stream)
+                    + [("swiglu.fwd", lambda: abi.qlora_swiglu_packed_fwd(p(sgu.H), p(self.a), M,
+                                                                          I, stream))]
+                    + sd.fwd_stages(stream) + sd.bwd_stages(stream)
+                    + [("swiglu.bwd", lambda: abi.qlora_swiglu_packed_bwd(
+                        p(sgu.H), p(sd.dX), p(sgu.dY), M, I, stream))]
+                    + sgu.bwd_stages(stream))
         if self.glue is None:
             out = []
             for st in self.states:
@@ -316,7 +353,6 @@ class Step:
             return out
         sg, su, sd, dg, du = self.glue
         n = self.a.numel()
-        p = lambda t: t.data_ptr()
         return (sg.fwd_stages(stream) + su.fwd_stages(stream)
                 + [("swiglu.fwd", lambda: abi.qlora_swiglu_fwd(p(sg.H), p(su.H), p(self.a), n,
                                                                stream))]
@@ -328,6 +364,15 @@ class Step:
     def e2e(self):
         """One step through the public Python entry points (linear.forward / backward and the
         SwiGLU glue), on the device buffers already holding this step's inputs."""
+        if self.pglue is not None:
+            sgu, sd = self.pglue
+            sgu.forward()
+            linear.swiglu_packed_forward(sgu.H, a=self.a)
+            sd.forward()
+            sd.backward()
+            linear.swiglu_packed_backward(sgu.H, sd.dX, dgu=sgu.dY)
+            sgu.backward()
+            return
         if self.glue is None:
             for st in self.states:
                 st.forward()
@@ -347,6 +392,9 @@ class Step:
 
     def outputs(self):
         """Result tensors a user reads back after a step."""
+        if self.pglue is not None:
+            sgu, sd = self.pglue
+            return [sd.H, sgu.dX] + [t for st in self.states for t in (st.dA, st.dB)]
         if self.glue is None:
             return [t for st in self.states for t in (st.H, st.dX, st.dA, st.dB)]
         sg, su, sd, _, _ = self.glue
@@ -645,6 +693,9 @@ def workload_config(w, unpacked=False):
     if w.grouped:
         c["adapters"] = ("unpacked: one layer per adapter on the shared input" if unpacked else
                          "packed: one stacked NF4 weight, adapters along its rows, shared input")
+    if w.mlp:
+        c["adapters"] = ("unpacked: gate and up as separate layers" if unpacked else
+                         "gate and up packed into one layer on the shared input")
     return c
 
 
@@ -678,7 +729,8 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="launch every stage from Python instead of replaying a CUDA graph")
     ap.add_argument("--unpacked", action="store_true",
-                    help="adapters sharing an input (qkv_8b) run as separate layers")
+                    help="adapters sharing an input (qkv_8b, mlp_8b's gate/up) run as "
+                         "separate layers")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

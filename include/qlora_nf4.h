@@ -174,6 +174,16 @@ QLORA_API qlora_status qlora_swiglu_fwd(const void* g, const void* u, void* a, i
 QLORA_API qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void* da, void* dg, void* du,
                               int64_t n, qlora_stream_t stream);
 
+/* The same glue on the output of a packed gate/up layer (gate and up adapters sharing X, see
+ * qlora_grouped_fwd with group_rows {I, I}): gu [M, 2I] bf16 holds g in columns [0, I) and u
+ * in [I, 2I) of each row; a and da are [M, I]; dgu [M, 2I] receives dg and du in the same
+ * places, i.e. the upstream gradient of the packed layer.  I must be a multiple of 8.  M = 0
+ * does nothing. */
+QLORA_API qlora_status qlora_swiglu_packed_fwd(const void* gu, void* a, int64_t M, int I,
+                                               qlora_stream_t stream);
+QLORA_API qlora_status qlora_swiglu_packed_bwd(const void* gu, const void* da, void* dgu,
+                                               int64_t M, int I, qlora_stream_t stream);
+
 /* ---- The stages the two linear entry points are composed of (same validation rules). ---- */
 
 /* The stage calls take an optional adapter split, `group_rows` (host array of n_groups row

@@ -32,6 +32,8 @@ EXPORTS = (
     "qlora_grouped_workspace_bytes",
     "qlora_grouped_fwd",
     "qlora_grouped_bwd",
+    "qlora_swiglu_packed_fwd",
+    "qlora_swiglu_packed_bwd",
 )
 
 STATUS = {
@@ -98,6 +100,8 @@ def _lib():
             "qlora_noalloc_scratch_bytes": (_SZ, []),
             "qlora_device_error": (_I, [ctypes.POINTER(ctypes.c_int)]),
             "qlora_grouped_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+            "qlora_swiglu_packed_fwd": (_I, [_VP, _VP, _I64, _I, _VP]),
+            "qlora_swiglu_packed_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _VP]),
             "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
                                        _VP]),
@@ -179,6 +183,14 @@ def qlora_grouped_bwd(dY, X, weight, A, B, XA_saved, group_rows, M, r, alpha, dX
     _check("qlora_grouped_bwd", _lib().qlora_grouped_bwd(dY, X, ctypes.byref(weight), A, B,
                                                          XA_saved, rows, n, M, r, float(alpha),
                                                          dX, dA, dB, ws, ws_bytes, stream))
+
+
+def qlora_swiglu_packed_fwd(gu, a, M, I, stream):
+    _check("qlora_swiglu_packed_fwd", _lib().qlora_swiglu_packed_fwd(gu, a, M, I, stream))
+
+
+def qlora_swiglu_packed_bwd(gu, da, dgu, M, I, stream):
+    _check("qlora_swiglu_packed_bwd", _lib().qlora_swiglu_packed_bwd(gu, da, dgu, M, I, stream))
 
 
 def qlora_swiglu_fwd(g, u, a, n, stream):

@@ -161,5 +161,10 @@ cudaError_t launch_swiglu_fwd(const __nv_bfloat16* g, const __nv_bfloat16* u, __
 cudaError_t launch_swiglu_bwd(const __nv_bfloat16* g, const __nv_bfloat16* u,
                               const __nv_bfloat16* da, __nv_bfloat16* dg, __nv_bfloat16* du,
                               int64_t n, cudaStream_t stream);
+// Packed gate/up [M, 2I] (g in columns [0, I), u in [I, 2I)); a, da [M, I]; dgu [M, 2I].
+cudaError_t launch_swiglu_packed_fwd(const __nv_bfloat16* gu, __nv_bfloat16* a, int64_t M, int I,
+                                     cudaStream_t stream);
+cudaError_t launch_swiglu_packed_bwd(const __nv_bfloat16* gu, const __nv_bfloat16* da,
+                                     __nv_bfloat16* dgu, int64_t M, int I, cudaStream_t stream);
 
 }  // namespace qlora

@@ -683,6 +683,38 @@ qlora_status qlora_swiglu_bwd(const void* g, const void* u, const void* da, void
   return st;
 }
 
+qlora_status qlora_swiglu_packed_fwd(const void* gu, void* a, int64_t M, int I,
+                                     qlora_stream_t stream) {
+  if (!gu || !a) return QLORA_ERR_NULL;
+  if (M < 0 || I < 8 || I % 8) return QLORA_ERR_SHAPE;
+  if (!aligned16(gu) || !aligned16(a)) return QLORA_ERR_ALIGN;
+  if (M == 0) return QLORA_OK;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_swiglu_packed_fwd(static_cast<const __nv_bfloat16*>(gu),
+                                            static_cast<__nv_bfloat16*>(a), M, I,
+                                            static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+qlora_status qlora_swiglu_packed_bwd(const void* gu, const void* da, void* dgu, int64_t M, int I,
+                                     qlora_stream_t stream) {
+  if (!gu || !da || !dgu) return QLORA_ERR_NULL;
+  if (M < 0 || I < 8 || I % 8) return QLORA_ERR_SHAPE;
+  if (!aligned16(gu) || !aligned16(da) || !aligned16(dgu)) return QLORA_ERR_ALIGN;
+  if (M == 0) return QLORA_OK;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_swiglu_packed_bwd(
+      static_cast<const __nv_bfloat16*>(gu), static_cast<const __nv_bfloat16*>(da),
+      static_cast<__nv_bfloat16*>(dgu), M, I, static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
 qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, const void* A,
                                       const void* B, int M, int r, float alpha, void* H,
                                       void* XA_saved, qlora_stream_t stream) {

@@ -35,6 +35,24 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return v;
 }
 
+// a = silu(g) * u and its gradients, 8 elements at a time.
+__device__ __forceinline__ void swiglu8(const float (&fg)[8], const float (&fu)[8],
+                                        float (&fa)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) fa[k] = fg[k] * sigmoid_f(fg[k]) * fu[k];
+}
+
+__device__ __forceinline__ void swiglu_grad8(const float (&fg)[8], const float (&fu)[8],
+                                             const float (&fd)[8], float (&og)[8],
+                                             float (&ou)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float sg = sigmoid_f(fg[k]);
+    og[k] = fd[k] * fu[k] * sg * (1.f + fg[k] * (1.f - sg));
+    ou[k] = fd[k] * fg[k] * sg;
+  }
+}
+
 __global__ void swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ g,
                                   const __nv_bfloat16* __restrict__ u,
                                   __nv_bfloat16* __restrict__ a, int64_t n) {
@@ -45,8 +63,7 @@ __global__ void swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ g,
     float fg[8], fu[8], fa[8];
     unpack8(__ldg(reinterpret_cast<const uint4*>(g) + i), fg);
     unpack8(__ldg(reinterpret_cast<const uint4*>(u) + i), fu);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) fa[k] = fg[k] * sigmoid_f(fg[k]) * fu[k];
+    swiglu8(fg, fu, fa);
     reinterpret_cast<uint4*>(a)[i] = pack8(fa);
   }
   for (int64_t i = nv * 8 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -69,12 +86,7 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ g,
     unpack8(__ldg(reinterpret_cast<const uint4*>(g) + i), fg);
     unpack8(__ldg(reinterpret_cast<const uint4*>(u) + i), fu);
     unpack8(__ldg(reinterpret_cast<const uint4*>(da) + i), fd);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float sg = sigmoid_f(fg[k]);
-      og[k] = fd[k] * fu[k] * sg * (1.f + fg[k] * (1.f - sg));
-      ou[k] = fd[k] * fg[k] * sg;
-    }
+    swiglu_grad8(fg, fu, fd, og, ou);
     reinterpret_cast<uint4*>(dg)[i] = pack8(og);
     reinterpret_cast<uint4*>(du)[i] = pack8(ou);
   }
@@ -85,6 +97,47 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ g,
     const float sg = sigmoid_f(x);
     dg[i] = __float2bfloat16_rn(d * y * sg * (1.f + x * (1.f - sg)));
     du[i] = __float2bfloat16_rn(d * x * sg);
+  }
+}
+
+// Packed gate/up: gu [M, 2I] holds g in columns [0, I) and u in [I, 2I) of every row (the
+// output of a packed gate/up layer); a and da are [M, I]; dgu [M, 2I] takes dg and du in the
+// same places (the upstream gradient of that layer).  I % 8 == 0.
+__global__ void swiglu_packed_fwd_kernel(const __nv_bfloat16* __restrict__ gu,
+                                         __nv_bfloat16* __restrict__ a, int64_t M, int I) {
+  const int64_t per_row = I / 8;
+  const int64_t nv = M * per_row;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv;
+       v += stride) {
+    const int64_t m = v / per_row, c = v - m * per_row;
+    const __nv_bfloat16* row = gu + m * 2 * I;
+    float fg[8], fu[8], fa[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(row) + c), fg);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(row + I) + c), fu);
+    swiglu8(fg, fu, fa);
+    reinterpret_cast<uint4*>(a)[v] = pack8(fa);
+  }
+}
+
+__global__ void swiglu_packed_bwd_kernel(const __nv_bfloat16* __restrict__ gu,
+                                         const __nv_bfloat16* __restrict__ da,
+                                         __nv_bfloat16* __restrict__ dgu, int64_t M, int I) {
+  const int64_t per_row = I / 8;
+  const int64_t nv = M * per_row;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv;
+       v += stride) {
+    const int64_t m = v / per_row, c = v - m * per_row;
+    const __nv_bfloat16* row = gu + m * 2 * I;
+    __nv_bfloat16* drow = dgu + m * 2 * I;
+    float fg[8], fu[8], fd[8], og[8], ou[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(row) + c), fg);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(row + I) + c), fu);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(da) + v), fd);
+    swiglu_grad8(fg, fu, fd, og, ou);
+    reinterpret_cast<uint4*>(drow)[c] = pack8(og);
+    reinterpret_cast<uint4*>(drow + I)[c] = pack8(ou);
   }
 }
 
@@ -106,6 +159,18 @@ cudaError_t launch_swiglu_bwd(const __nv_bfloat16* g, const __nv_bfloat16* u,
                               const __nv_bfloat16* da, __nv_bfloat16* dg, __nv_bfloat16* du,
                               int64_t n, cudaStream_t stream) {
   swiglu_bwd_kernel<<<grid_for(n), 256, 0, stream>>>(g, u, da, dg, du, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_packed_fwd(const __nv_bfloat16* gu, __nv_bfloat16* a, int64_t M, int I,
+                                     cudaStream_t stream) {
+  swiglu_packed_fwd_kernel<<<grid_for(M * I), 256, 0, stream>>>(gu, a, M, I);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_packed_bwd(const __nv_bfloat16* gu, const __nv_bfloat16* da,
+                                     __nv_bfloat16* dgu, int64_t M, int I, cudaStream_t stream) {
+  swiglu_packed_bwd_kernel<<<grid_for(M * I), 256, 0, stream>>>(gu, da, dgu, M, I);
   return cudaGetLastError();
 }
 

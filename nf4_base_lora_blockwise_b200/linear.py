@@ -195,6 +195,25 @@ def swiglu_backward(g, u, da, dg=None, du=None):
     return dg, du
 
 
+def swiglu_packed_forward(gu, a=None):
+    """a = silu(g) u for a packed gate/up output gu [M, 2I] (g first)."""
+    M, I2 = gu.shape
+    if a is None:
+        a = torch.empty((M, I2 // 2), dtype=gu.dtype, device=gu.device)
+    abi.qlora_swiglu_packed_fwd(gu.data_ptr(), a.data_ptr(), M, I2 // 2, _stream())
+    return a
+
+
+def swiglu_packed_backward(gu, da, dgu=None):
+    """dgu [M, 2I]: dg and du in the packed layer's column order."""
+    if dgu is None:
+        dgu = torch.empty_like(gu)
+    M, I2 = gu.shape
+    abi.qlora_swiglu_packed_bwd(gu.data_ptr(), da.data_ptr(), dgu.data_ptr(), M, I2 // 2,
+                                _stream())
+    return dgu
+
+
 def device_error():
     """Synchronising: the device error word (0 = none), cleared after reading."""
     return abi.qlora_device_error()

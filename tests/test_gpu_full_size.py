@@ -105,39 +105,16 @@ def test_full_size_workload(name):
         check_one_linear(lin["X"], lin["dY"], lin, L, f"{name}/{L.name}")
 
 
-def test_full_size_mlp():
-    """The MLP workload: gate/up 4096->14336, SwiGLU, down 14336->4096 on 8192 tokens.  Each
-    linear is checked at full size on its actual input (down's input is the GPU's SwiGLU output;
-    the SwiGLU itself is checked elementwise on the sampled rows)."""
-    w = synth.workload("mlp_8b")
-    inp = synth.make_inputs(w, seed=0)
-    gate, up, down = w.linears
-    lg, lu, ld = inp["linears"]
-    X = inp["X"]
-    rows = synth.sample_rows(w.M).numpy()
-    # Upstream gradients of gate and up: seeded stand-ins with the recipe's spread.
-    _, Hg, _ = check_one_linear(X, _grad_like(w.M, gate.N, 1), lg, gate, "mlp/gate")
-    _, Hu, _ = check_one_linear(X, _grad_like(w.M, up.N, 2), lu, up, "mlp/up")
-    a = linear.swiglu_forward(Hg, Hu)
-    torch.cuda.synchronize()
-    ref_a = qlora.swiglu_forward(parity.f32(Hg)[rows], parity.f32(Hu)[rows])
-    assert qlora.rel_err(parity.f32(a)[rows], ref_a) <= 1e-2
-    check_one_linear(a.cpu(), inp["dY"], ld, down, "mlp/down")
-
-
-def test_full_size_packed_qkv():
-    """The packed-adapter workload: q 4096->4096, k and v 4096->1024 on one stacked NF4 weight
-    with their own r 16 adapters, sharing 4096 tokens, in the grouped launch sequence.  Codes
-    and absmax of the stacked weight bit-exact on sampled rows; h and dX on the sampled token
-    rows, per adapter; XA, dA and dB in full, per adapter."""
-    w = synth.workload("qkv_8b")
-    inp = synth.make_inputs(w, seed=0)
-    Ns = [L.N for L in w.linears]
-    L0 = w.linears[0]
-    W0 = torch.cat([d["W0"] for d in inp["linears"]])
-    A = torch.cat([d["A"] for d in inp["linears"]])
-    B = torch.cat([d["B"] for d in inp["linears"]])
-    X, dY = inp["X"].cuda(), inp["dY"].cuda()
+def check_packed(X_cpu, dY_cpu, lins, Ls, tag):
+    """Adapters sharing X packed into one layer, at full size: codes and absmax of the stacked
+    weight bit-exact on sampled rows; h and dX on the sampled token rows, h per adapter; XA, dA
+    and dB in full, per adapter.  Returns the GPU's packed output H."""
+    Ns = [L.N for L in Ls]
+    L0 = Ls[0]
+    W0 = torch.cat([d["W0"] for d in lins])
+    A = torch.cat([d["A"] for d in lins])
+    B = torch.cat([d["B"] for d in lins])
+    X, dY = X_cpu.cuda(), dY_cpu.cuda()
     wg = linear.nf4_pack(W0.cuda())
     H, XA = linear.grouped_forward(X, wg, A.cuda(), B.cuda(), Ns, L0.alpha)
     dX, dA, dB = linear.grouped_backward(dY, X, wg, A.cuda(), B.cuda(), XA, Ns, L0.alpha)
@@ -148,28 +125,60 @@ def test_full_size_packed_qkv():
     del wg
     Wd = parity.oracle_dequant(full)
     del full
-    rows = synth.sample_rows(w.M).numpy()
-    Xf, dYf = parity.f32(inp["X"]), parity.f32(inp["dY"])
+    M = X_cpu.shape[0]
+    rows = synth.sample_rows(M).numpy()
+    Xf, dYf = parity.f32(X_cpu), parity.f32(dY_cpu)
     Xr, dYr = Xf[rows].astype(np.float64), dYf[rows].astype(np.float64)
     s = L0.alpha / L0.r
     edges = np.cumsum([0] + Ns)
     r = L0.r
     dx_ref = np.zeros((len(rows), L0.K))
+    Hr = parity.f32(H)[rows]
+    XAf, dAf, dBf = parity.f32(XA), parity.f32(dA), parity.f32(dB)
     errs = {}
-    for g, d in enumerate(inp["linears"]):
+    for g, d in enumerate(lins):
         a, b = edges[g], edges[g + 1]
         Ag = parity.f32(d["A"]).astype(np.float64)
         Bg = parity.f32(d["B"]).astype(np.float64)
         h_ref = _rows_matmul(Xr, Wd[a:b]) + s * ((Xr @ Ag.T) @ Bg.T)
-        errs[f"h{g}"] = qlora.rel_err(parity.f32(H)[rows][:, a:b], h_ref)
+        errs[f"h{g}"] = qlora.rel_err(Hr[:, a:b], h_ref)
         dx_ref += _rows_matmul_t(dYr[:, a:b], Wd[a:b]) + s * ((dYr[:, a:b] @ Bg) @ Ag)
         wts = qlora.backward_weights(dYf[:, a:b], Xf, Ag, Bg, L0.alpha)
-        errs[f"XA{g}"] = qlora.rel_err(parity.f32(XA)[:, g * r:(g + 1) * r], wts["XA"])
-        errs[f"dA{g}"] = qlora.rel_err(parity.f32(dA)[g * r:(g + 1) * r], wts["dA"])
-        errs[f"dB{g}"] = qlora.rel_err(parity.f32(dB)[a:b], wts["dB"])
+        errs[f"XA{g}"] = qlora.rel_err(XAf[:, g * r:(g + 1) * r], wts["XA"])
+        errs[f"dA{g}"] = qlora.rel_err(dAf[g * r:(g + 1) * r], wts["dA"])
+        errs[f"dB{g}"] = qlora.rel_err(dBf[a:b], wts["dB"])
     errs["dX"] = qlora.rel_err(parity.f32(dX)[rows], dx_ref)
     for k, v in errs.items():
-        assert v <= parity.TOL, f"qkv_8b {k}: {v:.3e}"
+        assert v <= parity.TOL, f"{tag} {k}: {v:.3e}"
+    return H
+
+
+def test_full_size_mlp():
+    """The MLP workload in the bench's launch configuration: gate and up 4096->14336 packed
+    into one layer on 8192 tokens, the packed SwiGLU, down 14336->4096.  The packed layer is
+    checked per adapter with a seeded upstream gradient; down is checked on its actual input
+    (the GPU's SwiGLU output), and the SwiGLU elementwise on the sampled rows."""
+    w = synth.workload("mlp_8b")
+    inp = synth.make_inputs(w, seed=0)
+    gate, up, down = w.linears
+    lg, lu, ld = inp["linears"]
+    rows = synth.sample_rows(w.M).numpy()
+    H = check_packed(inp["X"], _grad_like(w.M, 2 * gate.N, 1), [lg, lu], [gate, up],
+                     "mlp/gate+up")
+    a = linear.swiglu_packed_forward(H)
+    torch.cuda.synchronize()
+    g, u = qlora.split_cols(parity.f32(H)[rows], [gate.N, up.N])
+    assert qlora.rel_err(parity.f32(a)[rows], qlora.swiglu_forward(g, u)) <= 1e-2
+    del H
+    check_one_linear(a.cpu(), inp["dY"], ld, down, "mlp/down")
+
+
+def test_full_size_packed_qkv():
+    """The packed-adapter workload: q 4096->4096, k and v 4096->1024 on one stacked NF4 weight
+    with their own r 16 adapters, sharing 4096 tokens, in the grouped launch sequence."""
+    w = synth.workload("qkv_8b")
+    inp = synth.make_inputs(w, seed=0)
+    check_packed(inp["X"], inp["dY"], inp["linears"], list(w.linears), "qkv_8b")
 
 
 def _grad_like(M, N, seed):

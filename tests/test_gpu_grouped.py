@@ -105,3 +105,20 @@ def test_grouped_recompute_xa_is_bit_identical():
     assert torch.equal(H, H2)
     for a, b, k in zip(saved, recomputed, ("dX", "dA", "dB")):
         assert torch.equal(a, b), k
+
+
+@pytest.mark.parametrize("M,I", [(3, 1000), (64, 14336 // 8)])
+def test_swiglu_packed_parity(M, I):
+    """SwiGLU on a packed gate/up output [M, 2I] against the oracle on its column blocks."""
+    gen = torch.Generator().manual_seed(M + I)
+    gu = torch.randn(M, 2 * I, generator=gen).to(torch.bfloat16)
+    da = torch.randn(M, I, generator=gen).to(torch.bfloat16)
+    a = linear.swiglu_packed_forward(gu.cuda())
+    dgu = linear.swiglu_packed_backward(gu.cuda(), da.cuda())
+    torch.cuda.synchronize()
+    g, u = qlora.split_cols(parity.f32(gu), [I, I])
+    assert qlora.rel_err(parity.f32(a), qlora.swiglu_forward(g, u)) <= 1e-2
+    rg, ru = qlora.swiglu_backward(g, u, parity.f32(da))
+    dg, du = qlora.split_cols(parity.f32(dgu), [I, I])
+    assert qlora.rel_err(dg, rg) <= 1e-2
+    assert qlora.rel_err(du, ru) <= 1e-2
