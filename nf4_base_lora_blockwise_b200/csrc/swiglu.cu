@@ -102,43 +102,51 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ g,
 
 // Packed gate/up: gu [M, 2I] holds g in columns [0, I) and u in [I, 2I) of every row (the
 // output of a packed gate/up layer); a and da are [M, I]; dgu [M, 2I] takes dg and du in the
-// same places (the upstream gradient of that layer).  I % 8 == 0.
+// same places (the upstream gradient of that layer).  I % 8 == 0.  Blocks walk rows and
+// threads the row's 8-element vectors, so no index is divided.
 __global__ void swiglu_packed_fwd_kernel(const __nv_bfloat16* __restrict__ gu,
                                          __nv_bfloat16* __restrict__ a, int64_t M, int I) {
-  const int64_t per_row = I / 8;
-  const int64_t nv = M * per_row;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv;
-       v += stride) {
-    const int64_t m = v / per_row, c = v - m * per_row;
-    const __nv_bfloat16* row = gu + m * 2 * I;
-    float fg[8], fu[8], fa[8];
-    unpack8(__ldg(reinterpret_cast<const uint4*>(row) + c), fg);
-    unpack8(__ldg(reinterpret_cast<const uint4*>(row + I) + c), fu);
-    swiglu8(fg, fu, fa);
-    reinterpret_cast<uint4*>(a)[v] = pack8(fa);
+  const int per_row = I / 8;
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const uint4* g4 = reinterpret_cast<const uint4*>(gu + m * 2 * I);
+    const uint4* u4 = reinterpret_cast<const uint4*>(gu + m * 2 * I + I);
+    uint4* a4 = reinterpret_cast<uint4*>(a + m * I);
+    for (int c = threadIdx.x; c < per_row; c += blockDim.x) {
+      float fg[8], fu[8], fa[8];
+      unpack8(__ldg(g4 + c), fg);
+      unpack8(__ldg(u4 + c), fu);
+      swiglu8(fg, fu, fa);
+      a4[c] = pack8(fa);
+    }
   }
 }
 
 __global__ void swiglu_packed_bwd_kernel(const __nv_bfloat16* __restrict__ gu,
                                          const __nv_bfloat16* __restrict__ da,
                                          __nv_bfloat16* __restrict__ dgu, int64_t M, int I) {
-  const int64_t per_row = I / 8;
-  const int64_t nv = M * per_row;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv;
-       v += stride) {
-    const int64_t m = v / per_row, c = v - m * per_row;
-    const __nv_bfloat16* row = gu + m * 2 * I;
-    __nv_bfloat16* drow = dgu + m * 2 * I;
-    float fg[8], fu[8], fd[8], og[8], ou[8];
-    unpack8(__ldg(reinterpret_cast<const uint4*>(row) + c), fg);
-    unpack8(__ldg(reinterpret_cast<const uint4*>(row + I) + c), fu);
-    unpack8(__ldg(reinterpret_cast<const uint4*>(da) + v), fd);
-    swiglu_grad8(fg, fu, fd, og, ou);
-    reinterpret_cast<uint4*>(drow)[c] = pack8(og);
-    reinterpret_cast<uint4*>(drow + I)[c] = pack8(ou);
+  const int per_row = I / 8;
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const uint4* g4 = reinterpret_cast<const uint4*>(gu + m * 2 * I);
+    const uint4* u4 = reinterpret_cast<const uint4*>(gu + m * 2 * I + I);
+    const uint4* d4 = reinterpret_cast<const uint4*>(da + m * I);
+    uint4* dg4 = reinterpret_cast<uint4*>(dgu + m * 2 * I);
+    uint4* du4 = reinterpret_cast<uint4*>(dgu + m * 2 * I + I);
+    for (int c = threadIdx.x; c < per_row; c += blockDim.x) {
+      float fg[8], fu[8], fd[8], og[8], ou[8];
+      unpack8(__ldg(g4 + c), fg);
+      unpack8(__ldg(u4 + c), fu);
+      unpack8(__ldg(d4 + c), fd);
+      swiglu_grad8(fg, fu, fd, og, ou);
+      dg4[c] = pack8(og);
+      du4[c] = pack8(ou);
+    }
   }
+}
+
+// Rows per launch of the packed kernels: every row at once up to 16 blocks per SM.
+unsigned grid_rows(int64_t M) {
+  const int64_t cap = 148 * 16;
+  return static_cast<unsigned>(M < 1 ? 1 : (M > cap ? cap : M));
 }
 
 unsigned grid_for(int64_t n) {
@@ -164,13 +172,13 @@ cudaError_t launch_swiglu_bwd(const __nv_bfloat16* g, const __nv_bfloat16* u,
 
 cudaError_t launch_swiglu_packed_fwd(const __nv_bfloat16* gu, __nv_bfloat16* a, int64_t M, int I,
                                      cudaStream_t stream) {
-  swiglu_packed_fwd_kernel<<<grid_for(M * I), 256, 0, stream>>>(gu, a, M, I);
+  swiglu_packed_fwd_kernel<<<grid_rows(M), 256, 0, stream>>>(gu, a, M, I);
   return cudaGetLastError();
 }
 
 cudaError_t launch_swiglu_packed_bwd(const __nv_bfloat16* gu, const __nv_bfloat16* da,
                                      __nv_bfloat16* dgu, int64_t M, int I, cudaStream_t stream) {
-  swiglu_packed_bwd_kernel<<<grid_for(M * I), 256, 0, stream>>>(gu, da, dgu, M, I);
+  swiglu_packed_bwd_kernel<<<grid_rows(M), 256, 0, stream>>>(gu, da, dgu, M, I);
   return cudaGetLastError();
 }
 
