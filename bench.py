@@ -228,6 +228,63 @@ class LinearState:
                             dX=self.dX, dA=self.dA, dB=self.dB, ws=self.ws)
 
 
+class CeState:
+    """Device buffers of the LM head + cross-entropy on M tokens, in chunks: per step the label
+    count, then for each chunk the forward GEMM into the logits buffer, the cross-entropy rows
+    (token losses, gradient in place) and the dX GEMM, then the mean loss."""
+
+    def __init__(self, L, M, X, labels, W0, chunk, dev):
+        self.L, self.Mtot = L, M
+        self.chunk = min(chunk, M)
+        self.M, self.R, self.groups = self.chunk, 0, None  # tokens per GEMM launch
+        self.X, self.labels = X.to(dev), labels.to(dev)
+        self.w = linear.nf4_pack(W0.to(dev))
+        self.cw = self.w.c_struct()
+        self.z = torch.empty((self.chunk, L.N), dtype=torch.bfloat16, device=dev)
+        self.tl = torch.empty(M, dtype=torch.float32, device=dev)
+        self.cnt = torch.empty(64, dtype=torch.int32, device=dev)
+        self.loss = torch.empty(1, dtype=torch.float32, device=dev)
+        self.dX = torch.empty((M, L.K), dtype=torch.bfloat16, device=dev)
+        n = abi.qlora_lm_head_ce_workspace_bytes(M, L.N, L.K, self.chunk)
+        self.ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+
+    def twin(self):
+        t = copy.copy(self)
+        for name in ("X", "labels", "z", "tl", "cnt", "loss", "dX", "ws"):
+            setattr(t, name, torch.empty_like(getattr(self, name)))
+        return t
+
+    def stages(self, stream):
+        L, M, c, p = self.L, self.Mtot, self.chunk, lambda t: t.data_ptr()
+        ws, wsb = p(self.ws), self.ws.numel()
+        out = [("lm_head.ce_count",
+                lambda: abi.qlora_cross_entropy_count(p(self.labels), M, L.N, p(self.cnt), stream))]
+        for m0 in range(0, M, c):
+            mc = min(c, M - m0)
+            out += [
+                ("lm_head.gemm_fwd",
+                 lambda m0=m0, mc=mc: abi.qlora_nf4_gemm(p(self.X) + 2 * m0 * L.K, self.cw, 0, None,
+                                                         None, mc, 0, None, p(self.z), ws, wsb,
+                                                         stream)),
+                ("lm_head.ce_rows",
+                 lambda m0=m0, mc=mc: abi.qlora_cross_entropy_rows(
+                     p(self.z), mc, L.N, p(self.labels) + 4 * m0, p(self.cnt), p(self.tl) + 4 * m0,
+                     1, stream)),
+                ("lm_head.gemm_dx",
+                 lambda m0=m0, mc=mc: abi.qlora_nf4_gemm(p(self.z), self.cw, 1, None, None, mc, 0,
+                                                         None, p(self.dX) + 2 * m0 * L.K, ws, wsb,
+                                                         stream)),
+            ]
+        out.append(("lm_head.ce_mean",
+                    lambda: abi.qlora_cross_entropy_mean(p(self.tl), M, p(self.cnt), p(self.loss),
+                                                         stream)))
+        return out
+
+    def e2e(self):
+        linear.lm_head_ce(self.X, self.w, self.labels, chunk=self.chunk, dX=self.dX,
+                          token_loss=self.tl, ws=self.ws)
+
+
 class Step:
     """One step of a workload: its linears' states and the ordered (name, call) stages."""
 
@@ -235,8 +292,15 @@ class Step:
         self.w = w
         self.share_x = False
         self.pglue = None
+        self.ce = None
         inp = synth.make_inputs(w, seed=seed)
         bf = dict(dtype=torch.bfloat16, device=dev)
+        if w.ce:
+            st = CeState(w.linears[0], w.M, inp["X"], inp["labels"], inp["linears"][0]["W0"],
+                         synth.CE_CHUNK, dev)
+            self.states, self.ce, self.glue = [st], st, None
+            self.inputs = [(st, "X"), (st, "labels")]
+            return
         if w.grouped:
             # Adapters sharing X: one packed-adapter layer (stacked W0, A, B), or, unpacked,
             # one layer per adapter on the same X with its own column block of dY.
@@ -305,6 +369,11 @@ class Step:
     def twin(self):
         """A second set of step buffers over the same weights (see LinearState.twin)."""
         t = copy.copy(self)
+        if self.ce is not None:
+            t.ce = self.ce.twin()
+            t.states = [t.ce]
+            t.inputs = [(t.ce, "X"), (t.ce, "labels")]
+            return t
         if self.pglue is not None:
             sgu, sd = (st.twin() for st in self.pglue)
             t.a = torch.empty_like(self.a)
@@ -336,6 +405,8 @@ class Step:
 
     def stages(self, stream):
         p = lambda t: t.data_ptr()
+        if self.ce is not None:
+            return self.ce.stages(stream)
         if self.pglue is not None:
             sgu, sd = self.pglue
             M, I = self.a.shape
@@ -364,6 +435,9 @@ class Step:
     def e2e(self):
         """One step through the public Python entry points (linear.forward / backward and the
         SwiGLU glue), on the device buffers already holding this step's inputs."""
+        if self.ce is not None:
+            self.ce.e2e()
+            return
         if self.pglue is not None:
             sgu, sd = self.pglue
             sgu.forward()
@@ -392,6 +466,8 @@ class Step:
 
     def outputs(self):
         """Result tensors a user reads back after a step."""
+        if self.ce is not None:
+            return [self.ce.loss, self.ce.dX]
         if self.pglue is not None:
             sgu, sd = self.pglue
             return [sd.H, sgu.dX] + [t for st in self.states for t in (st.dA, st.dB)]
@@ -551,7 +627,10 @@ def roofline(step, per_stage, peaks, workload):
         st = next(s for s in step.states if s.L.name == lin_name)
         M, L, R = st.M, st.L, st.R  # R: packed rank columns (r for a single adapter)
         if stage.startswith("gemm"):
-            flops, byts = gemm_work(L, M, stage == "gemm_dx", R // L.r)
+            flops, byts = gemm_work(L, M, stage == "gemm_dx", R // L.r if L.r else 1)
+        elif stage.startswith("ce_"):
+            # the rows stage reads the chunk's logits and writes their gradient in place
+            flops, byts = 0.0, (4 * M * L.N if stage == "ce_rows" else 4 * st.Mtot)
         elif stage.startswith("lora_down"):
             # X A^T: every input column feeds R outputs; dY B: each feeds its adapter's r.
             C, per = (L.K, R) if stage.endswith("fwd") else (L.N, L.r)
@@ -593,7 +672,9 @@ def oracle_prepare(w, seed):
             eff = nf4.dq_effective_absmax(q8, sc).reshape(am.shape)
         else:
             eff = am
-        q = nf4.pack_codes(nf4.choose_codes(Wf, eff))
+        q = np.empty((L.N, L.K // 2), dtype=np.uint8)
+        for r0 in range(0, L.N, 8192):  # row chunks bound the host memory of the code choice
+            q[r0:r0 + 8192] = nf4.pack_codes(nf4.choose_codes(Wf[r0:r0 + 8192], eff[r0:r0 + 8192]))
         t1 = time.perf_counter()
         Wds.append(nf4.dequantize(q, eff, L.N, L.K).astype(np.float64))
         t_deq += time.perf_counter() - t1
@@ -607,6 +688,11 @@ def oracle_rows(w, prep, n):
     from oracle import qlora  # test infrastructure: only here and in the reference arm
     inp, Wds, _ = prep
     f64 = lambda t: t.float().numpy().astype(np.float64)
+    if w.ce:
+        from oracle import lm_head  # test infrastructure, as above
+        t0 = time.perf_counter()
+        lm_head.lm_head_ce(f64(inp["X"][:n]), Wds[0], inp["labels"][:n].numpy())
+        return time.perf_counter() - t0
     lora = [(f64(d["A"]), f64(d["B"])) for d in inp["linears"]]
     t0 = time.perf_counter()
     if w.grouped:
@@ -696,6 +782,9 @@ def workload_config(w, unpacked=False):
     if w.mlp:
         c["adapters"] = ("unpacked: gate and up as separate layers" if unpacked else
                          "gate and up packed into one layer on the shared input")
+    if w.ce:
+        c["loss"] = (f"cross-entropy over the {w.linears[0].N}-word vocabulary, uniform labels, "
+                     f"chunks of {synth.CE_CHUNK} tokens; frozen NF4 head, no adapter")
     return c
 
 

@@ -184,6 +184,39 @@ QLORA_API qlora_status qlora_swiglu_packed_fwd(const void* gu, void* a, int64_t 
 QLORA_API qlora_status qlora_swiglu_packed_bwd(const void* gu, const void* da, void* dgu,
                                                int64_t M, int I, qlora_stream_t stream);
 
+/* ---- LM head + cross-entropy over a frozen NF4 head, chunked over tokens. ----
+ * "Unsloth vs QLoRA vs Liger-Kernel", section 3 (fused cross-entropy): the projection to the
+ * vocabulary and the loss are computed in chunks of tokens so the [tokens x vocab] logits are
+ * never held at once.  For each chunk of `chunk` tokens (<= 0: all M at once):
+ *   z = X_c deq(W)^T                    [chunk, V] bf16 in the workspace (the dequant GEMM)
+ *   token_loss_m = logsumexp(z_m) - z_m[label_m]          (fp32, online max / sum of exp)
+ *   dz = (softmax(z) - onehot(label)) / count, in place   (only when dX is requested)
+ *   dX_c = dz deq(W)                    [chunk, K] bf16 (the dequant GEMM, transposed access)
+ * and loss = sum(token_loss) / count, count = number of labels in [0, V).  A label outside
+ * [0, V) (e.g. -100) ignores its token: loss 0, gradient 0, not counted; with no counted token
+ * loss and dX are 0.  W is the NF4 head [V, K] (V % 64 == 0, K % 64 == 0, K >= 128); it gets
+ * no gradient.
+ *   X [M, K] bf16, labels [M] int32 (device, read); loss [1] fp32 (device, written);
+ *   token_loss [M] fp32 (device, written; may be NULL); dX [M, K] bf16 (written; NULL: loss
+ *   only).  ws: device scratch of qlora_lm_head_ce_workspace_bytes(M, V, K, chunk) bytes,
+ *   about chunk x V x 2 plus the GEMM's partial sums. */
+QLORA_API size_t qlora_lm_head_ce_workspace_bytes(int M, int V, int K, int chunk);
+QLORA_API qlora_status qlora_lm_head_ce(const void* X, const qlora_nf4_weight* W, const int* labels,
+                                        int M, int chunk, float* loss, float* token_loss, void* dX,
+                                        void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Its cross-entropy stages, for custom compositions (the GEMMs are qlora_nf4_gemm with r = 0):
+ * count_out[0] = number of labels in [0, V); z [rows, V] bf16 (V % 8 == 0) -> token_loss
+ * [rows] and, with write_grad, z := (softmax(z) - onehot) / count_in[0] in place;
+ * loss[0] = sum(token_loss[0..M)) / count_in[0] (0 when the count is 0). */
+QLORA_API qlora_status qlora_cross_entropy_count(const int* labels, int M, int V, int* count_out,
+                                                 qlora_stream_t stream);
+QLORA_API qlora_status qlora_cross_entropy_rows(void* z, int rows, int V, const int* labels,
+                                                const int* count_in, float* token_loss,
+                                                int write_grad, qlora_stream_t stream);
+QLORA_API qlora_status qlora_cross_entropy_mean(const float* token_loss, int M, const int* count_in,
+                                                float* loss, qlora_stream_t stream);
+
 /* ---- The stages the two linear entry points are composed of (same validation rules). ---- */
 
 /* The stage calls take an optional adapter split, `group_rows` (host array of n_groups row
@@ -200,7 +233,8 @@ QLORA_API qlora_status qlora_lora_down(const void* in, int M, int C, const void*
                                        int n_groups, float scale, void* saved, void* scaled,
                                        void* ws, size_t ws_bytes, qlora_stream_t stream);
 
-/* The dequant GEMM with the fused rank-r extension:
+/* The dequant GEMM with the fused rank-r extension (r = 0: none, ext_w / ext_act may be NULL,
+ * and the reduction, K or N, must be at least 128):
  *   transpose_w = 0: out[M, N] = act[M, K] . deq(W0)^T + ext_act[M, r] . ext_w^T, ext_w = B [N, r]
  *   transpose_w = 1: out[M, K] = act[M, N] . deq(W0)   + ext_act[M, r] . ext_w,   ext_w = A [r, K]
  * act, ext_w, ext_act bf16 device (read); out bf16 device (written).  The scale s is expected

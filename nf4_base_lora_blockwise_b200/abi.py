@@ -34,6 +34,11 @@ EXPORTS = (
     "qlora_grouped_bwd",
     "qlora_swiglu_packed_fwd",
     "qlora_swiglu_packed_bwd",
+    "qlora_lm_head_ce_workspace_bytes",
+    "qlora_lm_head_ce",
+    "qlora_cross_entropy_count",
+    "qlora_cross_entropy_rows",
+    "qlora_cross_entropy_mean",
 )
 
 STATUS = {
@@ -102,6 +107,12 @@ def _lib():
             "qlora_grouped_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
             "qlora_swiglu_packed_fwd": (_I, [_VP, _VP, _I64, _I, _VP]),
             "qlora_swiglu_packed_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _VP]),
+            "qlora_lm_head_ce_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+            "qlora_lm_head_ce": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _I, _I, _VP, _VP, _VP,
+                                      _VP, _SZ, _VP]),
+            "qlora_cross_entropy_count": (_I, [_VP, _I, _I, _VP, _VP]),
+            "qlora_cross_entropy_rows": (_I, [_VP, _I, _I, _VP, _VP, _VP, _I, _VP]),
+            "qlora_cross_entropy_mean": (_I, [_VP, _I, _VP, _VP, _VP]),
             "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
                                        _VP]),
@@ -191,6 +202,31 @@ def qlora_swiglu_packed_fwd(gu, a, M, I, stream):
 
 def qlora_swiglu_packed_bwd(gu, da, dgu, M, I, stream):
     _check("qlora_swiglu_packed_bwd", _lib().qlora_swiglu_packed_bwd(gu, da, dgu, M, I, stream))
+
+
+def qlora_lm_head_ce_workspace_bytes(M, V, K, chunk):
+    return int(_lib().qlora_lm_head_ce_workspace_bytes(M, V, K, chunk))
+
+
+def qlora_lm_head_ce(X, weight, labels, M, chunk, loss, token_loss, dX, ws, ws_bytes, stream):
+    _check("qlora_lm_head_ce", _lib().qlora_lm_head_ce(X, ctypes.byref(weight), labels, M, chunk,
+                                                       loss, token_loss, dX, ws, ws_bytes,
+                                                       stream))
+
+
+def qlora_cross_entropy_count(labels, M, V, count_out, stream):
+    _check("qlora_cross_entropy_count", _lib().qlora_cross_entropy_count(labels, M, V, count_out,
+                                                                         stream))
+
+
+def qlora_cross_entropy_rows(z, rows, V, labels, count_in, token_loss, write_grad, stream):
+    _check("qlora_cross_entropy_rows", _lib().qlora_cross_entropy_rows(
+        z, rows, V, labels, count_in, token_loss, int(write_grad), stream))
+
+
+def qlora_cross_entropy_mean(token_loss, M, count_in, loss, stream):
+    _check("qlora_cross_entropy_mean", _lib().qlora_cross_entropy_mean(token_loss, M, count_in,
+                                                                       loss, stream))
 
 
 def qlora_swiglu_fwd(g, u, a, n, stream):

@@ -155,6 +155,15 @@ cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_
                              int r, const RowGroups& groups, float scale, float* out, bool out_cr,
                              float* partial, const GradPlan& plan, cudaStream_t stream);
 
+// ------------------------------ LM-head cross-entropy ---------------------------------------
+// count = number of labels in [0, V); z [rows, V] bf16 (V % 8 == 0) -> loss [rows] and, with
+// write_grad, z := (softmax(z) - onehot(label)) / count in place; out = sum(token_loss) / count.
+cudaError_t launch_ce_count(const int* labels, int M, int V, int* count, cudaStream_t stream);
+cudaError_t launch_ce_rows(__nv_bfloat16* z, int rows, int V, const int* labels, const int* count,
+                           float* loss, bool write_grad, cudaStream_t stream);
+cudaError_t launch_ce_mean(const float* token_loss, int M, const int* count, float* out,
+                           cudaStream_t stream);
+
 // ------------------------------ SwiGLU ------------------------------------------------------
 cudaError_t launch_swiglu_fwd(const __nv_bfloat16* g, const __nv_bfloat16* u, __nv_bfloat16* a,
                               int64_t n, cudaStream_t stream);

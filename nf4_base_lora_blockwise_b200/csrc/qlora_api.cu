@@ -266,6 +266,11 @@ qlora_status gemm_maps(GemmMaps* m, const qlora_nf4_weight* W, bool trans, const
     st = encode_2d(&m->q, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->q, W->K / 2, W->N, W->K / 2, 64, 64,
                    CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != QLORA_OK) return st;
+  if (r == 0) {  // no extension steps: the kernel never loads through these, only prefetches
+    m->ext_w = m->act;
+    m->ext_act = m->act;
+    return QLORA_OK;
+  }
   if (!trans)  // B_lora [N, r]
     st = encode_2d(&m->ext_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ext_w, r, W->N, r * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B);
@@ -603,16 +608,21 @@ qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int tran
                             const void* ext_w, const void* ext_act, int M, int r,
                             const int* group_rows, int n_groups, void* out, void* ws,
                             size_t ws_bytes, qlora_stream_t stream) {
-  if (!act || !ext_w || !ext_act || !out) return QLORA_ERR_NULL;
+  if (!act || !out || (r != 0 && (!ext_w || !ext_act))) return QLORA_ERR_NULL;
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  if (M < 1 || !rank_ok(r)) return QLORA_ERR_SHAPE;
+  if (M < 1 || (r != 0 && !rank_ok(r))) return QLORA_ERR_SHAPE;
+  // Without an extension a tile is its reduction steps alone; the dequant groups take two
+  // steps at a time, so there must be at least two of them.
+  if (r == 0 && (transpose_w ? W->N : W->K) < 128) return QLORA_ERR_SHAPE;
+  if (r == 0 && group_rows) return QLORA_ERR_SHAPE;
   RowGroups g = single_group(transpose_w ? W->K : W->N);
   if (group_rows) {  // forward only: adapters along W0's rows, ext_act [M, n, r]
     if (transpose_w) return QLORA_ERR_SHAPE;
     if ((st = make_groups(group_rows, n_groups, W->N, r, &g)) != QLORA_OK) return st;
   }
-  if (!aligned16(act) || !aligned16(ext_w) || !aligned16(ext_act) || !aligned16(out))
+  if (!aligned16(act) || (ext_w && !aligned16(ext_w)) || (ext_act && !aligned16(ext_act)) ||
+      !aligned16(out))
     return QLORA_ERR_ALIGN;
   const size_t need = gemm_ws_bytes(M, W->N, W->K, g.n * r, transpose_w != 0);
   if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
@@ -711,6 +721,109 @@ qlora_status qlora_swiglu_packed_bwd(const void* gu, const void* da, void* dgu, 
   st = cuda_status(launch_swiglu_packed_bwd(
       static_cast<const __nv_bfloat16*>(gu), static_cast<const __nv_bfloat16*>(da),
       static_cast<__nv_bfloat16*>(dgu), M, I, static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+size_t qlora_lm_head_ce_workspace_bytes(int M, int V, int K, int chunk) {
+  if (M < 1 || V < 64 || V % 64 || K < 128 || K % 64) return 0;
+  const int c = chunk < 1 || chunk > M ? M : chunk;
+  const size_t scratch = std::max(gemm_ws_bytes(c, V, K, 0, false), gemm_ws_bytes(c, V, K, 0, true));
+  return align256(static_cast<size_t>(c) * V * 2) + align256(static_cast<size_t>(M) * 4) + 256 +
+         align256(scratch);
+}
+
+qlora_status qlora_lm_head_ce(const void* X, const qlora_nf4_weight* W, const int* labels, int M,
+                              int chunk, float* loss, float* token_loss, void* dX, void* ws,
+                              size_t ws_bytes, qlora_stream_t stream) {
+  if (!X || !labels || !loss) return QLORA_ERR_NULL;
+  qlora_status st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  const int V = W->N, K = W->K;
+  if (M < 1 || K < 128) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(labels) || !aligned16(loss) ||
+      (token_loss && !aligned16(token_loss)) || (dX && !aligned16(dX)))
+    return QLORA_ERR_ALIGN;
+  const int c = chunk < 1 || chunk > M ? M : chunk;
+  const size_t need = qlora_lm_head_ce_workspace_bytes(M, V, K, chunk);
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  int dev;
+  if ((st = current_device(&dev)) != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Workspace: logits chunk [c, V] bf16 | token losses [M] fp32 | count | GEMM partial sums.
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  auto* z = reinterpret_cast<__nv_bfloat16*>(w8);
+  size_t off = align256(static_cast<size_t>(c) * V * 2);
+  float* tl = token_loss ? token_loss : reinterpret_cast<float*>(w8 + off);
+  off += align256(static_cast<size_t>(M) * 4);
+  int* cnt = reinterpret_cast<int*>(w8 + off);
+  off += 256;
+  void* scratch = w8 + off;
+  const size_t scratch_bytes = need - off;
+
+  if ((st = cuda_status(launch_ce_count(labels, M, V, cnt, s))) != QLORA_OK) return st;
+  count(1);
+  const auto* x = static_cast<const __nv_bfloat16*>(X);
+  auto* dx = static_cast<__nv_bfloat16*>(dX);
+  for (int m0 = 0; m0 < M; m0 += c) {
+    const int mc = std::min(c, M - m0);
+    // z = X_c deq(W)^T: the chunk's logits, then its loss rows and (with dX) the gradient
+    // dz = (softmax(z) - onehot) / count in place, then dX_c = dz deq(W).
+    st = do_gemm(x + static_cast<size_t>(m0) * K, W, false, nullptr, nullptr, mc, 0,
+                 single_group(V), z, err, scratch, scratch_bytes, s);
+    if (st != QLORA_OK) return st;
+    st = cuda_status(launch_ce_rows(z, mc, V, labels + m0, cnt, tl + m0, dX != nullptr, s));
+    if (st != QLORA_OK) return st;
+    count(1);
+    if (dX) {
+      st = do_gemm(z, W, true, nullptr, nullptr, mc, 0, single_group(K),
+                   dx + static_cast<size_t>(m0) * K, err, scratch, scratch_bytes, s);
+      if (st != QLORA_OK) return st;
+    }
+  }
+  st = cuda_status(launch_ce_mean(tl, M, cnt, loss, s));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+qlora_status qlora_cross_entropy_count(const int* labels, int M, int V, int* count_out,
+                                       qlora_stream_t stream) {
+  if (!labels || !count_out) return QLORA_ERR_NULL;
+  if (M < 1 || V < 8 || V % 8) return QLORA_ERR_SHAPE;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_ce_count(labels, M, V, count_out, static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+qlora_status qlora_cross_entropy_rows(void* z, int rows, int V, const int* labels,
+                                      const int* count_in, float* token_loss, int write_grad,
+                                      qlora_stream_t stream) {
+  if (!z || !labels || !count_in || !token_loss) return QLORA_ERR_NULL;
+  if (rows < 1 || V < 8 || V % 8) return QLORA_ERR_SHAPE;
+  if (!aligned16(z)) return QLORA_ERR_ALIGN;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_ce_rows(static_cast<__nv_bfloat16*>(z), rows, V, labels, count_in,
+                                  token_loss, write_grad != 0, static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
+qlora_status qlora_cross_entropy_mean(const float* token_loss, int M, const int* count_in,
+                                      float* loss, qlora_stream_t stream) {
+  if (!token_loss || !count_in || !loss) return QLORA_ERR_NULL;
+  if (M < 1) return QLORA_ERR_SHAPE;
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  st = cuda_status(launch_ce_mean(token_loss, M, count_in, loss, static_cast<cudaStream_t>(stream)));
   if (st == QLORA_OK) count(1);
   return st;
 }

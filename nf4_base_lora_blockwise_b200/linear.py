@@ -214,6 +214,29 @@ def swiglu_packed_backward(gu, da, dgu=None):
     return dgu
 
 
+def lm_head_ce(X, w: NF4Weight, labels, chunk=1024, need_dx=True, dX=None, token_loss=None,
+               ws=None):
+    """Chunked LM head + cross-entropy (qlora_lm_head_ce): X [M, K] bf16, w the NF4 head
+    [V, K], labels [M] int32 (outside [0, V): ignored).  Returns (loss [1] fp32, token_loss
+    [M] fp32, dX [M, K] bf16 or None)."""
+    M = X.shape[0]
+    _need(X, torch.bfloat16, (M, w.K), "X")
+    _need(labels, torch.int32, (M,), "labels")
+    dev = X.device
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    if token_loss is None:
+        token_loss = torch.empty(M, dtype=torch.float32, device=dev)
+    if need_dx and dX is None:
+        dX = torch.empty((M, w.K), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        n = abi.qlora_lm_head_ce_workspace_bytes(M, w.N, w.K, chunk)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    abi.qlora_lm_head_ce(X.data_ptr(), w.c_struct(), labels.data_ptr(), M, chunk,
+                         loss.data_ptr(), token_loss.data_ptr(), _ptr(dX) if need_dx else None,
+                         ws.data_ptr(), ws.numel(), _stream())
+    return loss, token_loss, (dX if need_dx else None)
+
+
 def device_error():
     """Synchronising: the device error word (0 = none), cleared after reading."""
     return abi.qlora_device_error()

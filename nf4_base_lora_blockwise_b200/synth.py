@@ -8,7 +8,8 @@ Recipe: one ``torch.Generator`` (CPU) seeded with ``seed`` draws, in this order:
 linear (or independent projections, one after the other) X, W0, A, B, dY; for the MLP
 workload X, then W0, A, B of gate, up and down, then dY; for a packed-adapter workload (q/k/v
 sharing X) X, then W0, A, B of each adapter, then dY over all adapters' outputs.  Values are
-drawn in fp32 and cast to bf16 (round to nearest even).  "N(0, s)" means standard deviation s.  The LoRA down-projection A is either uniform
+drawn in fp32 and cast to bf16 (round to nearest even).  The LM-head workload draws X, the
+head W0 and then int32 labels uniform over the vocabulary.  "N(0, s)" means standard deviation s.  The LoRA down-projection A is either uniform
 on (-a, a) with a = 1/sqrt(in) ("Kaiming-uniform" with torch's nn.Linear default slope
 sqrt(5)), or the explicit bound of the tiny workload.  B is N(0, 0.01) -- non-zero, so the
 LoRA path contributes to h and to dX.
@@ -45,6 +46,7 @@ class Workload:
     mlp: bool = False             # gate/up -> SwiGLU -> down
     notes: str = ""
     grouped: bool = False         # the linears share X and run as one packed-adapter layer
+    ce: bool = False              # one frozen NF4 LM head (r = 0) + cross-entropy on labels
 
 
 def _lin(name, K, N, r, alpha, w_std=0.02, dq=False):
@@ -75,6 +77,12 @@ WORKLOADS["qkv_8b"] = Workload("qkv_8b", 4096, (_lin("q_proj", 4096, 4096, 16, 3
                                                 _lin("v_proj", 4096, 1024, 16, 32.0)),
                                grouped=True)
 
+# Llama-3-8B LM head 4096 -> 128256 (frozen, no adapter) + cross-entropy on 4096 tokens with
+# uniform labels, processed in chunks of 1024 tokens.
+WORKLOADS["lm_head_ce_8b"] = Workload("lm_head_ce_8b", 4096,
+                                      (_lin("lm_head", 4096, 128256, 0, 0.0),), ce=True)
+CE_CHUNK = 1024
+
 # Token-count sweep on 4096 -> 14336, r 16, alpha 32.
 SWEEP_M = (1, 16, 128, 1024, 16384)
 for _m in SWEEP_M:
@@ -87,7 +95,7 @@ def workload(name, M=None):
     w = WORKLOADS[name]
     if M is not None and M != w.M:
         w = Workload(w.name, M, w.linears, w.x_std, w.dy_std, w.a_bound, w.b_std, w.mlp,
-                     w.notes, w.grouped)
+                     w.notes, w.grouped, w.ce)
     return w
 
 
@@ -122,6 +130,12 @@ def make_inputs(w, seed=0):
         return {"W0": W0, "A": A, "B": B}
 
     lins = []
+    if w.ce:
+        L = w.linears[0]
+        X = _normal(gen, (w.M, L.K), w.x_std)
+        W0 = _normal(gen, (L.N, L.K), L.w_std)
+        labels = torch.randint(0, L.N, (w.M,), generator=gen, dtype=torch.int64).to(torch.int32)
+        return {"X": X, "linears": [{"W0": W0}], "labels": labels}
     if w.grouped:
         X = _normal(gen, (w.M, w.linears[0].K), w.x_std)
         for L in w.linears:
@@ -159,6 +173,19 @@ def make_grouped(M, K, Ns, r, alpha=None, seed=0, x_std=1.0, w_std=0.02, a_bound
     w = Workload("adhoc_grouped", M, lins, x_std=x_std, dy_std=dy_std, a_bound=a_bound,
                  b_std=b_std, grouped=True)
     return make_inputs(w, seed)
+
+
+def make_lm_head(M, K, V, seed=0, ignore_frac=0.0, x_std=1.0, w_std=0.02):
+    """Inputs of an ad-hoc LM head + cross-entropy: X [M, K], W0 [V, K], labels [M] int32
+    uniform in [0, V), of which a seeded fraction is replaced by -100 (ignored)."""
+    w = Workload("adhoc_ce", M, (_lin("lm_head", K, V, 0, 0.0, w_std),), x_std=x_std, ce=True)
+    inp = make_inputs(w, seed)
+    if ignore_frac > 0:
+        gen = torch.Generator(device="cpu")
+        gen.manual_seed(seed + 1)
+        drop = torch.rand(M, generator=gen) < ignore_frac
+        inp["labels"] = torch.where(drop, torch.full_like(inp["labels"], -100), inp["labels"])
+    return inp
 
 
 def sample_rows(M, count=512, seed=1234):
