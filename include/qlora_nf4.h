@@ -27,6 +27,11 @@
  *   Codebook: the 16 NormalFloat levels (asymmetric N(0,1) quantiles with an exact zero,
  *   normalised to [-1, 1]) in fp32; code c dequantises to bf16(fp32(level[c] * absmax)).
  *
+ * Beyond the single layer: several adapters sharing X packed into one layer
+ * (qlora_grouped_*), the layer without a saved X A^T (XA_saved = NULL: recomputed), the
+ * SwiGLU glue (flat or on a packed gate/up output) and the LM head + cross-entropy over a
+ * frozen NF4 head, chunked over tokens (qlora_lm_head_ce).
+ *
  * Conventions for every entry point:
  *   - Pointers named as device memory are caller-owned device allocations on the current
  *     device; the library allocates nothing and keeps no state between calls.
