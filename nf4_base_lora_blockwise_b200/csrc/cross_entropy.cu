@@ -27,14 +27,21 @@ __device__ __forceinline__ void unpack8_bf16(const uint4 v, float (&f)[8]) {
   }
 }
 
-// Running (max, sum of exp(x - max)) pairs, combined exactly as the online softmax does.
-__device__ __forceinline__ void ms_add(float& m, float& s, float x) {
-  if (x > m) {
-    s = s * expf(m - x) + 1.f;
-    m = x;
-  } else {
-    s += expf(x - m);
+// Running (max, sum of exp(x - max)) pairs, combined as the online softmax does: eight values
+// at a time, so the running pair is rescaled once per vector and the eight exponentials are
+// independent of one another.
+__device__ __forceinline__ void ms_add8(float& m, float& s, const float (&f)[8]) {
+  float m8 = f[0];
+#pragma unroll
+  for (int k = 1; k < 8; ++k) m8 = fmaxf(m8, f[k]);
+  if (m8 > m) {
+    s *= __expf(m - m8);
+    m = m8;
   }
+  float t = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) t += __expf(f[k] - m);
+  s += t;
 }
 __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2) {
   if (m2 > m) {
@@ -79,8 +86,7 @@ __global__ void __launch_bounds__(kCeThreads) ce_rows_kernel(__nv_bfloat16* __re
   for (int i = tid; i < nv; i += kCeThreads) {
     float f[8];
     unpack8_bf16(z4[i], f);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) ms_add(m, s, f[k]);
+    ms_add8(m, s, f);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -116,8 +122,8 @@ __global__ void __launch_bounds__(kCeThreads) ce_rows_kernel(__nv_bfloat16* __re
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int v0 = i * 8 + 2 * k;
-      const float g0 = (expf(f[2 * k] - lse) - (v0 == label ? 1.f : 0.f)) * scale;
-      const float g1 = (expf(f[2 * k + 1] - lse) - (v0 + 1 == label ? 1.f : 0.f)) * scale;
+      const float g0 = (__expf(f[2 * k] - lse) - (v0 == label ? 1.f : 0.f)) * scale;
+      const float g1 = (__expf(f[2 * k + 1] - lse) - (v0 + 1 == label ? 1.f : 0.f)) * scale;
       const __nv_bfloat162 p = __floats2bfloat162_rn(g0, g1);
       ow[k] = *reinterpret_cast<const uint32_t*>(&p);
     }
