@@ -723,7 +723,12 @@ def oracle_desc(w, n):
             f"per linear per step charged per batch of M tokens; quantisation not timed")
 
 
+ORACLE_THREADS = 0  # set from --oracle-threads; 0 = all host cores
+
+
 def blas_threads():
+    if ORACLE_THREADS > 0:
+        return ORACLE_THREADS
     try:
         from threadpoolctl import threadpool_info
         return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
@@ -817,6 +822,9 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="launch every stage from Python instead of replaying a CUDA graph")
+    ap.add_argument("--oracle-threads", type=int, default=0,
+                    help="BLAS threads for the oracle legs (cpu_baseline, --impl reference); "
+                         "0 = all host cores")
     ap.add_argument("--unpacked", action="store_true",
                     help="adapters sharing an input (qkv_8b, mlp_8b's gate/up) run as "
                          "separate layers")
@@ -824,6 +832,11 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
+    if args.oracle_threads > 0:
+        from threadpoolctl import threadpool_limits
+        global ORACLE_THREADS, _ORACLE_LIMITS
+        ORACLE_THREADS = args.oracle_threads
+        _ORACLE_LIMITS = threadpool_limits(args.oracle_threads, user_api="blas")
     if args.impl == "reference":
         run_reference(args)
         return
