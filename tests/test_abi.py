@@ -135,3 +135,33 @@ def test_xa_saved_may_be_null(lib):
                                  32.0, FAKE, FAKE, FAKE, FAKE, 16, None) == 5
     assert lib.qlora_linear_fwd(FAKE, ctypes.byref(W), FAKE, FAKE, 64, 16, 32.0, FAKE, FAKE + 8,
                                 FAKE, 1 << 30, None) == 3
+
+
+def test_lm_head_and_plain_gemm_validation(lib):
+    """LM head + cross-entropy and the GEMM without extension: argument checks answer before
+    any device work."""
+    head = _w(N=1024, K=256)
+    args = lambda W=head, X=FAKE, labels=FAKE, loss=FAKE, ws_bytes=1 << 34: (
+        X, ctypes.byref(W), labels, 64, 16, loss, None, FAKE, FAKE, ws_bytes, None)
+    assert lib.qlora_lm_head_ce(*args(X=None)) == 1
+    assert lib.qlora_lm_head_ce(*args(labels=None)) == 1
+    assert lib.qlora_lm_head_ce(*args(loss=None)) == 1
+    assert lib.qlora_lm_head_ce(*args(W=_w(N=1024, K=64))) == 2      # K < 128
+    assert lib.qlora_lm_head_ce(*args(W=_w(N=1000, K=256))) == 2     # V % 64
+    assert lib.qlora_lm_head_ce(*args(ws_bytes=16)) == 5
+    need = lib.qlora_lm_head_ce_workspace_bytes(64, 1024, 256, 16)
+    assert need >= 16 * 1024 * 2 + 64 * 4                          # one chunk of logits + losses
+    assert lib.qlora_lm_head_ce_workspace_bytes(64, 1024, 256, 0) >= 64 * 1024 * 2
+    assert lib.qlora_lm_head_ce_workspace_bytes(64, 1024, 64, 16) == 0
+    # r = 0: no extension operands needed, but the reduction must be >= 128 and unsplit.
+    W = _w(N=128, K=64)
+    assert lib.qlora_nf4_gemm(FAKE, ctypes.byref(W), 0, None, None, 64, 0, None, 0, FAKE, FAKE,
+                              1 << 30, None) == 2                  # K = 64: one step per tile
+    W = _w(N=128, K=256)
+    arr = (ctypes.c_int * 1)(128)
+    assert lib.qlora_nf4_gemm(FAKE, ctypes.byref(W), 0, None, None, 64, 0, arr, 1, FAKE, FAKE,
+                              1 << 30, None) == 2                  # no adapter split without r
+    assert lib.qlora_nf4_gemm(FAKE, ctypes.byref(W), 0, None, None, 64, 8, None, 0, FAKE, FAKE,
+                              1 << 30, None) == 1                  # r > 0 needs its operands
+    assert lib.qlora_cross_entropy_rows(FAKE, 4, 100, FAKE, FAKE, FAKE, 1, None) == 2  # V % 8
+    assert lib.qlora_cross_entropy_count(None, 4, 128, FAKE, None) == 1
