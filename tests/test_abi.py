@@ -165,3 +165,28 @@ def test_lm_head_and_plain_gemm_validation(lib):
                               1 << 30, None) == 1                  # r > 0 needs its operands
     assert lib.qlora_cross_entropy_rows(FAKE, 4, 100, FAKE, FAKE, FAKE, 1, None) == 2  # V % 8
     assert lib.qlora_cross_entropy_count(None, 4, 128, FAKE, None) == 1
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/qlora_nf4.h is a C header: a C11 translation unit that includes it and calls
+    every entry point compiles with gcc (syntax and types only)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "qlora_nf4.h"\n'
+                   "int main(void) {\n"
+                   "  qlora_nf4_weight w = {0};\n"
+                   "  size_t n = qlora_workspace_bytes(64, 128, 128, 16);\n"
+                   "  n += qlora_grouped_workspace_bytes(64, 256, 128, 16, 2);\n"
+                   "  n += qlora_lm_head_ce_workspace_bytes(64, 1024, 256, 16);\n"
+                   "  (void)qlora_linear_fwd(0, &w, 0, 0, 64, 16, 32.0f, 0, 0, 0, n, 0);\n"
+                   "  (void)qlora_status_str(QLORA_OK);\n"
+                   "  return 0;\n"
+                   "}\n")
+    r = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-fsyntax-only",
+                        "-I" + os.path.join(ROOT, "include"), str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
