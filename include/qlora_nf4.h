@@ -264,6 +264,15 @@ QLORA_API qlora_status qlora_lora_grad(const void* big, int M, int C, const void
                                        float* out, int out_r_by_c, void* ws, size_t ws_bytes,
                                        qlora_stream_t stream);
 
+/* Host-only (no GPU needed): the dequant GEMM's launch plan for a problem of M tokens, rows_w
+ * output rows (N for the forward, K for dX) and steps_per_tile 64-deep reduction steps (K/64
+ * or N/64, plus the extension's) on a device with sm_count SMs.  Writes the token tile (bt
+ * tokens per MMA, nh halves per tile), the schedule (0: whole tiles, one CTA per SM; 1:
+ * stream-K), the grid and the stream-K partial-sum bytes the workspace must hold. */
+QLORA_API qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count,
+                                       int* bt, int* nh, int* streamk, int* grid,
+                                       size_t* partial_bytes);
+
 /* Number of kernels this library has launched in this process so far (all devices). */
 QLORA_API uint64_t qlora_launch_counter(void);
 

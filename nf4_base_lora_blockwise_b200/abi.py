@@ -39,6 +39,7 @@ EXPORTS = (
     "qlora_cross_entropy_count",
     "qlora_cross_entropy_rows",
     "qlora_cross_entropy_mean",
+    "qlora_gemm_plan",
 )
 
 STATUS = {
@@ -113,6 +114,9 @@ def _lib():
             "qlora_cross_entropy_count": (_I, [_VP, _I, _I, _VP, _VP]),
             "qlora_cross_entropy_rows": (_I, [_VP, _I, _I, _VP, _VP, _VP, _I, _VP]),
             "qlora_cross_entropy_mean": (_I, [_VP, _I, _VP, _VP, _VP]),
+            "qlora_gemm_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                     ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                     ctypes.POINTER(_SZ)]),
             "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
                                        _VP]),
@@ -265,6 +269,17 @@ def qlora_lora_grad(big, M, C, small, r, group_rows, scale, out, out_r_by_c, ws,
     rows, n = _groups(group_rows)
     _check("qlora_lora_grad", _lib().qlora_lora_grad(big, M, C, small, r, rows, n, float(scale),
                                                      out, int(out_r_by_c), ws, ws_bytes, stream))
+
+
+def qlora_gemm_plan(M, rows_w, steps_per_tile, sm_count):
+    """dict(bt, nh, streamk, grid, partial_bytes) of the dequant GEMM's launch plan."""
+    v = [_I() for _ in range(4)]
+    pb = _SZ()
+    _check("qlora_gemm_plan", _lib().qlora_gemm_plan(M, rows_w, steps_per_tile, sm_count,
+                                                     *[ctypes.byref(x) for x in v],
+                                                     ctypes.byref(pb)))
+    return {"bt": v[0].value, "nh": v[1].value, "streamk": v[2].value, "grid": v[3].value,
+            "partial_bytes": pb.value}
 
 
 def qlora_launch_counter():

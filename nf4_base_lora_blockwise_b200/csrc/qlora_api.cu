@@ -656,6 +656,20 @@ qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, i
                       static_cast<float*>(ws), static_cast<cudaStream_t>(stream));
 }
 
+qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count, int* bt,
+                             int* nh, int* streamk, int* grid, size_t* partial_bytes) {
+  if (!bt || !nh || !streamk || !grid || !partial_bytes) return QLORA_ERR_NULL;
+  if (M < 1 || rows_w < 1 || steps_per_tile < 2 || sm_count < 1) return QLORA_ERR_SHAPE;
+  const GemmTile t = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count);
+  const GemmSchedule sc = gemm_schedule(M, rows_w, steps_per_tile, sm_count);
+  *bt = t.bt;
+  *nh = t.nh;
+  *streamk = sc.streamk;
+  *grid = sc.grid;
+  *partial_bytes = 4 * sc.partial_floats;
+  return QLORA_OK;
+}
+
 uint64_t qlora_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
 
 qlora_status qlora_swiglu_fwd(const void* g, const void* u, void* a, int64_t n,

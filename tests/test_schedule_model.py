@@ -142,3 +142,59 @@ def test_step_cursor_matches_division():
                 if k >= total:
                     k -= total
                     t += 1 if streamk else G
+
+
+def test_gemm_plan_properties():
+    """The dequant GEMM's launch plan (qlora_gemm_plan, host only) on random problems:
+    * token tiles: one half of M rounded up to 16 for M <= 256, else two halves of a multiple
+      of 16 in [128, 256];
+    * stream-K exactly when 512-token tiles would leave SMs idle;
+    * the grid and the partial-sum bytes that follow from the schedule;
+    * qlora_workspace_bytes covers the partial sums of both GEMMs of a layer for every device
+      of up to 160 SMs."""
+    import os
+    from nf4_base_lora_blockwise_b200 import abi
+    if not os.path.exists(abi.LIB_PATH):
+        from nf4_base_lora_blockwise_b200 import build
+        build.build()
+    rng = random.Random(17)
+    for _ in range(400):
+        M = rng.choice([1, 7, 16, 33, 128, 200, 256, 257, 300, 1024, 2048, 4096, 8192, 16384])
+        N, K = 64 * rng.randint(1, 300), 64 * rng.randint(2, 300)
+        r = rng.choice([8, 16, 64])
+        sms = rng.choice([132, 148, 160])
+        for trans in (False, True):
+            rows, steps = (K, N // 64) if trans else (N, K // 64)
+            steps += ((r + 15) // 16 * 16 + 63) // 64
+            p = abi.qlora_gemm_plan(M, rows, steps, sms)
+            if M <= 256:
+                assert p["nh"] == 1 and p["bt"] == max(16, (M + 15) // 16 * 16)
+            else:
+                assert p["nh"] == 2 and p["bt"] % 16 == 0 and 128 <= p["bt"] <= 256
+            G = min(sms, 160)
+            tt = p["bt"] * p["nh"]
+            tiles = ((rows + 127) // 128) * ((M + tt - 1) // tt)
+            wide = ((rows + 127) // 128) * ((M + (512 if M > 256 else tt) - 1)
+                                           // (512 if M > 256 else tt))
+            assert p["streamk"] == (1 if wide < G else 0)
+            if p["streamk"]:
+                assert p["bt"] == (256 if M > 256 else p["bt"])
+                assert p["grid"] == min(tiles * steps, G)
+                assert p["partial_bytes"] == p["grid"] * 2 * tt * 128 * 4
+            else:
+                assert p["grid"] == G and tiles >= G and p["partial_bytes"] == 0
+        if M > 32:  # the few-token forward has its own slots; larger M uses these GEMMs only
+            need = abi.qlora_workspace_bytes(M, N, K, r)
+            for trans in (False, True):
+                rows, steps = (K, N // 64) if trans else (N, K // 64)
+                steps += ((r + 15) // 16 * 16 + 63) // 64
+                for s2 in (100, 132, 148, 160):
+                    assert abi.qlora_gemm_plan(M, rows, steps, s2)["partial_bytes"] <= need
+
+
+def test_gemm_plan_headline_tile():
+    """q_proj 4096 -> 4096 at 4096 tokens on 148 SMs: 480-token tiles (288 tiles, two per CTA
+    on 140 CTAs) instead of 512 (256 tiles, where 108 CTAs run two)."""
+    from nf4_base_lora_blockwise_b200 import abi
+    p = abi.qlora_gemm_plan(4096, 4096, 64 + 1, 148)
+    assert (p["bt"], p["nh"], p["streamk"], p["grid"]) == (240, 2, 0, 148)
