@@ -300,6 +300,13 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_w
 /* Size in bytes of the fixed scratch array used by qlora_linear_fwd_noalloc. */
 QLORA_API size_t qlora_noalloc_scratch_bytes(void);
 
+/* Self-test of the failure detection: enqueues one thread that waits, through the kernels'
+ * own bounded wait, on a barrier nothing completes.  The wait runs out after its 2 s limit and
+ * the kernel returns; a following qlora_device_error() then reports QLORA_ERR_TIMEOUT with
+ * code 6 (the self-test's site, CTA 0, tag 0), provided the word was clear before.  The
+ * context stays usable. */
+QLORA_API qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream);
+
 /* Synchronising: returns the device error word of the current device (0 = none; otherwise
  * a code naming the wait that ran out) and clears it. */
 QLORA_API qlora_status qlora_device_error(int* code);

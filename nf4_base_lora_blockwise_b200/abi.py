@@ -40,6 +40,7 @@ EXPORTS = (
     "qlora_cross_entropy_rows",
     "qlora_cross_entropy_mean",
     "qlora_gemm_plan",
+    "qlora_selftest_bounded_wait",
 )
 
 STATUS = {
@@ -105,6 +106,7 @@ def _lib():
                                               _F, _VP, _VP, _VP]),
             "qlora_noalloc_scratch_bytes": (_SZ, []),
             "qlora_device_error": (_I, [ctypes.POINTER(ctypes.c_int)]),
+            "qlora_selftest_bounded_wait": (_I, [_VP]),
             "qlora_grouped_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
             "qlora_swiglu_packed_fwd": (_I, [_VP, _VP, _I64, _I, _VP]),
             "qlora_swiglu_packed_bwd": (_I, [_VP, _VP, _VP, _I64, _I, _VP]),
@@ -294,6 +296,10 @@ def qlora_linear_fwd_noalloc(X, weight, A, B, M, r, alpha, H, XA_saved, stream):
 
 def qlora_noalloc_scratch_bytes():
     return int(_lib().qlora_noalloc_scratch_bytes())
+
+
+def qlora_selftest_bounded_wait(stream):
+    _check("qlora_selftest_bounded_wait", _lib().qlora_selftest_bounded_wait(stream))
 
 
 def qlora_device_error():

@@ -164,6 +164,10 @@ cudaError_t launch_ce_rows(__nv_bfloat16* z, int rows, int V, const int* labels,
 cudaError_t launch_ce_mean(const float* token_loss, int M, const int* count, float* out,
                            cudaStream_t stream);
 
+// ------------------------------ failure-detection self-test ---------------------------------
+// One thread waits on an mbarrier nothing completes; the bounded wait runs out and sets *err.
+cudaError_t launch_bounded_wait_selftest(int* err, cudaStream_t stream);
+
 // ------------------------------ SwiGLU ------------------------------------------------------
 cudaError_t launch_swiglu_fwd(const __nv_bfloat16* g, const __nv_bfloat16* u, __nv_bfloat16* a,
                               int64_t n, cudaStream_t stream);

@@ -20,6 +20,7 @@ enum WaitSite : int {
   kErrWaitDequant = 3,
   kErrWaitAcc = 4,
   kErrWaitDrain = 5,
+  kErrWaitSelftest = 6,  // the bounded-wait self-test, whose barrier nothing completes
 };
 
 // Wall-clock bound for any spin on another warp's progress (nanoseconds).

@@ -670,6 +670,17 @@ qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count
   return QLORA_OK;
 }
 
+qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream) {
+  int dev;
+  qlora_status st = current_device(&dev);
+  if (st != QLORA_OK) return st;
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  st = cuda_status(launch_bounded_wait_selftest(err, static_cast<cudaStream_t>(stream)));
+  if (st == QLORA_OK) count(1);
+  return st;
+}
+
 uint64_t qlora_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
 
 qlora_status qlora_swiglu_fwd(const void* g, const void* u, void* a, int64_t n,
