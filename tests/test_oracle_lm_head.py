@@ -111,3 +111,27 @@ def test_rows_variant_matches_full():
     tl, dx = lm_head.lm_head_ce_rows(X, Wd, y, [0, 4, 8], out["count"])
     assert np.allclose(tl, out["token_loss"][[0, 4, 8]], rtol=1e-13, atol=1e-13)
     assert np.allclose(dx, out["dX"][[0, 4, 8]], rtol=1e-12, atol=1e-15)
+
+
+def test_chunking_changes_nothing():
+    """Reading R13: processing the tokens in chunks (each chunk's logits, its rows' losses and
+    gradient scaled by the whole batch's count) gives the unchunked losses, loss and dX, for
+    any chunk size including a ragged last chunk."""
+    rng = np.random.default_rng(6)
+    M, K, V = 23, 128, 96
+    X = rng.standard_normal((M, K))
+    Wd = _deq(V, K, rng)
+    y = rng.integers(0, V, M)
+    y[[2, 9]] = -100
+    full = lm_head.lm_head_ce(X, Wd, y)
+    n = lm_head.valid_count(y, V)
+    for c in (1, 5, 8, 23, 64):
+        tl, dx = [], []
+        for m0 in range(0, M, c):
+            t, d = lm_head.ce_from_logits(X[m0:m0 + c] @ Wd.T, y[m0:m0 + c], n)
+            tl.append(t)
+            dx.append(d @ Wd)
+        tl, dx = np.concatenate(tl), np.concatenate(dx)
+        assert np.allclose(tl, full["token_loss"], rtol=1e-13, atol=1e-13)
+        assert abs(tl.sum() / n - full["loss"]) < 1e-12
+        assert np.allclose(dx, full["dX"], rtol=1e-12, atol=1e-15)
