@@ -7,7 +7,8 @@ Checked against:
 * central finite differences of the loss in X;
 * ignored tokens (labels outside [0, V)) and the all-ignored batch;
 * stability and shift invariance of the logits' cross-entropy at large magnitude;
-* zero row sums of the logits' gradient.
+* zero row sums of the logits' gradient;
+* chunking over tokens, which changes nothing.
 """
 
 import math
@@ -114,9 +115,9 @@ def test_rows_variant_matches_full():
 
 
 def test_chunking_changes_nothing():
-    """Reading R13: processing the tokens in chunks (each chunk's logits, its rows' losses and
-    gradient scaled by the whole batch's count) gives the unchunked losses, loss and dX, for
-    any chunk size including a ragged last chunk."""
+    """The fused loss is read as chunks of tokens: each chunk's logits, its rows' losses and its
+    gradient scaled by the whole batch's count.  That gives the unchunked losses, loss and dX
+    for any chunk size, including a ragged last chunk."""
     rng = np.random.default_rng(6)
     M, K, V = 23, 128, 96
     X = rng.standard_normal((M, K))
