@@ -199,8 +199,8 @@ QLORA_API qlora_status qlora_swiglu_packed_bwd(const void* gu, const void* da, v
  *   dX_c = dz deq(W)                    [chunk, K] bf16 (the dequant GEMM, transposed access)
  * and loss = sum(token_loss) / count, count = number of labels in [0, V).  A label outside
  * [0, V) (e.g. -100) ignores its token: loss 0, gradient 0, not counted; with no counted token
- * loss and dX are 0.  W is the NF4 head [V, K] (V % 64 == 0, K % 64 == 0, K >= 128); it gets
- * no gradient.
+ * loss and dX are 0.  W is the NF4 head [V, K] (V % 64 == 0, K % 64 == 0, V >= 128, K >= 128;
+ * QLORA_ERR_SHAPE otherwise); it gets no gradient.
  *   X [M, K] bf16, labels [M] int32 (device, read); loss [1] fp32 (device, written);
  *   token_loss [M] fp32 (device, written; may be NULL); dX [M, K] bf16 (written; NULL: loss
  *   only).  ws: device scratch of qlora_lm_head_ce_workspace_bytes(M, V, K, chunk) bytes,

@@ -319,8 +319,9 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
       count(2);
       return QLORA_OK;
     }
+    // cudaErrorInvalidValue: the scratch is too small for its partials (nothing was launched,
+    // so no error is pending); use the tcgen05 kernel instead.
     if (e != cudaErrorInvalidValue) return QLORA_ERR_CUDA;
-    (void)cudaGetLastError();  // scratch too small for its partials: use the tcgen05 kernel
   }
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -751,7 +752,7 @@ qlora_status qlora_swiglu_packed_bwd(const void* gu, const void* da, void* dgu, 
 }
 
 size_t qlora_lm_head_ce_workspace_bytes(int M, int V, int K, int chunk) {
-  if (M < 1 || V < 64 || V % 64 || K < 128 || K % 64) return 0;
+  if (M < 1 || V < 128 || V % 64 || K < 128 || K % 64) return 0;
   const int c = chunk < 1 || chunk > M ? M : chunk;
   const size_t scratch = std::max(gemm_ws_bytes(c, V, K, 0, false), gemm_ws_bytes(c, V, K, 0, true));
   return align256(static_cast<size_t>(c) * V * 2) + align256(static_cast<size_t>(M) * 4) + 256 +
@@ -765,7 +766,9 @@ qlora_status qlora_lm_head_ce(const void* X, const qlora_nf4_weight* W, const in
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
   const int V = W->N, K = W->K;
-  if (M < 1 || K < 128) return QLORA_ERR_SHAPE;
+  // Both GEMMs run without an extension, so each reduction (K forward, V for dX) must give
+  // every tile at least the two steps the dequant groups take at a time.
+  if (M < 1 || K < 128 || V < 128) return QLORA_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(labels) || !aligned16(loss) ||
       (token_loss && !aligned16(token_loss)) || (dX && !aligned16(dX)))
     return QLORA_ERR_ALIGN;

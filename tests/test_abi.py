@@ -148,6 +148,8 @@ def test_lm_head_and_plain_gemm_validation(lib):
     assert lib.qlora_lm_head_ce(*args(loss=None)) == 1
     assert lib.qlora_lm_head_ce(*args(W=_w(N=1024, K=64))) == 2      # K < 128
     assert lib.qlora_lm_head_ce(*args(W=_w(N=1000, K=256))) == 2     # V % 64
+    assert lib.qlora_lm_head_ce(*args(W=_w(N=64, K=256))) == 2       # V < 128 (dX: one step)
+    assert lib.qlora_lm_head_ce_workspace_bytes(64, 64, 256, 16) == 0
     assert lib.qlora_lm_head_ce(*args(ws_bytes=16)) == 5
     need = lib.qlora_lm_head_ce_workspace_bytes(64, 1024, 256, 16)
     assert need >= 16 * 1024 * 2 + 64 * 4                          # one chunk of logits + losses

@@ -26,8 +26,12 @@ def _cuda():
         pytest.skip("needs a CUDA device")
 
 
-def test_noalloc_forward_matches_workspace_forward_twice():
-    M, K, N, r = 300, 512, 384, 16
+@pytest.mark.parametrize("M,K,N,r", [
+    (16, 512, 384, 16),      # few tokens: the register-direct kernel's slots in the scratch
+    (300, 512, 384, 16),     # stream-K tcgen05 GEMM whose partials fit beside s*XA
+    (16384, 4096, 384, 16),  # stream-K partials too large for what is left: whole tiles
+])
+def test_noalloc_forward_matches_workspace_forward_twice(M, K, N, r):
     inp, L = parity.make(M, K, N, r, seed=21)
     lin = inp["linears"][0]
     X, A, B = inp["X"].cuda(), lin["A"].cuda(), lin["B"].cuda()
