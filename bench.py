@@ -595,21 +595,32 @@ def run_e2e(step, steps):
     return a.elapsed_time(b) / steps, h2d, d2h
 
 
+def kernel_source_digest(files):
+    """sha256 over the kernel's source files with comments and blank space removed, so an edit
+    to a comment, or to code no kernel statement changes, does not void a recorded capture."""
+    import hashlib
+    import re
+    m = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, name)) as g:
+            txt = g.read()
+        txt = re.sub(r"/\*.*?\*/", " ", txt, flags=re.S)
+        txt = re.sub(r"//[^\n]*", " ", txt)
+        m.update(" ".join(txt.split()).encode())
+    return m.hexdigest()
+
+
 def ncu_traffic(workload, stage):
     """DRAM bytes per launch of `stage` from the committed ncu capture (profiles/ncu_traffic.json),
     or None when there is none or the kernel sources changed since it was taken."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(f"{workload}.{stage}")
         if not rec:
             return None
-        m = hashlib.sha256()
-        for name in rec["source_files"]:
-            with open(os.path.join(ROOT, name), "rb") as g:
-                m.update(g.read())
-        return rec["traffic_bytes"] if m.hexdigest() == rec["source_sha256"] else None
+        ok = kernel_source_digest(rec["source_files"]) == rec["source_digest"]
+        return rec["traffic_bytes"] if ok else None
     except (OSError, ValueError, KeyError):
         return None
 
@@ -736,12 +747,35 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, seed=0, rows=32):
+def oracle_sample_rows(w, prep, seconds):
+    """Token rows of a sample that keeps the oracle busy about `seconds` (at least 512 rows, or
+    all M when fewer), calibrated on 8 rows."""
+    per_row = oracle_rows(w, prep, min(8, w.M)) / min(8, w.M)
+    n = int(seconds / max(per_row, 1e-9))
+    return int(max(min(512, w.M), min(w.M, n)))
+
+
+def cpu_baseline(w, seed=0, seconds=10.0):
+    """The fp64 oracle on the host cores, on a calibrated sample of the workload's token rows
+    (about `seconds` of work), plus the single-thread figure of the tiny configuration."""
     prep = oracle_prepare(w, seed)
-    n = min(rows, w.M)
+    n = oracle_sample_rows(w, prep, seconds)
     per_token = oracle_rows(w, prep, n) / n + prep[2] / w.M
-    return {"value": round(1.0 / per_token, 2), "unit": "tokens/s", "cores": blas_threads(),
-            "kind": "oracle", "sample": oracle_desc(w, n)}
+    out = {"value": round(1.0 / per_token, 2), "unit": "tokens/s", "cores": blas_threads(),
+           "kind": "oracle", "sample": oracle_desc(w, n)}
+    try:
+        from threadpoolctl import threadpool_limits
+        tw = synth.workload("tiny")
+        with threadpool_limits(1, user_api="blas"):
+            tprep = oracle_prepare(tw, seed)
+            oracle_rows(tw, tprep, tw.M)  # warm
+            t = min(oracle_rows(tw, tprep, tw.M) for _ in range(5))
+        out["single_thread_tiny"] = {"value": round(tw.M / (t + tprep[2]), 1),
+                                     "unit": "tokens/s", "cores": 1,
+                                     "sample": oracle_desc(tw, tw.M) + ", best of 5"}
+    except Exception as exc:  # threadpoolctl missing: leave the figure out, say why
+        out["single_thread_tiny"] = {"unavailable": str(exc)}
+    return out
 
 
 def run_reference(args):
@@ -774,6 +808,74 @@ def run_reference(args):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------
+# Every other configuration, measured in the same run (one line, key "configs")
+# ----------------------------------------------------------------------------------------------
+CONFIG_WORKLOADS = ("tiny", "mlp_8b", "proj_70b_dq", "sweep_m1", "sweep_m16", "sweep_m128",
+                    "sweep_m1024", "sweep_m16384")
+SPEC_HBM_GBS = 8000.0  # the ~8 TB/s HBM3e figure the targets quote, beside the measured copy
+
+
+def min_bytes(L, M, backward):
+    """Minimum HBM bytes of one pass of a linear: the packed weight once, the bf16 activations,
+    the LoRA factors (and, backward, their fp32 gradients)."""
+    small = 2 * L.r * (L.K + L.N)
+    if not backward:
+        return weight_stream_bytes(L) + 2 * M * L.K + 2 * M * L.N + 2 * M * L.r + small
+    return (weight_stream_bytes(L) + 2 * M * L.N + 4 * M * L.K + 2 * M * L.r + small
+            + 4 * L.r * (L.K + L.N))
+
+
+def is_fwd_stage(name):
+    st = name.split(".", 1)[1]
+    return st in ("lora_down_fwd", "gemm_fwd", "fwd")
+
+
+def measure_config(name, dev, steps, warmup, peaks, flush, clocks_on):
+    """tokens/s, step TFLOP/s, forward and backward times (and, for one linear, their GB/s of
+    minimum traffic), the dominant stage's roofline and the clocks, for one workload timed as
+    the headline is: CUDA-graph replays with L2 flushed before each."""
+    w = synth.workload(name)
+    step = Step(w, dev, seed=0)
+    stream = torch.cuda.current_stream()
+    run_steps(step, warmup, stream, flush, record=False)
+    graph = GraphStep(step)
+    graph.run(3, flush, record=True)
+    sampler = ClockSampler(dev.index or 0)
+    if clocks_on:
+        sampler.start()
+        time.sleep(0.3)
+    per_step, per_stage = graph.run(steps, flush, record=True)
+    clocks = sampler.stop() if clocks_on else None
+    if abi.qlora_device_error() != 0:
+        raise SystemExit(f"device error word set while timing {name}")
+    ms = statistics.mean(per_step)
+    means = {k: statistics.mean(v) for k, v in per_stage.items()}
+    fwd = sum(v for k, v in means.items() if is_fwd_stage(k))
+    bwd = sum(v for k, v in means.items() if not is_fwd_stage(k))
+    tflops = step_flops(w) / (ms * 1e-3) / 1e12
+    rec = {"M": w.M, "ms_per_step": round(ms, 5), "tokens_per_s": round(w.M / (ms * 1e-3), 1),
+           "tflops": round(tflops, 2),
+           "tflops_frac_of_peak": round(tflops / peaks["bf16_tflops"], 4),
+           "fwd_ms": round(fwd, 5), "bwd_ms": round(bwd, 5),
+           "stages_ms": {k: round(v, 5) for k, v in means.items()},
+           "roofline": roofline(step, per_stage, peaks, name),
+           "graph_launches_per_step": graph.launches_per_step, "steps": steps, "clocks": clocks}
+    if len(w.linears) == 1 and not w.mlp:
+        L = w.linears[0]
+        for d, t in (("fwd", fwd), ("bwd", bwd)):
+            b = min_bytes(L, w.M, d == "bwd")
+            gbs = b / (t * 1e-3) / 1e9
+            rec[f"{d}_min_bytes"] = b
+            rec[f"{d}_gbs"] = round(gbs, 1)
+            rec[f"{d}_hbm_frac"] = {"measured": round(gbs / peaks["hbm_gbs"], 4),
+                                    "spec_8000": round(gbs / SPEC_HBM_GBS, 4)}
+    del graph, step
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def workload_config(w, unpacked=False):
@@ -820,6 +922,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations (the \"configs\" key)")
+    ap.add_argument("--config-steps", type=int, default=10,
+                    help="timed steps per configuration of the \"configs\" key")
     ap.add_argument("--eager", action="store_true",
                     help="launch every stage from Python instead of replaying a CUDA graph")
     ap.add_argument("--oracle-threads", type=int, default=0,
@@ -928,6 +1034,16 @@ def main():
             "launch_mode": "cuda_graph" if graph is not None else "eager",
             "clocks": clocks,
         }
+        if world == 1 and not args.no_configs:
+            line["configs"] = {}
+            del step
+            torch.cuda.empty_cache()
+            for name in CONFIG_WORKLOADS:
+                if name == w.name:
+                    continue
+                line["configs"][name] = measure_config(name, dev, args.config_steps,
+                                                       args.warmup, peaks, flush,
+                                                       not args.no_clocks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
