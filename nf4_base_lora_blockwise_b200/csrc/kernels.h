@@ -126,34 +126,44 @@ cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const 
                                 __nv_bfloat16* out, float* partial, size_t partial_floats,
                                 const Codebook& cb, cudaStream_t stream);
 
-// ------------------------------ rank-r skinny products (mma.sync) --------------------------
-// out[m, j] = sum_c in[m, c] * Wl(j, c); Wl(j, c) = w[j * C + c] (w_is_rc = true, i.e. A [r, C])
-// or w[c * r + j] (w_is_rc = false, i.e. B [C, r]).  Writes bf16 RN(v) to `saved` (if not
-// null) and bf16 RN(scale * v) to `scaled`.  `partial` is fp32 scratch [split, M, r].
-// With w_is_rc = false and groups.n > 1, r = n r_g and w is B_cat [C, r_g]: Wl is the
-// block-diagonal matrix with Wl(g r_g + j, c) = w[c * r_g + j] for the rows c of adapter g and
-// zero elsewhere; the zero blocks are neither loaded nor multiplied.
-struct DownPlan {
-  int split;
-  size_t partial_floats;
+// ------------------------------ rank-r products (TMA ring, mma.sync, cluster reduction) ------
+// down: out[m, j] = sum_c in[m, c] Wl(j, c), Wl = A [R, C] (w_rc) or B [C, rg] (block-diagonal
+//       over n adapters along C when groups.n > 1: R = n rg); writes bf16(out) to `saved`
+//       (nullable) and bf16(scale * out) to `scaled`, both [M, R].
+// grad: G[c, j] = scale * sum_m big[m, c] small[m, g(c) R + j], small [M, ld_small], g(c) the
+//       adapter of column c; written as out[c R + j] (out_cr) or out[j C + c].
+// The reduction is split over the CTAs of a cluster and summed in rank order through
+// distributed shared memory: one launch, no scratch, deterministic.
+struct SmallTile {   // a [64 rows, w columns] bf16 tile as TMA writes it
+  int blocks;        // 1, or 2 for w = 128 (two 64-column blocks)
+  int box_w;         // columns per TMA box
+  uint32_t pitch;    // bytes per row of a block
+  uint32_t mask;     // swizzle mask (pitch / 16 - 1 when swizzled, else 0)
+  int swizzle;       // TMA swizzle span in bytes (0 = none, 32, 64, 128)
+  uint32_t bytes;    // bytes per stage
 };
-DownPlan lora_down_plan(int M, int C, int r);
-cudaError_t launch_lora_down(const __nv_bfloat16* in, int M, int C, const __nv_bfloat16* w,
-                             bool w_is_rc, int r, const RowGroups& groups, float scale,
-                             __nv_bfloat16* saved, __nv_bfloat16* scaled, float* partial,
-                             const DownPlan& plan, cudaStream_t stream);
-
-// G[c, j] = scale * sum_m big[m, c] * small[m, g(c) r + j]; written as out[c * r + j] (out_cr)
-// or out[j * C + c].  small is [M, groups.n r]; g(c) is the adapter of column c (0 for
-// groups.n = 1).  `partial` is fp32 scratch [split, C, r].
-struct GradPlan {
-  int split;
-  size_t partial_floats;
+SmallTile small_tile(int w);
+struct RankPlan {
+  int split;   // CTAs per cluster
+  int grid;
+  int stages;
+  size_t smem;
+  SmallTile small;
 };
-GradPlan lora_grad_plan(int M, int C, int r);
-cudaError_t launch_lora_grad(const __nv_bfloat16* big, int M, int C, const __nv_bfloat16* small,
-                             int r, const RowGroups& groups, float scale, float* out, bool out_cr,
-                             float* partial, const GradPlan& plan, cudaStream_t stream);
+struct RankMaps {
+  CUtensorMap big;    // in / big [M, C] bf16: box {64, 128} (down) or {64, 64} (grad), SW128
+  CUtensorMap small;  // down: A [R, C] box {64, R} SW128, or B [C, rg] per small_tile(rg);
+                      // grad: small [M, ld_small] per small_tile(R)
+};
+RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count);
+RankPlan rank_grad_plan(int M, int C, int R, int sm_count);
+cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int C, int R, int rg,
+                             bool w_rc, const RowGroups& groups, float scale,
+                             __nv_bfloat16* saved, __nv_bfloat16* scaled, int* err,
+                             cudaStream_t stream);
+cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int C, int R,
+                             int ld_small, const RowGroups& groups, float scale, float* out,
+                             bool out_cr, int* err, cudaStream_t stream);
 
 // ------------------------------ LM-head cross-entropy ---------------------------------------
 // count = number of labels in [0, V); z [rows, V] bf16 (V % 8 == 0) -> loss [rows] and, with

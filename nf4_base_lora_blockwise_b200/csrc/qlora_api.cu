@@ -197,9 +197,9 @@ size_t gemm_ws_bytes(int M, int N, int K, int r, bool trans) {
 // Workspace layout (each region 256-byte aligned):
 //   [0]  small0   bf16 [M, r]   s*XA (forward) / dYB (backward)
 //   [1]  small1   bf16 [M, r]   s*dYB (backward)
-//   [2]  scratch  fp32 partial sums, written and read within one stage: the split partials of
-//                 the rank-r down-projection, the stream-K partials of the dequant GEMM, then
-//                 the split partials of dB and dA (stages run one after another on the stream)
+//   [2]  scratch  fp32 partial sums of the dequant GEMM (stream-K slots, or the few-token
+//                 kernel's segment slots), written and read within one launch pair
+// The rank-r products reduce inside their clusters and need no scratch.
 // ---------------------------------------------------------------------------------------------
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -210,15 +210,11 @@ struct WsLayout {
 WsLayout ws_layout(int M, int N, int K, int r) {
   WsLayout L;
   const size_t small = align256(static_cast<size_t>(M) * r * 2);
-  const size_t down = 4 * std::max(lora_down_plan(M, K, r).partial_floats,
-                                   lora_down_plan(M, N, r).partial_floats);
-  const size_t grad = 4 * std::max(lora_grad_plan(M, N, r).partial_floats,
-                                   lora_grad_plan(M, K, r).partial_floats);
   const size_t gemm = std::max(gemm_ws_bytes(M, N, K, r, false), gemm_ws_bytes(M, N, K, r, true));
   L.small0 = 0;
   L.small1 = small;
   L.scratch = 2 * small;
-  L.scratch_bytes = align256(std::max(std::max(down, grad), gemm));
+  L.scratch_bytes = align256(gemm);
   L.total = L.scratch + L.scratch_bytes;
   return L;
 }
@@ -289,17 +285,40 @@ void count(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_o
 // ---------------------------------------------------------------------------------------------
 // Stage bodies (validated by their callers).
 // ---------------------------------------------------------------------------------------------
+// Swizzle enum of a TMA span in bytes (0 = none).
+CUtensorMapSwizzle swizzle_of(int span) {
+  switch (span) {
+    case 32: return CU_TENSOR_MAP_SWIZZLE_32B;
+    case 64: return CU_TENSOR_MAP_SWIZZLE_64B;
+    case 128: return CU_TENSOR_MAP_SWIZZLE_128B;
+    default: return CU_TENSOR_MAP_SWIZZLE_NONE;
+  }
+}
+
 // groups: the adapters packed along the rows of B (w_rc = false); r is then n r_g.
 qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc, int r,
                           const RowGroups& groups, float scale, void* saved, void* scaled,
-                          float* partial, cudaStream_t s) {
-  const DownPlan dp = lora_down_plan(M, C, r);
-  cudaError_t e = launch_lora_down(static_cast<const __nv_bfloat16*>(in), M, C,
-                                   static_cast<const __nv_bfloat16*>(w), w_rc, r, groups, scale,
-                                   static_cast<__nv_bfloat16*>(saved),
-                                   static_cast<__nv_bfloat16*>(scaled), partial, dp, s);
+                          int* err, cudaStream_t s) {
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int rg = w_rc ? r : r / groups.n;
+  const RankPlan p = rank_down_plan(M, C, r, rg, w_rc, sms);
+  RankMaps maps;
+  qlora_status st = encode_2d(&maps.big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, in, C, M, C * 2ull,
+                              64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLORA_OK) return st;
+  if (w_rc)  // A [r, C]: box {64 columns, r rows}
+    st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, C, r, C * 2ull, 64, r,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  else  // B [C, rg]: box {box_w, 64 rows}
+    st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, rg, C, rg * 2ull,
+                   p.small.box_w, 64, swizzle_of(p.small.swizzle));
+  if (st != QLORA_OK) return st;
+  const cudaError_t e = launch_rank_down(maps, p, M, C, r, rg, w_rc, groups, scale,
+                                         static_cast<__nv_bfloat16*>(saved),
+                                         static_cast<__nv_bfloat16*>(scaled), err, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  count(dp.split > 1 ? 2 : 1);
+  count(1);
   return QLORA_OK;
 }
 
@@ -339,19 +358,25 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
 
 // groups: the adapters packed along the columns of `big`; small is then [M, n r].
 qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int r,
-                          const RowGroups& groups, float scale, float* out, bool out_cr,
-                          float* partial, cudaStream_t s) {
-  const GradPlan gp = lora_grad_plan(M, C, r);
-  cudaError_t e = launch_lora_grad(static_cast<const __nv_bfloat16*>(big), M, C,
-                                   static_cast<const __nv_bfloat16*>(small), r, groups, scale, out,
-                                   out_cr, partial, gp, s);
+                          const RowGroups& groups, float scale, float* out, bool out_cr, int* err,
+                          cudaStream_t s) {
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  const RankPlan p = rank_grad_plan(M, C, r, sms);
+  const int ld_small = groups.n * r;
+  RankMaps maps;
+  qlora_status st = encode_2d(&maps.big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, big, C, M, C * 2ull,
+                              64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLORA_OK) return st;
+  st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, small, ld_small, M,
+                 ld_small * 2ull, p.small.box_w, 64, swizzle_of(p.small.swizzle));
+  if (st != QLORA_OK) return st;
+  const cudaError_t e =
+      launch_rank_grad(maps, p, M, C, r, ld_small, groups, scale, out, out_cr, err, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  count(gp.split > 1 ? 2 : 1);
+  count(1);
   return QLORA_OK;
 }
-
-size_t down_ws_bytes(int M, int C, int r) { return 4 * lora_down_plan(M, C, r).partial_floats; }
-size_t grad_ws_bytes(int M, int C, int r) { return 4 * lora_grad_plan(M, C, r).partial_floats; }
 
 // ---------------------------------------------------------------------------------------------
 // The layer over n adapters packed along W0's rows (n = 1: a single adapter).  W is
@@ -382,8 +407,7 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
 
   // XA = X A^T [M, n r] (saved in bf16 unless XA_saved is NULL) and s * XA: every adapter's
   // down-projection in one pass over X.
-  st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa,
-                    reinterpret_cast<float*>(w8 + L.scratch), s);
+  st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa, err, s);
   if (st != QLORA_OK) return st;
   // h = X deq(W0)^T + (s XA_g) B_g^T for the rows of each adapter g, in one launch.
   return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s);
@@ -417,13 +441,13 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
   // Without a saved XA, recompute it from X (the forward's own kernel on the same inputs, so
   // bit for bit the value it would have saved) and take dB first, while small0 holds it.
   if (!XA_saved) {
-    st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, dyb, sdyb, scratch, s);
+    st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, dyb, sdyb, err, s);
     if (st != QLORA_OK) return st;
-    st = do_lora_grad(dY, M, W->N, dyb, r, g, scale, dB, true, scratch, s);
+    st = do_lora_grad(dY, M, W->N, dyb, r, g, scale, dB, true, err, s);
     if (st != QLORA_OK) return st;
   }
   // dYB = dY B_bd [M, n r] (bf16, for dA) and s * dYB, B_bd the block-diagonal of the B_g.
-  st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, scratch, s);
+  st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, err, s);
   if (st != QLORA_OK) return st;
   // dX = dY deq(W0) + (s dYB) A: one extension over all n r columns sums the adapters' terms.
   if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
@@ -431,10 +455,10 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
     return st;
   // dB_g = s dY_g^T XA_g  [N, r];  dA = s dYB^T X  [n r, K].
   if (XA_saved) {
-    st = do_lora_grad(dY, M, W->N, XA_saved, r, g, scale, dB, true, scratch, s);
+    st = do_lora_grad(dY, M, W->N, XA_saved, r, g, scale, dB, true, err, s);
     if (st != QLORA_OK) return st;
   }
-  return do_lora_grad(X, M, W->K, dyb, R, single_group(W->K), scale, dA, false, scratch, s);
+  return do_lora_grad(X, M, W->K, dyb, R, single_group(W->K), scale, dA, false, err, s);
 }
 
 }  // namespace
@@ -595,14 +619,15 @@ qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_
   }
   if (!aligned16(in) || !aligned16(w) || !aligned16(scaled) || (saved && !aligned16(saved)))
     return QLORA_ERR_ALIGN;
-  const size_t need = down_ws_bytes(M, C, r);
-  if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
-  if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
+  (void)ws;  // the cluster reduction needs no scratch
+  (void)ws_bytes;
   int dev;
   qlora_status st = current_device(&dev);
   if (st != QLORA_OK) return st;
-  return do_lora_down(in, M, C, w, w_is_r_by_c != 0, r, g, scale, saved, scaled,
-                      static_cast<float*>(ws), static_cast<cudaStream_t>(stream));
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  return do_lora_down(in, M, C, w, w_is_r_by_c != 0, r, g, scale, saved, scaled, err,
+                      static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,
@@ -647,14 +672,15 @@ qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, i
     if (gs != QLORA_OK) return gs;
   }
   if (!aligned16(big) || !aligned16(small) || !aligned16(out)) return QLORA_ERR_ALIGN;
-  const size_t need = grad_ws_bytes(M, C, r);
-  if (need && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
-  if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
+  (void)ws;  // the cluster reduction needs no scratch
+  (void)ws_bytes;
   int dev;
   qlora_status st = current_device(&dev);
   if (st != QLORA_OK) return st;
-  return do_lora_grad(big, M, C, small, r, g, scale, out, out_r_by_c == 0,
-                      static_cast<float*>(ws), static_cast<cudaStream_t>(stream));
+  int* err;
+  if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
+  return do_lora_grad(big, M, C, small, r, g, scale, out, out_r_by_c == 0, err,
+                      static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count, int* bt,
@@ -866,11 +892,10 @@ qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, 
   if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) ||
       (XA_saved && !aligned16(XA_saved)))
     return QLORA_ERR_ALIGN;
-  // The forward needs s*XA [M, r] bf16 plus the down-projection's split partials; the GEMM's
-  // stream-K partials use what is left of the scratch (whole tiles if they do not fit).
+  // The forward needs s*XA [M, r] bf16; the GEMM's partial sums use what is left of the
+  // scratch (whole tiles if they do not fit).
   const size_t sxa_bytes = align256(static_cast<size_t>(M) * r * 2);
-  const size_t need = sxa_bytes + align256(down_ws_bytes(M, W->K, r));
-  if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (sxa_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
   int dev;
   if ((st = current_device(&dev)) != QLORA_OK) return st;
   int* err;
@@ -882,8 +907,7 @@ qlora_status qlora_linear_fwd_noalloc(const void* X, const qlora_nf4_weight* W, 
   auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8);
   const float scale = alpha / static_cast<float>(r);
   // Both scratch regions are written in full before they are read: nothing needs clearing.
-  st = do_lora_down(X, M, W->K, A, true, r, single_group(W->K), scale, XA_saved, sxa,
-                    reinterpret_cast<float*>(w8 + sxa_bytes), s);
+  st = do_lora_down(X, M, W->K, A, true, r, single_group(W->K), scale, XA_saved, sxa, err, s);
   if (st != QLORA_OK) return st;
   return do_gemm(X, W, false, B, sxa, M, r, single_group(W->N), H, err, w8 + sxa_bytes,
                  kNoAllocScratchBytes - sxa_bytes, s);
