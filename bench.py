@@ -509,38 +509,63 @@ def run_steps(step, n, stream, flush, record):
 
 
 class GraphStep:
-    """The whole step captured once into a CUDA graph, with timing events (recorded by the
-    graph itself) between the stages, so host-side launch cost never shows up as idle time
-    between kernels.  Each replay is preceded by the L2 flush (outside the graph) and
-    followed by a synchronize to read that replay's events."""
+    """The whole step captured into CUDA graphs, so host-side launch cost never shows up as idle
+    time between kernels.  Two captures of the same stages:
+      plain         no timing nodes inside: each timed step is one replay bracketed by events
+                    recorded on the replay stream -- the step as a user's graph runs it;
+      instrumented  an event (recorded by the graph itself) between every two stages, for the
+                    per-stage attribution; its event nodes add a little time of their own, so
+                    its stage times are slight upper bounds.
+    Each replay is preceded by the L2 flush (outside the graph) and followed by a synchronize."""
 
     def __init__(self, step):
-        side = torch.cuda.Stream()
-        calls = step.stages(side.cuda_stream)
+        self.side = torch.cuda.Stream()
+        calls = step.stages(self.side.cuda_stream)
         self.names = [name for name, _ in calls]
         self.evs = [torch.cuda.Event(enable_timing=True, external=True)
                     for _ in range(len(calls) + 1)]
-        self.graph = torch.cuda.CUDAGraph()
+        self.graph_i = torch.cuda.CUDAGraph()
         n0 = abi.qlora_launch_counter()
-        with torch.cuda.graph(self.graph, stream=side, capture_error_mode="relaxed"):
+        with torch.cuda.graph(self.graph_i, stream=self.side, capture_error_mode="relaxed"):
             for (_, fn), e in zip(calls, self.evs):
                 e.record()
                 fn()
             self.evs[-1].record()
         self.launches_per_step = abi.qlora_launch_counter() - n0
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.side, capture_error_mode="relaxed"):
+            for _, fn in calls:
+                fn()
 
     def run(self, n, flush, record):
-        per_step, per_stage = [], {}
+        """n plain replays; per-step device times (ms)."""
+        per_step = []
         for _ in range(n):
             flush.zero_()
             flush.max()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
             self.graph.replay()
+            b.record()
             torch.cuda.synchronize()
             if record:
-                per_step.append(self.evs[0].elapsed_time(self.evs[-1]))
-                for name, a, b in zip(self.names, self.evs[:-1], self.evs[1:]):
-                    per_stage.setdefault(name, []).append(a.elapsed_time(b))
-        return per_step, per_stage
+                per_step.append(a.elapsed_time(b))
+        return per_step
+
+    def run_stages(self, n, flush):
+        """n instrumented replays: ({stage: [ms...]}, [step ms...] between the first and last
+        interior events)."""
+        per_stage, per_step = {}, []
+        for _ in range(n):
+            flush.zero_()
+            flush.max()
+            self.graph_i.replay()
+            torch.cuda.synchronize()
+            per_step.append(self.evs[0].elapsed_time(self.evs[-1]))
+            for name, a, b in zip(self.names, self.evs[:-1], self.evs[1:]):
+                per_stage.setdefault(name, []).append(a.elapsed_time(b))
+        return per_stage, per_step
 
 
 def run_e2e(step, steps):
@@ -847,8 +872,9 @@ def measure_config(name, dev, steps, warmup, peaks, flush, clocks_on):
     if clocks_on:
         sampler.start()
         time.sleep(0.3)
-    per_step, per_stage = graph.run(steps, flush, record=True)
+    per_step = graph.run(steps, flush, record=True)
     clocks = sampler.stop() if clocks_on else None
+    per_stage, _ = graph.run_stages(max(5, steps), flush)
     if abi.qlora_device_error() != 0:
         raise SystemExit(f"device error word set while timing {name}")
     ms = statistics.mean(per_step)
@@ -973,6 +999,7 @@ def main():
         try:
             graph = GraphStep(step)
             graph.run(3, flush, record=True)
+            graph.run_stages(2, flush)
         except Exception as exc:  # a runtime without timing events in graphs: time eagerly
             print(f"CUDA graph timing unavailable ({exc}); timing eager launches",
                   file=sys.stderr)
@@ -988,7 +1015,7 @@ def main():
     torch.cuda.synchronize()
     n0 = abi.qlora_launch_counter()
     if graph is not None:
-        per_step, per_stage = graph.run(args.steps, flush, record=True)
+        per_step = graph.run(args.steps, flush, record=True)
         launches = graph.launches_per_step * args.steps
     else:
         per_step, per_stage = run_steps(step, args.steps, stream, flush, record=True)
@@ -999,6 +1026,10 @@ def main():
     clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
     if abi.qlora_device_error() != 0:
         raise SystemExit("device error word set during the timed region")
+    instrumented_ms = None
+    if graph is not None:  # stage attribution, after (and outside) the timed region
+        per_stage, steps_i = graph.run_stages(max(5, min(args.steps, 20)), flush)
+        instrumented_ms = statistics.mean(steps_i)
 
     total_ms = max_over_ranks(sum(per_step), dist, dev)
     value = job_tokens_per_s(world, w.M, args.steps, total_ms)
@@ -1027,6 +1058,10 @@ def main():
             "tflops": round(tflops, 2),
             "tflops_frac_of_peak": round(tflops / peaks["bf16_tflops"], 4),
             "stages_ms": {k: round(statistics.mean(v), 5) for k, v in per_stage.items()},
+            "stages_note": ("per-stage times from a second capture of the same step with an event "
+                            "between every two stages (replayed after the timed region); the "
+                            "timed step has no interior events"),
+            "instrumented_ms_per_step": (round(instrumented_ms, 5) if instrumented_ms else None),
             "roofline": roofline(step, per_stage, peaks, w.name),
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
