@@ -105,6 +105,17 @@ size_t gemm_smem_bytes(int bt, int nh);
 cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
                               size_t partial_floats_avail, cudaStream_t stream, int* launched);
 
+// The same GEMM on CTA pairs (tcgen05.mma.cta_group::2, M = 256 over two SMs; qlora_gemm2.cu)
+// for the whole-tile regime: pair tiles of 256 weight rows x (nh x bt) tokens, each CTA of a
+// pair holding 128 rows and bt / 2 tokens of every MMA's activation block (TMA boxes of bt / 2
+// rows).  No partial sums.  gemm2_applies: enough pair tiles for every pair, and no adapter
+// boundary inside a 256-row pair tile.
+GemmTile gemm2_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count);
+bool gemm2_applies(int M, int rows_w, int steps_per_tile, int sm_count, const RowGroups& groups);
+size_t gemm2_smem_bytes(int bt, int nh);
+cudaError_t launch_qlora_gemm2(bool trans_w, const GemmMaps& maps, const GemmArgs& args,
+                               cudaStream_t stream, int* launched);
+
 // ------------------------------ few-token forward (mma.sync, register-direct) ---------------
 // h[M, N] = X[M, K] . deq(W0)^T + ext_act[M, g(n), r] . ext_w[N, r]^T for M <= 32 (g(n) the
 // adapter of row n): stream-K over (128-row tile, 64-block) units with fp32 partial slots and

@@ -347,6 +347,21 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;
+#ifndef QLORA_NO_CTA_PAIRS
+  if (gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
+    // Enough whole tiles for every SM pair: M = 256 MMAs over CTA pairs (each CTA loads half of
+    // every activation block, so the tensor maps' boxes are bt / 2 tokens high).
+    const GemmTile t2 = gemm2_pick_tile(M, a.rows_w, a.kt + a.n_ext, sms);
+    a.bt = t2.bt;
+    a.nh = t2.nh;
+    qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, groups.n, a.bt / 2);
+    if (st != QLORA_OK) return st;
+    int launched = 0;
+    const cudaError_t e = launch_qlora_gemm2(trans, maps, a, s, &launched);
+    count(launched);
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  }
+#endif
   qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, groups.n, a.bt);
   if (st != QLORA_OK) return st;
   int launched = 0;
