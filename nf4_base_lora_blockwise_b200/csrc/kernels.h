@@ -11,6 +11,33 @@
 
 namespace qlora {
 
+// Launch `kernel` as a programmatic dependent of the previous kernel on the stream (its CTAs
+// call pdl_wait() before touching global memory), optionally as clusters of `cluster` CTAs.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = static_cast<unsigned>(n);
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 // ------------------------------ adapters packed along the output rows -----------------------
 // A stacked base weight [sum N_g, K] whose rows are split into n adapters (q/k/v, gate/up):
 // adapter g owns rows [end[g-1], end[g]) and columns [g r, (g + 1) r) of the packed rank-r
@@ -155,11 +182,14 @@ struct SmallTile {   // a [64 rows, w columns] bf16 tile as TMA writes it
 };
 SmallTile small_tile(int w);
 struct RankPlan {
-  int split;   // CTAs per cluster
+  int rows;         // down only: 1 = whole token rows per warp (no cross-CTA reduction)
+  int split;        // CTAs per cluster
   int grid;
   int stages;
   size_t smem;
-  SmallTile small;
+  SmallTile small;  // the Wl / small tile of one stage
+  int box_rows_in;  // TMA box height of `in` / `big`
+  int box_rows_w;   // TMA box height of Wl (A: R; B: 64 or 256) / small (64)
 };
 struct RankMaps {
   CUtensorMap big;    // in / big [M, C] bf16: box {64, 128} (down) or {64, 64} (grad), SW128
@@ -175,6 +205,14 @@ cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int
 cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int C, int R,
                              int ld_small, const RowGroups& groups, float scale, float* out,
                              bool out_cr, int* err, cudaStream_t stream);
+// Two gradients of one backward (dB and dA) in one launch, when they share the rank, the
+// cluster size and the small-tile layout (rank_grad_pair_ok); same results as two launches.
+bool rank_grad_pair_ok(const RankPlan& p1, int R1, const RankPlan& p2, int R2);
+cudaError_t launch_rank_grad_pair(const RankMaps& m1, const RankPlan& p1, int M, int C1, int R,
+                                  int ld1, const RowGroups& g1, float* out1, bool cr1,
+                                  const RankMaps& m2, const RankPlan& p2, int C2, int ld2,
+                                  const RowGroups& g2, float* out2, bool cr2, float scale,
+                                  int* err, cudaStream_t stream);
 
 // ------------------------------ LM-head cross-entropy ---------------------------------------
 // count = number of labels in [0, V); z [rows, V] bf16 (V % 8 == 0) -> loss [rows] and, with

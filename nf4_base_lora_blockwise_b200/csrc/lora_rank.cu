@@ -220,6 +220,8 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
 
   float acc[NT][4];
 #pragma unroll
@@ -357,10 +359,20 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
 // over tokens in steps of 64.  A = big^T (transposed 8x8 loads of the [64 tokens x 128 c]
 // tile, two SW128 blocks of 64 columns), B = small [64 tokens x R] (rows tokens).
 // ------------------------------------------------------------------------------------------
+// Two independent problems (dB and dA of one backward) may share a launch: CTAs below `grid1`
+// take the first (maps *1, a1), the rest the second, so neither waits for the other's tail.
 template <int NT>
 __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
-    rank_grad_kernel(const __grid_constant__ CUtensorMap tm_big,
-                     const __grid_constant__ CUtensorMap tm_small, const RankArgs a) {
+    rank_grad_kernel(const __grid_constant__ CUtensorMap tm_big1,
+                     const __grid_constant__ CUtensorMap tm_small1, const __grid_constant__ RankArgs a1,
+                     const __grid_constant__ CUtensorMap tm_big2,
+                     const __grid_constant__ CUtensorMap tm_small2, const __grid_constant__ RankArgs a2,
+                     int grid1) {
+  const bool second = static_cast<int>(blockIdx.x) >= grid1;
+  const RankArgs& a = second ? a2 : a1;
+  const CUtensorMap& tm_big = second ? tm_big2 : tm_big1;
+  const CUtensorMap& tm_small = second ? tm_small2 : tm_small1;
+  const int bid = second ? static_cast<int>(blockIdx.x) - grid1 : static_cast<int>(blockIdx.x);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -368,7 +380,7 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
   uint64_t* empty = full + a.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int tile = static_cast<int>(blockIdx.x) / a.split;
+  const int tile = bid / a.split;
   const int c0 = tile * kTileRows;
   // This tile's columns belong to one adapter, whose R columns of `small` it reads.
   const int j0 = row_group(a.groups, c0) * a.R;
@@ -383,6 +395,8 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
 
   float acc[NT][4];
 #pragma unroll
@@ -498,26 +512,150 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
   cluster_sync_all();
 }
 
-// Launch with the cluster dimension (S CTAs along x).
+// ------------------------------------------------------------------------------------------
+// down, many tokens (rank_down_rows_kernel): each warp owns 16 token rows over the whole
+// reduction, so there is nothing to reduce across warps or CTAs.  A CTA (2 consumer warps, 32
+// rows) streams its rows in stages of 256 columns -- 512 contiguous bytes of every row, four
+// 64-column SW128 boxes -- together with the matching 256 columns of Wl (A [R, C]: four boxes
+// of R rows; B [C, rg]: one box of 256 rows).  For R <= 32, where Wl's slice is no larger than
+// the activation's.
+// ------------------------------------------------------------------------------------------
+constexpr int kRowWarps = 2;
+constexpr int kRowThreads = 32 * (kRowWarps + 1);
+constexpr int kRowRows = 16 * kRowWarps;
+constexpr uint32_t kRowXBytes = kRowRows * 512u;  // 32 rows x 256 bf16
+
+template <int NT, bool kWrc>
+__global__ void __launch_bounds__(kRowThreads, 2)
+    rank_down_rows_kernel(const __grid_constant__ CUtensorMap tm_in,
+                          const __grid_constant__ CUtensorMap tm_w, const RankArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + a.ring_bytes);
+  uint64_t* empty = full + a.stages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = static_cast<int>(blockIdx.x) * kRowRows;
+  const int n = a.steps;  // stages of 256 columns
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, kRowWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
+
+  if (warp == kRowWarps) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_in);
+      tma_prefetch_desc(&tm_w);
+      rank_produce(a, ring, full, empty, n, [&](int i, uint8_t* dst, uint64_t* bar) {
+        const int c0 = i * 256;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          tma_load_2d(dst + b * (kRowXBytes / 4), &tm_in, bar, c0 + 64 * b, row0);
+        uint8_t* w = dst + kRowXBytes;
+        if (kWrc) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            tma_load_2d(w + b * (a.small_bytes / 4), &tm_w, bar, c0 + 64 * b, 0);  // A [R, 64]
+        } else {
+          tma_load_2d(w, &tm_w, bar, 0, c0);  // B [256 c, rg]
+        }
+      });
+    }
+    return;
+  }
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  bool failed = false;
+  const int ar = 16 * warp + (lane & 15);
+  for (int i = 0; i < n; ++i) {
+    const int st = i % a.stages;
+    if (!failed)
+      failed = !mbar_wait_warp(full + st, static_cast<uint32_t>(i / a.stages) & 1u,
+                               kErrWaitFull, a.err, i);
+    if (!failed) {
+      const uint32_t xb = smem_u32(ring + st * a.stage_bytes);
+      const uint32_t wb = xb + kRowXBytes;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t xbb = xb + b * (kRowXBytes / 4);
+        const int g = kWrc ? 0 : row_group(a.groups, i * 256 + 64 * b);
+        const int t_lo = kWrc ? 0 : g * (a.rg / 8);
+        const int t_hi = kWrc ? NT : t_lo + a.rg / 8;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t af[4];
+          ldsm_x4(af, xbb + sw128_off(ar, 2 * kk + (lane >> 4)));
+          if (kWrc) {
+            const uint32_t wbb = wb + b * (a.small_bytes / 4);
+#pragma unroll
+            for (int t = 0; t + 1 < NT; t += 2) {
+              const int j = t * 8 + (lane & 7) + ((lane >> 4) << 3);
+              uint32_t bb[4];
+              ldsm_x4(bb, wbb + sw128_off(j, 2 * kk + ((lane >> 3) & 1)));
+              mma16816(acc[t], af, bb[0], bb[1]);
+              mma16816(acc[t + 1], af, bb[2], bb[3]);
+            }
+            if (NT & 1) {
+              constexpr int t = NT - 1;
+              const int l = lane & 15;
+              uint32_t bb[2];
+              ldsm_x2(bb, wbb + sw128_off(t * 8 + (l & 7), 2 * kk + (l >> 3)));
+              mma16816(acc[t], af, bb[0], bb[1]);
+            }
+          } else {
+            const int l = lane & 15;
+            const int k = 64 * b + 16 * kk + (l & 7) + ((l >> 3) << 3);  // row c of the B tile
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              if (t >= t_lo && t < t_hi) {
+                uint32_t bb[2];
+                ldsm_x2_t(bb, wb + small_off(a, k, static_cast<uint32_t>(t - t_lo)));
+                mma16816(acc[t], af, bb[0], bb[1]);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + st);
+  }
+  const int r_lo = row0 + 16 * warp + (lane >> 2);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int col = t * 8 + (lane & 3) * 2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = r_lo + 8 * h;
+      if (m >= a.M) continue;
+      const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
+      const long long o = static_cast<long long>(m) * a.R + col;
+      if (a.saved)
+        *reinterpret_cast<__nv_bfloat162*>(a.saved + o) = __floats2bfloat162_rn(v0, v1);
+      *reinterpret_cast<__nv_bfloat162*>(a.scaled + o) =
+          __floats2bfloat162_rn(a.scale * v0, a.scale * v1);
+    }
+  }
+}
+
+// Launch with the cluster dimension (S CTAs along x), as a programmatic dependent.
 template <typename K>
 cudaError_t launch_clustered(K kernel, int grid, int split, size_t smem, cudaStream_t stream,
-                             const CUtensorMap& m0, const CUtensorMap& m1, const RankArgs& a) {
+                             const CUtensorMap& m0, const CUtensorMap& m1, const RankArgs& a,
+                             int threads = kRankThreads) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kRankThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(split);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, m0, m1, a);
+  return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
+                    split, m0, m1, a);
 }
 
 // CTAs per cluster: the largest power of two (<= 8, <= the steps) that keeps the grid within
@@ -562,11 +700,31 @@ namespace {
 
 RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count) {
   RankPlan p;
+  const int row_ctas = (M + kRowRows - 1) / kRowRows;
+  if (R <= 32 && 3 * row_ctas >= 2 * sm_count) {
+    // Many tokens and a narrow rank: whole rows per warp, no reduction across CTAs.
+    p.rows = 1;
+    p.split = 1;
+    p.grid = row_ctas;
+    p.box_rows_in = kRowRows;
+    p.small = w_rc ? SmallTile{1, 64, 128u, 7u, 128, static_cast<uint32_t>(R) * 512u}
+                   : small_tile(rg);
+    if (!w_rc) p.small.bytes = 256u * p.small.pitch;  // one box of 256 rows of B
+    p.box_rows_w = w_rc ? R : 256;
+    const uint32_t stage = kRowXBytes + ((p.small.bytes + 1023u) & ~1023u);
+    p.stages = static_cast<int>((110u * 1024u - 2048u) / stage);
+    if (p.stages > 8) p.stages = 8;
+    p.smem = 1024 + static_cast<size_t>(p.stages) * stage + 2 * 8 * p.stages;
+    return p;
+  }
+  p.rows = 0;
   const int tiles = (M + kTileRows - 1) / kTileRows;
   p.split = pick_split(tiles, C / 64, sm_count);
   p.grid = tiles * p.split;
+  p.box_rows_in = kTileRows;
   p.small = w_rc ? SmallTile{1, 64, 128u, 7u, 128, static_cast<uint32_t>(R) * 128u}
                  : small_tile(rg);
+  p.box_rows_w = w_rc ? R : 64;
   const RankLayout L = rank_layout(p.small.bytes, R, R <= 64 ? 110 * 1024 : 200 * 1024);
   p.stages = L.stages;
   p.smem = L.smem;
@@ -575,6 +733,9 @@ RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count) {
 
 RankPlan rank_grad_plan(int M, int C, int R, int sm_count) {
   RankPlan p;
+  p.rows = 0;
+  p.box_rows_in = 64;
+  p.box_rows_w = 64;
   const int tiles = (C + kTileRows - 1) / kTileRows;
   p.split = pick_split(tiles, (M + 63) / 64, sm_count);
   p.grid = tiles * p.split;
@@ -592,6 +753,13 @@ RankPlan rank_grad_plan(int M, int C, int R, int sm_count) {
                 : launch_clustered(rank_down_kernel<NTV, false>, p.grid, p.split, p.smem,      \
                                    stream, maps.big, maps.small, a);
 
+#define QLORA_RANK_ROWS_CASE(NTV)                                                              \
+  case NTV:                                                                                   \
+    return w_rc ? launch_clustered(rank_down_rows_kernel<NTV, true>, p.grid, 1, p.smem, stream,  \
+                                   maps.big, maps.small, a, kRowThreads)                      \
+                : launch_clustered(rank_down_rows_kernel<NTV, false>, p.grid, 1, p.smem,       \
+                                   stream, maps.big, maps.small, a, kRowThreads);
+
 cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int C, int R, int rg,
                              bool w_rc, const RowGroups& groups, float scale,
                              __nv_bfloat16* saved, __nv_bfloat16* scaled, int* err,
@@ -603,6 +771,30 @@ cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int
   a.rg = rg;
   a.steps = C / 64;
   a.split = p.split;
+  if (p.rows) {
+    a.steps = (C + 255) / 256;
+    a.stages = p.stages;
+    a.small_bytes = (p.small.bytes + 1023u) & ~1023u;
+    a.stage_bytes = kRowXBytes + a.small_bytes;
+    a.ring_bytes = static_cast<uint32_t>(p.stages) * a.stage_bytes;
+    a.small_pitch = p.small.pitch;
+    a.small_mask = p.small.mask;
+    a.small_blocks = p.small.blocks;
+    a.scale = scale;
+    a.groups = groups;
+    a.saved = saved;
+    a.scaled = scaled;
+    a.err = err;
+    if (a.small_bytes != p.small.bytes || p.small.blocks != 1) return cudaErrorInvalidValue;
+    switch (R / 8) {
+      QLORA_RANK_ROWS_CASE(1)
+      QLORA_RANK_ROWS_CASE(2)
+      QLORA_RANK_ROWS_CASE(3)
+      QLORA_RANK_ROWS_CASE(4)
+      default:
+        return cudaErrorInvalidValue;
+    }
+  }
   const RankLayout L = rank_layout(p.small.bytes, R, R <= 64 ? 110 * 1024 : 200 * 1024);
   a.stages = L.stages;
   a.stage_bytes = L.stage_bytes;
@@ -640,15 +832,12 @@ cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int
   }
 }
 #undef QLORA_RANK_DOWN_CASE
+#undef QLORA_RANK_ROWS_CASE
 
-#define QLORA_RANK_GRAD_CASE(NTV)                                                                \
-  case NTV:                                                                                     \
-    return launch_clustered(rank_grad_kernel<NTV>, p.grid, p.split, p.smem, stream, maps.big,   \
-                            maps.small, a);
+namespace {
 
-cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int C, int R,
-                             int ld_small, const RowGroups& groups, float scale, float* out,
-                             bool out_cr, int* err, cudaStream_t stream) {
+RankArgs grad_args(const RankPlan& p, int M, int C, int R, int ld_small, const RowGroups& groups,
+                   float scale, float* out, bool out_cr, int* err, bool* ok) {
   RankArgs a = {};
   a.M = M;
   a.C = C;
@@ -665,14 +854,36 @@ cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int
   a.small_mask = p.small.mask;
   a.small_blocks = p.small.blocks;
   // The ring's expected bytes per stage are exactly what its copies deliver.
-  if (L.small_bytes != p.small.bytes) return cudaErrorInvalidValue;
+  *ok = L.small_bytes == p.small.bytes;
   a.ld_small = ld_small;
   a.scale = scale;
   a.groups = groups;
   a.out = out;
   a.out_cr = out_cr ? 1 : 0;
   a.err = err;
+  return a;
+}
+
+template <int NT>
+cudaError_t launch_grad_nt(const RankMaps& m1, const RankArgs& a1, int grid1, const RankMaps& m2,
+                           const RankArgs& a2, int grid2, int split, size_t smem,
+                           cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(rank_grad_kernel<NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(rank_grad_kernel<NT>, dim3(static_cast<unsigned>(grid1 + grid2)),
+                    dim3(kRankThreads), smem, stream, split, m1.big, m1.small, a1, m2.big,
+                    m2.small, a2, grid1);
+}
+
+cudaError_t launch_grad_any(int R, const RankMaps& m1, const RankArgs& a1, int grid1,
+                            const RankMaps& m2, const RankArgs& a2, int grid2, int split,
+                            size_t smem, cudaStream_t stream) {
   switch (R / 8) {
+#define QLORA_RANK_GRAD_CASE(NTV) \
+  case NTV:                       \
+    return launch_grad_nt<NTV>(m1, a1, grid1, m2, a2, grid2, split, smem, stream);
     QLORA_RANK_GRAD_CASE(1)
     QLORA_RANK_GRAD_CASE(2)
     QLORA_RANK_GRAD_CASE(3)
@@ -693,6 +904,36 @@ cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int
       return cudaErrorInvalidValue;
   }
 }
+
+}  // namespace
+
+cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int C, int R,
+                             int ld_small, const RowGroups& groups, float scale, float* out,
+                             bool out_cr, int* err, cudaStream_t stream) {
+  bool ok = true;
+  const RankArgs a = grad_args(p, M, C, R, ld_small, groups, scale, out, out_cr, err, &ok);
+  if (!ok) return cudaErrorInvalidValue;
+  return launch_grad_any(R, maps, a, p.grid, maps, a, 0, p.split, p.smem, stream);
+}
+
+bool rank_grad_pair_ok(const RankPlan& p1, int R1, const RankPlan& p2, int R2) {
+  return R1 == R2 && p1.split == p2.split && p1.small.bytes == p2.small.bytes &&
+         p1.small.pitch == p2.small.pitch && p1.small.blocks == p2.small.blocks;
+}
+
+cudaError_t launch_rank_grad_pair(const RankMaps& m1, const RankPlan& p1, int M, int C1, int R,
+                                  int ld1, const RowGroups& g1, float* out1, bool cr1,
+                                  const RankMaps& m2, const RankPlan& p2, int C2, int ld2,
+                                  const RowGroups& g2, float* out2, bool cr2, float scale,
+                                  int* err, cudaStream_t stream) {
+  bool ok1 = true, ok2 = true;
+  const RankArgs a1 = grad_args(p1, M, C1, R, ld1, g1, scale, out1, cr1, err, &ok1);
+  const RankArgs a2 = grad_args(p2, M, C2, R, ld2, g2, scale, out2, cr2, err, &ok2);
+  if (!ok1 || !ok2 || !rank_grad_pair_ok(p1, R, p2, R)) return cudaErrorInvalidValue;
+  return launch_grad_any(R, m1, a1, p1.grid, m2, a2, p2.grid, p1.split,
+                         p1.smem > p2.smem ? p1.smem : p2.smem, stream);
+}
+
 #undef QLORA_RANK_GRAD_CASE
 
 }  // namespace qlora

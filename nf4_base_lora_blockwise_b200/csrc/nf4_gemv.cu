@@ -28,6 +28,7 @@
 
 #include "kernels.h"
 #include "nf4_dequant.cuh"
+#include "ptx.cuh"
 
 namespace qlora {
 
@@ -153,6 +154,8 @@ __global__ void __launch_bounds__(kGvThreads, 2)
 
   Nf4Lut lut;
   nf4_build_lut(cb, 1.0f, lut);  // the unscaled codebook in bf16
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
 
   // Two cursors walk the stage list: loads run S - 1 stages ahead of the compute.
   GvCursor cl, cc;
@@ -290,6 +293,8 @@ __global__ void __launch_bounds__(kGvRows) nf4_gemv_finalize(
     int Mp, const __nv_bfloat16* __restrict__ ext_act, const __nv_bfloat16* __restrict__ ext_w,
     int r, const RowGroups groups, __nv_bfloat16* __restrict__ out) {
   __shared__ int s_first, s_last, s_seg0;
+  pdl_wait();  // the segment partial sums are complete
+  pdl_trigger();
   const int KB = K / 64;
   const int rt = blockIdx.x, tok = blockIdx.y;
   if (threadIdx.x == 0) {
@@ -382,29 +387,35 @@ cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const 
       e = cudaFuncSetAttribute(nf4_gemv_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(p.smem));
       if (e != cudaSuccess) return e;
-      nf4_gemv_fwd_kernel<1><<<p.grid, kGvThreads, p.smem, stream>>>(
-          X, q, absmax, absmax_q8, absmax_scale, dq, M, N, K, p.units, p.max_seg, partial, cb);
+      e = launch_pdl(nf4_gemv_fwd_kernel<1>, dim3(p.grid), dim3(kGvThreads), p.smem, stream, 1,
+                     X, q, absmax, absmax_q8, absmax_scale, dq, M, N, K, p.units, p.max_seg,
+                     partial, cb);
+      if (e != cudaSuccess) return e;
       break;
     case 2:
       e = cudaFuncSetAttribute(nf4_gemv_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(p.smem));
       if (e != cudaSuccess) return e;
-      nf4_gemv_fwd_kernel<2><<<p.grid, kGvThreads, p.smem, stream>>>(
-          X, q, absmax, absmax_q8, absmax_scale, dq, M, N, K, p.units, p.max_seg, partial, cb);
+      e = launch_pdl(nf4_gemv_fwd_kernel<2>, dim3(p.grid), dim3(kGvThreads), p.smem, stream, 1,
+                     X, q, absmax, absmax_q8, absmax_scale, dq, M, N, K, p.units, p.max_seg,
+                     partial, cb);
+      if (e != cudaSuccess) return e;
       break;
     default:
       e = cudaFuncSetAttribute(nf4_gemv_fwd_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(p.smem));
       if (e != cudaSuccess) return e;
-      nf4_gemv_fwd_kernel<4><<<p.grid, kGvThreads, p.smem, stream>>>(
-          X, q, absmax, absmax_q8, absmax_scale, dq, M, N, K, p.units, p.max_seg, partial, cb);
+      e = launch_pdl(nf4_gemv_fwd_kernel<4>, dim3(p.grid), dim3(kGvThreads), p.smem, stream, 1,
+                     X, q, absmax, absmax_q8, absmax_scale, dq, M, N, K, p.units, p.max_seg,
+                     partial, cb);
+      if (e != cudaSuccess) return e;
       break;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  nf4_gemv_finalize<<<dim3((N + kGvRows - 1) / kGvRows, M), kGvRows, 0, stream>>>(
-      partial, M, N, K, p.units, p.grid, p.max_seg, 8 * p.tt, ext_act, ext_w, r, groups, out);
-  return cudaGetLastError();
+  return launch_pdl(nf4_gemv_finalize, dim3((N + kGvRows - 1) / kGvRows, M), dim3(kGvRows), 0,
+                    stream, 1, static_cast<const float*>(partial), M, N, K, p.units, p.grid,
+                    p.max_seg, 8 * p.tt, ext_act, ext_w, r, groups, out);
 }
 
 }  // namespace qlora

@@ -264,43 +264,16 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
   return r;
 }
-// Arrive on an mbarrier anywhere in the cluster (release at cluster scope: this thread's earlier
-// writes, made visible to the async proxy where the tensor core reads them, precede it).
+// Arrive on an mbarrier anywhere in the cluster (default semantics, as for a local arrive).
+// A thread that wrote shared memory the peer's tensor-core instructions read makes those writes
+// visible to the async proxy (fence.proxy.async) before arriving.
 __device__ __forceinline__ void mbar_arrive_cl(uint32_t cl_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx_cl(uint32_t cl_addr, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
-                   cl_addr),
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(cl_addr),
                "r"(bytes)
                : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait (as mbar_wait) with cluster-scope acquire, for barriers the peer CTA arrives on.
-__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, int site, int* err,
-                                             int tag = 0) {
-  const unsigned long long t0 = globaltimer_ns();
-  for (;;) {
-    if (mbar_try_wait_cl(bar, parity)) return true;
-    if (*(volatile int*)err != 0) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      const int code = (site & 0xF) | ((static_cast<int>(blockIdx.x) & 0xFF) << 4) |
-                       ((tag & 0x7FFFF) << 12);
-      atomicCAS(err, 0, code == 0 ? 1 : code);
-      return false;
-    }
-  }
 }
 // TMA tile loads of a CTA pair: the bytes land in this CTA's shared memory and complete on an
 // mbarrier that may sit in either CTA of the pair (`cl_bar`, a shared::cluster address).
@@ -354,6 +327,19 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
       "[%0], %1;" ::"r"(smem_u32(bar)),
       "h"(mask)
       : "memory");
+}
+
+// ---------------------------------- programmatic dependent launch --------------------------
+// Kernels of the hot path are launched as programmatic dependents of the kernel before them on
+// the stream: a dependent's CTAs may start (and run their prologue: barrier set-up, tensor
+// memory allocation, descriptor prefetch) while the previous grid drains.  Every such kernel
+// calls pdl_wait() before its first access to global memory another kernel may write or read,
+// which blocks until the previous grid has completed and its writes are visible -- so the
+// stream order of every read and write is unchanged.  pdl_trigger() lets the next kernel's
+// CTAs be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------- misc --------------------------------------------------

@@ -305,14 +305,14 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
   const RankPlan p = rank_down_plan(M, C, r, rg, w_rc, sms);
   RankMaps maps;
   qlora_status st = encode_2d(&maps.big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, in, C, M, C * 2ull,
-                              64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+                              64, p.box_rows_in, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != QLORA_OK) return st;
   if (w_rc)  // A [r, C]: box {64 columns, r rows}
     st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, C, r, C * 2ull, 64, r,
                    CU_TENSOR_MAP_SWIZZLE_128B);
-  else  // B [C, rg]: box {box_w, 64 rows}
+  else  // B [C, rg]: box {box_w, 64 or 256 rows}
     st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, rg, C, rg * 2ull,
-                   p.small.box_w, 64, swizzle_of(p.small.swizzle));
+                   p.small.box_w, p.box_rows_w, swizzle_of(p.small.swizzle));
   if (st != QLORA_OK) return st;
   const cudaError_t e = launch_rank_down(maps, p, M, C, r, rg, w_rc, groups, scale,
                                          static_cast<__nv_bfloat16*>(saved),
@@ -347,7 +347,7 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;
-#ifndef QLORA_NO_CTA_PAIRS
+#ifdef QLORA_CTA_PAIRS
   if (gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
     // Enough whole tiles for every SM pair: M = 256 MMAs over CTA pairs (each CTA loads half of
     // every activation block, so the tensor maps' boxes are bt / 2 tokens high).
@@ -371,6 +371,17 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// Tensor maps of one rank-r gradient: big [M, C] in boxes of {64, 64}; small [M, ld] in boxes
+// of the plan's small tile.
+qlora_status grad_maps(RankMaps* maps, const RankPlan& p, const void* big, int M, int C,
+                       const void* small, int ld_small) {
+  qlora_status st = encode_2d(&maps->big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, big, C, M, C * 2ull,
+                              64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLORA_OK) return st;
+  return encode_2d(&maps->small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, small, ld_small, M,
+                   ld_small * 2ull, p.small.box_w, 64, swizzle_of(p.small.swizzle));
+}
+
 // groups: the adapters packed along the columns of `big`; small is then [M, n r].
 qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int r,
                           const RowGroups& groups, float scale, float* out, bool out_cr, int* err,
@@ -380,14 +391,36 @@ qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int 
   const RankPlan p = rank_grad_plan(M, C, r, sms);
   const int ld_small = groups.n * r;
   RankMaps maps;
-  qlora_status st = encode_2d(&maps.big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, big, C, M, C * 2ull,
-                              64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != QLORA_OK) return st;
-  st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, small, ld_small, M,
-                 ld_small * 2ull, p.small.box_w, 64, swizzle_of(p.small.swizzle));
+  qlora_status st = grad_maps(&maps, p, big, M, C, small, ld_small);
   if (st != QLORA_OK) return st;
   const cudaError_t e =
       launch_rank_grad(maps, p, M, C, r, ld_small, groups, scale, out, out_cr, err, s);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  count(1);
+  return QLORA_OK;
+}
+
+// dB = s dY^T XA (per adapter) and dA = s dYB^T X of one backward, in one launch when their
+// plans match (single adapter), else one after the other.
+qlora_status do_weight_grads(const void* dY, const void* X, const void* XA, const void* dYB,
+                             int M, int N, int K, int r, const RowGroups& g, float scale,
+                             float* dA, float* dB, int* err, cudaStream_t s) {
+  const int R = g.n * r;
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  const RankPlan pB = rank_grad_plan(M, N, r, sms);
+  const RankPlan pA = rank_grad_plan(M, K, R, sms);
+  if (!rank_grad_pair_ok(pB, r, pA, R)) {
+    qlora_status st = do_lora_grad(dY, M, N, XA, r, g, scale, dB, true, err, s);
+    if (st != QLORA_OK) return st;
+    return do_lora_grad(X, M, K, dYB, R, single_group(K), scale, dA, false, err, s);
+  }
+  RankMaps mB, mA;
+  qlora_status st = grad_maps(&mB, pB, dY, M, N, XA, R);
+  if (st != QLORA_OK) return st;
+  if ((st = grad_maps(&mA, pA, X, M, K, dYB, R)) != QLORA_OK) return st;
+  const cudaError_t e = launch_rank_grad_pair(mB, pB, M, N, r, R, g, dB, true, mA, pA, K, R,
+                                              single_group(K), dA, false, scale, err, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   count(1);
   return QLORA_OK;
@@ -468,11 +501,9 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
   if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
                           L.scratch_bytes, s)) != QLORA_OK)
     return st;
-  // dB_g = s dY_g^T XA_g  [N, r];  dA = s dYB^T X  [n r, K].
-  if (XA_saved) {
-    st = do_lora_grad(dY, M, W->N, XA_saved, r, g, scale, dB, true, err, s);
-    if (st != QLORA_OK) return st;
-  }
+  // dB_g = s dY_g^T XA_g  [N, r];  dA = s dYB^T X  [n r, K] (one launch when they match).
+  if (XA_saved)
+    return do_weight_grads(dY, X, XA_saved, dyb, M, W->N, W->K, r, g, scale, dA, dB, err, s);
   return do_lora_grad(X, M, W->K, dyb, R, single_group(W->K), scale, dA, false, err, s);
 }
 

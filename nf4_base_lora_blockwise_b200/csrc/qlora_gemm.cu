@@ -264,6 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the previous kernel's outputs (activations, rank-r operand) are complete
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------ X producer -------------------------------------------
@@ -634,6 +636,8 @@ __global__ void __launch_bounds__(256) qlora_gemm_finalize(const float* __restri
                                                            int M, int rows_w, int tile_tokens,
                                                            int total, long long T, int G,
                                                            __nv_bfloat16* __restrict__ out) {
+  pdl_wait();  // the GEMM's partial sums are complete
+  pdl_trigger();
   const int row_tiles = (rows_w + kRowsW - 1) / kRowsW;
   const int t = blockIdx.y;
   const long long gs = static_cast<long long>(t) * total;
@@ -793,14 +797,16 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
     e = cudaFuncSetAttribute(qlora_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    qlora_gemm_kernel<false><<<sc.grid, kThreads, smem, stream>>>(maps.act, maps.q, maps.ext_w,
-                                                                  maps.ext_act, args);
+    e = launch_pdl(qlora_gemm_kernel<false>, dim3(sc.grid), dim3(kThreads), smem, stream, 1,
+                   maps.act, maps.q, maps.ext_w, maps.ext_act, args);
+    if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(qlora_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    qlora_gemm_kernel<true><<<sc.grid, kThreads, smem, stream>>>(maps.act, maps.q, maps.ext_w,
-                                                                 maps.ext_act, args);
+    e = launch_pdl(qlora_gemm_kernel<true>, dim3(sc.grid), dim3(kThreads), smem, stream, 1,
+                   maps.act, maps.q, maps.ext_w, maps.ext_act, args);
+    if (e != cudaSuccess) return e;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -810,9 +816,9 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
   const long long T = static_cast<long long>(sc.n_tiles) * total;
   const int tile_elems = args.bt * args.nh * kRowsW;
   const dim3 fgrid((tile_elems / 4 + 255) / 256, sc.n_tiles);
-  qlora_gemm_finalize<<<fgrid, 256, 0, stream>>>(args.partial, args.M, args.rows_w,
-                                                 args.bt * args.nh, total, T, sc.grid, args.out);
-  e = cudaGetLastError();
+  e = launch_pdl(qlora_gemm_finalize, fgrid, dim3(256), 0, stream, 1,
+                 static_cast<const float*>(args.partial), args.M, args.rows_w,
+                 args.bt * args.nh, total, T, sc.grid, args.out);
   if (e == cudaSuccess) *launched = 2;
   return e;
 }

@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
   cluster_sync_all();  // both CTAs' barriers exist before either arrives on the other's
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the previous kernel's outputs (activations, rank-r operand) are complete
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------ X producer (both CTAs) --------------------------------
@@ -269,12 +271,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
       bool ok = true;
       int it = 0;
       for (int tl = 0; ok && tl < my_tiles; ++tl) {
-        if (!mbar_wait_cl(accempty, (static_cast<uint32_t>(tl) & 1u) ^ 1u, kErrWaitAcc, err, tl))
+        if (!mbar_wait(accempty, (static_cast<uint32_t>(tl) & 1u) ^ 1u, kErrWaitAcc, err, tl))
           break;
         tc_fence_after();
         for (int k = 0; k < total; ++k, ++it) {
           const int ws = w_slot2(it);
-          if (!mbar_wait_cl(full + ws, w_par2(it), kErrWaitDequant, err, it)) {
+          if (!mbar_wait(full + ws, w_par2(it), kErrWaitDequant, err, it)) {
             ok = false;
             break;
           }
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
     for (int tl = 0; tl < my_tiles; ++tl) {
       const int t = pair + tl * n_pairs;
       bool got = true;
-      if (lane == 0) got = mbar_wait_cl(accfull, static_cast<uint32_t>(tl) & 1u, kErrWaitAcc, err, tl);
+      if (lane == 0) got = mbar_wait(accfull, static_cast<uint32_t>(tl) & 1u, kErrWaitAcc, err, tl);
       if (!__shfl_sync(0xFFFFFFFFu, got, 0)) break;
       __syncwarp();
       tc_fence_after();
@@ -521,30 +523,18 @@ cudaError_t launch_qlora_gemm2(bool trans_w, const GemmMaps& maps, const GemmArg
                           ((args.M + tile_tokens - 1) / tile_tokens);
   const int grid = 2 * static_cast<int>(tiles < pairs ? tiles : pairs);
   const size_t smem = gemm2_smem_bytes(args.bt, args.nh);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads2);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   if (!trans_w) {
     e = cudaFuncSetAttribute(qlora_gemm2_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, qlora_gemm2_kernel<false>, maps.act, maps.q, maps.ext_w,
-                           maps.ext_act, args);
+    e = launch_pdl(qlora_gemm2_kernel<false>, dim3(grid), dim3(kThreads2), smem, stream, 2,
+                   maps.act, maps.q, maps.ext_w, maps.ext_act, args);
   } else {
     e = cudaFuncSetAttribute(qlora_gemm2_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, qlora_gemm2_kernel<true>, maps.act, maps.q, maps.ext_w,
-                           maps.ext_act, args);
+    e = launch_pdl(qlora_gemm2_kernel<true>, dim3(grid), dim3(kThreads2), smem, stream, 2,
+                   maps.act, maps.q, maps.ext_w, maps.ext_act, args);
   }
   if (e == cudaSuccess) *launched = 1;
   return e;

@@ -8,6 +8,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace qlora {
 
@@ -56,6 +57,8 @@ __device__ __forceinline__ void swiglu_grad8(const float (&fg)[8], const float (
 __global__ void swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ g,
                                   const __nv_bfloat16* __restrict__ u,
                                   __nv_bfloat16* __restrict__ a, int64_t n) {
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
   const int64_t nv = n / 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nv;
@@ -78,6 +81,8 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ g,
                                   const __nv_bfloat16* __restrict__ da,
                                   __nv_bfloat16* __restrict__ dg, __nv_bfloat16* __restrict__ du,
                                   int64_t n) {
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
   const int64_t nv = n / 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nv;
@@ -106,6 +111,8 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ g,
 // threads the row's 8-element vectors, so no index is divided.
 __global__ void swiglu_packed_fwd_kernel(const __nv_bfloat16* __restrict__ gu,
                                          __nv_bfloat16* __restrict__ a, int64_t M, int I) {
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
   const int per_row = I / 8;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint4* g4 = reinterpret_cast<const uint4*>(gu + m * 2 * I);
@@ -124,6 +131,8 @@ __global__ void swiglu_packed_fwd_kernel(const __nv_bfloat16* __restrict__ gu,
 __global__ void swiglu_packed_bwd_kernel(const __nv_bfloat16* __restrict__ gu,
                                          const __nv_bfloat16* __restrict__ da,
                                          __nv_bfloat16* __restrict__ dgu, int64_t M, int I) {
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
   const int per_row = I / 8;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint4* g4 = reinterpret_cast<const uint4*>(gu + m * 2 * I);
@@ -159,27 +168,26 @@ unsigned grid_for(int64_t n) {
 
 cudaError_t launch_swiglu_fwd(const __nv_bfloat16* g, const __nv_bfloat16* u, __nv_bfloat16* a,
                               int64_t n, cudaStream_t stream) {
-  swiglu_fwd_kernel<<<grid_for(n), 256, 0, stream>>>(g, u, a, n);
-  return cudaGetLastError();
+  return launch_pdl(swiglu_fwd_kernel, dim3(grid_for(n)), dim3(256), 0, stream, 1, g, u, a, n);
 }
 
 cudaError_t launch_swiglu_bwd(const __nv_bfloat16* g, const __nv_bfloat16* u,
                               const __nv_bfloat16* da, __nv_bfloat16* dg, __nv_bfloat16* du,
                               int64_t n, cudaStream_t stream) {
-  swiglu_bwd_kernel<<<grid_for(n), 256, 0, stream>>>(g, u, da, dg, du, n);
-  return cudaGetLastError();
+  return launch_pdl(swiglu_bwd_kernel, dim3(grid_for(n)), dim3(256), 0, stream, 1, g, u, da, dg, du,
+                    n);
 }
 
 cudaError_t launch_swiglu_packed_fwd(const __nv_bfloat16* gu, __nv_bfloat16* a, int64_t M, int I,
                                      cudaStream_t stream) {
-  swiglu_packed_fwd_kernel<<<grid_rows(M), 256, 0, stream>>>(gu, a, M, I);
-  return cudaGetLastError();
+  return launch_pdl(swiglu_packed_fwd_kernel, dim3(grid_rows(M)), dim3(256), 0, stream, 1, gu, a, M,
+                    I);
 }
 
 cudaError_t launch_swiglu_packed_bwd(const __nv_bfloat16* gu, const __nv_bfloat16* da,
                                      __nv_bfloat16* dgu, int64_t M, int I, cudaStream_t stream) {
-  swiglu_packed_bwd_kernel<<<grid_rows(M), 256, 0, stream>>>(gu, da, dgu, M, I);
-  return cudaGetLastError();
+  return launch_pdl(swiglu_packed_bwd_kernel, dim3(grid_rows(M)), dim3(256), 0, stream, 1, gu, da,
+                    dgu, M, I);
 }
 
 }  // namespace qlora

@@ -1,8 +1,10 @@
 """The rank-r products through the C ABI, element by element against the fp64 oracle.
 
-qlora_lora_down (X A^T, dY B with the block-diagonal B of packed adapters) and qlora_lora_grad
-(s dY^T XA, s dYB^T X) split their reduction over the CTAs of a cluster and sum the partials
-in a fixed order in distributed shared memory.  Covered here: every small-tile layout the
+qlora_lora_grad (s dY^T XA, s dYB^T X), and qlora_lora_down (X A^T, dY B with the
+block-diagonal B of packed adapters) when tokens are few or the rank wide, split their
+reduction over the CTAs of a cluster and sum the partials in a fixed order in distributed
+shared memory; qlora_lora_down with many tokens and r <= 32 gives each warp whole token rows
+(shapes with M >= 4096 below), including a reduction that is not a multiple of 256.  Covered here: every small-tile layout the
 kernels use (8, 16, 32, 64 and 128 columns, swizzled; 24, 40, 48, 72, 120, unswizzled rows),
 ragged token counts (M not a multiple of 64 or 128), column counts that leave half a 128-wide
 tile, cluster sizes 1 to 8, repeat calls bit for bit, and no scratch passed at all.
@@ -61,6 +63,7 @@ def _grad(big, small, R, out_cr, groups=None, scale=0.5):
 
 @pytest.mark.parametrize("M,C,R", [
     (1, 256, 16), (77, 192, 8), (300, 512, 24), (130, 1024, 32), (4096, 4096, 16),
+    (4500, 320, 24), (8192, 640, 32), (4096, 256, 8),
     (257, 640, 40), (64, 256, 48), (513, 448, 64), (100, 320, 72), (33, 256, 120),
     (200, 512, 128),
 ])
@@ -78,7 +81,8 @@ def test_down_A_form(M, C, R):
 
 
 @pytest.mark.parametrize("M,C,R", [(300, 512, 16), (65, 1024, 8), (129, 384, 24), (64, 512, 64),
-                                   (31, 256, 128)])
+                                   (31, 256, 128), (4096, 1024, 16), (4100, 448, 32),
+                                   (6000, 256, 8)])
 def test_down_B_form(M, C, R):
     dY = _rand((M, C), 1.0, 7 * M).cuda()
     B = _rand((C, R), 0.05, C).cuda()
@@ -87,10 +91,12 @@ def test_down_B_form(M, C, R):
     assert qlora.rel_err(_f64(saved), ref) <= TOL
 
 
-@pytest.mark.parametrize("Ns,r", [([256, 128, 128], 16), ([128, 384], 24), ([128] * 8, 8)])
-def test_down_block_diagonal(Ns, r):
+@pytest.mark.parametrize("M,Ns,r", [(200, [256, 128, 128], 16), (200, [128, 384], 24),
+                                    (200, [128] * 8, 8), (4096, [256, 128, 128], 16),
+                                    (4096, [128, 384], 8)])
+def test_down_block_diagonal(M, Ns, r):
     """dY B_bd: adapter g's columns of dY feed output columns g r .. g r + r - 1 only."""
-    M, C = 200, sum(Ns)
+    C = sum(Ns)
     dY = _rand((M, C), 1.0, 11).cuda()
     B = _rand((C, r), 0.05, 12).cuda()
     saved, _ = _down(dY, B, False, r * len(Ns), groups=Ns)
