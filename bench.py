@@ -510,12 +510,15 @@ def run_steps(step, n, stream, flush, record):
 
 class GraphStep:
     """The whole step captured into CUDA graphs, so host-side launch cost never shows up as idle
-    time between kernels.  Two captures of the same stages:
-      plain         no timing nodes inside: each timed step is one replay bracketed by events
-                    recorded on the replay stream -- the step as a user's graph runs it;
-      instrumented  an event (recorded by the graph itself) between every two stages, for the
-                    per-stage attribution; its event nodes add a little time of their own, so
-                    its stage times are slight upper bounds.
+    time between kernels.  Two captures:
+      plain         the layer's public calls (linear.forward / backward, i.e. qlora_linear_fwd /
+                    qlora_linear_bwd, and the SwiGLU glue), exactly as a user's step issues them,
+                    with no timing nodes inside: each timed step is one replay bracketed by
+                    events recorded on the replay stream;
+      instrumented  the same work as its stage entry points with an event (recorded by the
+                    graph itself) between every two stages, for the per-stage attribution; its
+                    event nodes add a little time of their own, so stage times are slight upper
+                    bounds.
     Each replay is preceded by the L2 flush (outside the graph) and followed by a synchronize."""
 
     def __init__(self, step):
@@ -531,11 +534,12 @@ class GraphStep:
                 e.record()
                 fn()
             self.evs[-1].record()
-        self.launches_per_step = abi.qlora_launch_counter() - n0
+        self.stage_launches_per_step = abi.qlora_launch_counter() - n0
         self.graph = torch.cuda.CUDAGraph()
+        n0 = abi.qlora_launch_counter()
         with torch.cuda.graph(self.graph, stream=self.side, capture_error_mode="relaxed"):
-            for _, fn in calls:
-                fn()
+            step.e2e()
+        self.launches_per_step = abi.qlora_launch_counter() - n0
 
     def run(self, n, flush, record):
         """n plain replays; per-step device times (ms)."""
@@ -1058,9 +1062,11 @@ def main():
             "tflops": round(tflops, 2),
             "tflops_frac_of_peak": round(tflops / peaks["bf16_tflops"], 4),
             "stages_ms": {k: round(statistics.mean(v), 5) for k, v in per_stage.items()},
-            "stages_note": ("per-stage times from a second capture of the same step with an event "
-                            "between every two stages (replayed after the timed region); the "
-                            "timed step has no interior events"),
+            "stages_note": ("the timed step replays the layer's public calls (qlora_linear_fwd / "
+                            "qlora_linear_bwd and the SwiGLU glue) with no interior events; "
+                            "per-stage times come from a second capture of the same work as its "
+                            "stage entry points with an event between every two stages, replayed "
+                            "after the timed region"),
             "instrumented_ms_per_step": (round(instrumented_ms, 5) if instrumented_ms else None),
             "roofline": roofline(step, per_stage, peaks, w.name),
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

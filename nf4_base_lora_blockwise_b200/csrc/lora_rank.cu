@@ -701,7 +701,8 @@ namespace {
 RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count) {
   RankPlan p;
   const int row_ctas = (M + kRowRows - 1) / kRowRows;
-  if (R <= 32 && 3 * row_ctas >= 2 * sm_count) {
+  // (A [R, C] only: with B the 256-row box of narrow rows measured slower than the cluster kernel.)
+  if (w_rc && R <= 32 && 3 * row_ctas >= 2 * sm_count) {
     // Many tokens and a narrow rank: whole rows per warp, no reduction across CTAs.
     p.rows = 1;
     p.split = 1;
