@@ -276,6 +276,30 @@ QLORA_API qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, in
                                        int* bt, int* nh, int* streamk, int* grid,
                                        size_t* partial_bytes);
 
+/* Host-only: 1 if the dequant GEMM launch for this problem computes the rank-r down-projection
+ * itself (X A^T in the forward, transpose_w = 0; dY B in dX, transpose_w = 1) for n adapters of
+ * rank r packed into rank_cols = n r columns, else 0 (the layer then launches it separately
+ * first).  *bt (nullable) receives the fused launch's tokens per half tile, else 0.  The
+ * tensor cores add the rank product on 128-token windows of a token tile's first tiles, so it
+ * fuses when: whole tiles of two halves of 144..240 tokens model at most 4 % slower than the
+ * GEMM's own choice of tile; rank_cols is a multiple of 8 up to 32 (dX: r = 16 or 32); the rank
+ * operand's tiles fit in shared memory; and every token tile's windows (up to 4) fall on its
+ * tiles in the first wave that reaches it.  No counterpart on the pages: it reports a scheduling
+ * decision of this implementation ("Unsloth vs QLoRA vs Liger-Kernel", section 2: the rank-r
+ * products fused into the layer's kernels). */
+QLORA_API int qlora_gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count,
+                                      int rank_cols, int r, int transpose_w, int* bt);
+
+/* Host-only, process-wide: 1 makes qlora_linear_* / qlora_grouped_* compute the rank-r
+ * down-projection inside the dequant GEMM launch whenever qlora_gemm_rank_fusable says that
+ * launch can (saving one launch and one read of X or dY); 0 (the default) always launches it
+ * separately.  Results agree within the parity tolerance either way (the fp32 sums run in a
+ * different order).  Off by default because on a B200 the fused q_proj step (4096 tokens,
+ * 4096 x 4096, r = 16) measured 0.388 ms against 0.359 ms separate: the other tiles of a token
+ * tile wait at their extension step for the window tiles.  Returns the previous setting.  No
+ * counterpart on the pages (a scheduling choice of this implementation). */
+QLORA_API int qlora_set_rank_fusion(int enable);
+
 /* Number of kernels this library has launched in this process so far (all devices). */
 QLORA_API uint64_t qlora_launch_counter(void);
 

@@ -40,6 +40,8 @@ EXPORTS = (
     "qlora_cross_entropy_rows",
     "qlora_cross_entropy_mean",
     "qlora_gemm_plan",
+    "qlora_gemm_rank_fusable",
+    "qlora_set_rank_fusion",
     "qlora_selftest_bounded_wait",
 )
 
@@ -119,6 +121,8 @@ def _lib():
             "qlora_gemm_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
                                      ctypes.POINTER(_I), ctypes.POINTER(_I),
                                      ctypes.POINTER(_SZ)]),
+            "qlora_gemm_rank_fusable": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
+            "qlora_set_rank_fusion": (_I, [_I]),
             "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
                                        _VP]),
@@ -282,6 +286,21 @@ def qlora_gemm_plan(M, rows_w, steps_per_tile, sm_count):
                                                      ctypes.byref(pb)))
     return {"bt": v[0].value, "nh": v[1].value, "streamk": v[2].value, "grid": v[3].value,
             "partial_bytes": pb.value}
+
+
+def qlora_gemm_rank_fusable(M, rows_w, steps_per_tile, sm_count, rank_cols, r, transpose_w):
+    """Tokens per half tile of the GEMM launch that computes the rank-r down-projection itself,
+    or 0 when that launch does not."""
+    bt = _I()
+    ok = _lib().qlora_gemm_rank_fusable(M, rows_w, steps_per_tile, sm_count, rank_cols, r,
+                                        int(transpose_w), ctypes.byref(bt))
+    return bt.value if ok else 0
+
+
+def qlora_set_rank_fusion(enable):
+    """Fuse the rank-r down-projections into the GEMM launches (process-wide); returns the
+    previous setting."""
+    return bool(_lib().qlora_set_rank_fusion(int(bool(enable))))
 
 
 def qlora_launch_counter():

@@ -94,6 +94,22 @@ struct GemmArgs {
   int streamk;     // set by the launcher
   RowGroups groups;  // forward: the adapter of each row tile selects its slice of ext_act
   Codebook cb;
+  // Rank-r down-projection fused into the launch (whole-tile schedules only; rank_cols <= 32):
+  // the tensor cores compute rank = act . Wr -- Wr = A^T [K, n r] for the forward (X A^T), the
+  // block-diagonal B [N, n r] for dX (dY B) -- in 128-token windows from the activation tiles
+  // already in shared memory, the epilogue warps write rank (bf16, nullable) and
+  // rank_scale * rank (bf16, the extension operand ext_act maps) and count the published windows
+  // per token tile in rank_flags, which every tile's extension step waits on.
+  int fuse;                     // 0: ext_act was written by an earlier launch
+  int rank_cols;                // n r
+  int rank_r;                   // r of one adapter
+  RowGroups rank_groups;        // dX: the adapters' row ranges of B (= column ranges of dY)
+  const __nv_bfloat16* rank_w;  // forward: A [n r, K]; dX: B [N, r]
+  __nv_bfloat16* rank_saved;    // [M, n r] or null
+  __nv_bfloat16* rank_scaled;   // [M, n r]
+  float rank_scale;
+  unsigned* rank_flags;         // [token tiles], zero before the launch
+  unsigned rank_slot;           // bytes of one rank-operand tile (gemm_rank_slot_bytes)
 };
 
 struct GemmMaps {
@@ -101,6 +117,8 @@ struct GemmMaps {
   CUtensorMap q;        // [N, K/2] u8
   CUtensorMap ext_w;    // B_lora [N, r] (fwd) or A_lora [r, K] (dX), bf16
   CUtensorMap ext_act;  // scaled rank-r activation [M, n, r] bf16 (n adapters), box {64, 1, bt}
+  CUtensorMap rank;     // fused down-projection: A [n r, K] box {64, n r} (fwd) or
+                        // B [N, r] box {r, 64} (dX); unused otherwise
 };
 
 // Work schedule of one launch: whole tiles (one CTA per tile, at most one per SM) or, with
@@ -113,7 +131,21 @@ struct GemmSchedule {
   int grid;
   size_t partial_floats;  // workspace the stream-K partials need
 };
-GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count);
+// fused: the tile a launch with the fused down-projection uses (two halves of 144..240 tokens).
+GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count,
+                           bool fused = false);
+// Whether a launch of this shape can fuse a rank-`rank_cols` down-projection (whole tiles, every
+// token tile's 16-token blocks spread over its first wave of tiles at most 2 per tile).
+bool gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int rank_cols,
+                       unsigned rank_slot);
+// Bytes of one rank-operand tile of the fused down-projection (0: that form is not fused):
+// forward A [n r rounded up to 16 rows, 64 k] (128 B rows); dX B [64 n rows, r] for r = 16, 32.
+inline unsigned gemm_rank_slot_bytes(bool trans_w, int rank_cols, int r) {
+  if (trans_w) return (r == 16 || r == 32) ? 128u * static_cast<unsigned>(r) : 0u;
+  return 128u * static_cast<unsigned>((rank_cols + 15) / 16 * 16);
+}
+// Counters the fused down-projection needs in the workspace (zeroed before each launch).
+size_t gemm_rank_flag_bytes(int M);
 // Partial-sum bytes any device (at most kGemmMaxCtas SMs) may need for this shape.
 size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile);
 
@@ -124,7 +156,7 @@ struct GemmTile {
   int bt;
   int nh;
 };
-GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count);
+GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count, bool fused = false);
 cudaError_t gemm_device_sms(int* sms);  // SMs of the current device (cached)
 size_t gemm_smem_bytes(int bt, int nh);
 // Falls back to whole tiles when stream-K is chosen but `partial` is null or smaller than the

@@ -40,49 +40,15 @@ constexpr int kTileRows = 128;
 constexpr uint32_t kBigTileBytes = kTileRows * 64 * 2;  // 128 rows x 64 bf16
 constexpr int kMaxSplit = 8;
 
-// Byte offset of 16-byte chunk `chunk` of row `row` in a TMA tile whose rows are `pitch` bytes.
-// A tile written with a swizzle whose span equals its pitch (32, 64 or 128 bytes) has bits 4..
-// of the offset XORed with bits 7.. (`mask` = pitch / 16 - 1); an unswizzled tile has mask 0.
-// Tiles start on 1024-byte boundaries, so offsets within the tile follow the same pattern.
-__device__ __forceinline__ uint32_t swz_off(uint32_t row, uint32_t chunk, uint32_t pitch,
-                                            uint32_t mask) {
-  const uint32_t o = row * pitch + (chunk << 4);
-  return o ^ (((o >> 7) & mask) << 4);
-}
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
   return swz_off(row, chunk, 128u, 7u);
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
 __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
 }
-__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // ---------------------------------- cluster helpers ---------------------------------------
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;

@@ -21,6 +21,7 @@ enum WaitSite : int {
   kErrWaitAcc = 4,
   kErrWaitDrain = 5,
   kErrWaitSelftest = 6,  // the bounded-wait self-test, whose barrier nothing completes
+  kErrWaitRank = 7,      // a tile's extension step, on the fused down-projection's blocks
 };
 
 // Wall-clock bound for any spin on another warp's progress (nanoseconds).
@@ -161,6 +162,80 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Same, for global memory: generic-proxy writes this thread made (or acquired from other
+// threads) become visible to later async-proxy (TMA) reads, and vice versa.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until the counter at `p` (written by other CTAs) reaches `target`; same error
+// protocol as mbar_wait.
+__device__ __forceinline__ bool wait_count(const unsigned* p, unsigned target, int site, int* err,
+                                           int tag = 0) {
+  if (ld_acquire_u32(p) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(128);
+    if (ld_acquire_u32(p) >= target) return true;
+    if (*(volatile int*)err != 0) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      const int code = (site & 0xF) | ((static_cast<int>(blockIdx.x) & 0xFF) << 4) |
+                       ((tag & 0x7FFFF) << 12);
+      atomicCAS(err, 0, code == 0 ? 1 : code);
+      return false;
+    }
+  }
+}
+
+// ---------------------------------- warp-level mma.sync -----------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a TMA tile whose rows are `pitch` bytes.
+// A tile written with a swizzle whose span equals its pitch (32, 64 or 128 bytes) has bits 4..
+// of the offset XORed with bits 7.. (`mask` = pitch / 16 - 1); an unswizzled tile has mask 0.
+// Tiles start on 1024-byte boundaries, so offsets within the tile follow the same pattern.
+__device__ __forceinline__ uint32_t swz_off(uint32_t row, uint32_t chunk, uint32_t pitch,
+                                            uint32_t mask) {
+  const uint32_t o = row * pitch + (chunk << 4);
+  return o ^ (((o >> 7) & mask) << 4);
+}
+// Transpose of the 8 x 8 b16 matrix a warp holds in the mma fragment layout (lane l: row l / 4,
+// columns 2 (l % 4) and 2 (l % 4) + 1).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t v) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(v));
+  return d;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // ---------------------------------- tcgen05 -----------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -235,6 +310,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Shared-memory matrix descriptor with an explicit layout type (bits 61-63: 0 none, 2 128B,
+// 4 64B, 6 32B swizzle).  K-major: sbo = stride between 8-row groups; MN-major: lbo = stride
+// between swizzle atoms along M/N, sbo = stride between 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint32_t layout) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
 }
 

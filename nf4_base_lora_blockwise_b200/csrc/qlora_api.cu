@@ -197,14 +197,16 @@ size_t gemm_ws_bytes(int M, int N, int K, int r, bool trans) {
 // Workspace layout (each region 256-byte aligned):
 //   [0]  small0   bf16 [M, r]   s*XA (forward) / dYB (backward)
 //   [1]  small1   bf16 [M, r]   s*dYB (backward)
-//   [2]  scratch  fp32 partial sums of the dequant GEMM (stream-K slots, or the few-token
+//   [2]  flags    u32 per token tile: the fused down-projection's published blocks, zeroed by
+//                 the call before the launch that counts them
+//   [3]  scratch  fp32 partial sums of the dequant GEMM (stream-K slots, or the few-token
 //                 kernel's segment slots), written and read within one launch pair
 // The rank-r products reduce inside their clusters and need no scratch.
 // ---------------------------------------------------------------------------------------------
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-  size_t small0, small1, scratch, scratch_bytes, total;
+  size_t small0, small1, flags, flags_bytes, scratch, scratch_bytes, total;
 };
 
 WsLayout ws_layout(int M, int N, int K, int r) {
@@ -213,21 +215,35 @@ WsLayout ws_layout(int M, int N, int K, int r) {
   const size_t gemm = std::max(gemm_ws_bytes(M, N, K, r, false), gemm_ws_bytes(M, N, K, r, true));
   L.small0 = 0;
   L.small1 = small;
-  L.scratch = 2 * small;
+  L.flags = 2 * small;
+  L.flags_bytes = align256(gemm_rank_flag_bytes(M));
+  L.scratch = L.flags + L.flags_bytes;
   L.scratch_bytes = align256(gemm);
   L.total = L.scratch + L.scratch_bytes;
   return L;
 }
 
+// The rank-r down-projection a dequant GEMM launch computes itself (see GemmArgs::fuse).
+struct RankFusion {
+  const void* w;      // forward: A [n r, K]; dX: B [N, r]
+  int cols, r;        // n r, r
+  RowGroups groups;   // dX: the adapters along N
+  void* saved;        // [M, n r] bf16 or null
+  void* scaled;       // [M, n r] bf16: the GEMM's extension operand
+  float scale;
+  unsigned* flags;    // workspace counters, zeroed here before the launch
+  size_t flag_bytes;
+};
+
 GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& groups, bool trans,
-                   void* out, int* err, int sms) {
+                   void* out, int* err, int sms, bool fused = false) {
   GemmArgs a;
   a.M = M;
   a.rows_w = trans ? W->K : W->N;
   a.kt = (trans ? W->N : W->K) / 64;
   a.r_pad16 = (r + 15) / 16 * 16;
   a.n_ext = (a.r_pad16 + 63) / 64;
-  const GemmTile tl = gemm_pick_tile(M, a.rows_w, a.kt + a.n_ext, sms);
+  const GemmTile tl = gemm_pick_tile(M, a.rows_w, a.kt + a.n_ext, sms, fused);
   a.bt = tl.bt;
   a.nh = tl.nh;
   a.kblocks = W->K / 64;
@@ -242,6 +258,16 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& gro
   a.streamk = 0;
   a.groups = groups;
   a.cb = codebook();
+  a.fuse = 0;
+  a.rank_cols = 0;
+  a.rank_r = 0;
+  a.rank_groups = single_group(64);
+  a.rank_w = nullptr;
+  a.rank_saved = nullptr;
+  a.rank_scaled = nullptr;
+  a.rank_scale = 0.f;
+  a.rank_flags = nullptr;
+  a.rank_slot = 0;
   return a;
 }
 
@@ -280,6 +306,10 @@ qlora_status gemm_maps(GemmMaps* m, const qlora_nf4_weight* W, bool trans, const
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
 std::atomic<uint64_t> g_launches{0};
+// Whether the layer fuses its rank-r down-projections into the dequant GEMM launches when the
+// schedule allows (qlora_set_rank_fusion; off by default: on the 4096-token q_proj step it
+// measured slower than the separate launches).
+std::atomic<int> g_rank_fusion{0};
 void count(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 // ---------------------------------------------------------------------------------------------
@@ -326,7 +356,8 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
 // groups (forward only): adapters packed along W0's rows, each with r columns of ext_act.
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
                      const void* ext_act, int M, int r, const RowGroups& groups, void* out,
-                     int* err, void* partial, size_t partial_bytes, cudaStream_t s) {
+                     int* err, void* partial, size_t partial_bytes, cudaStream_t s,
+                     const RankFusion* fuse = nullptr) {
   if (!trans && M <= kGemvMaxTokens && partial) {
     // Few tokens: the register-direct kernel streams the weight without the tcgen05 rings.
     const cudaError_t e = launch_nf4_gemv_fwd(
@@ -344,11 +375,11 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   }
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
-  GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms);
+  GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms, fuse != nullptr);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;
 #ifdef QLORA_CTA_PAIRS
-  if (gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
+  if (!fuse && gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
     // Enough whole tiles for every SM pair: M = 256 MMAs over CTA pairs (each CTA loads half of
     // every activation block, so the tensor maps' boxes are bt / 2 tokens high).
     const GemmTile t2 = gemm2_pick_tile(M, a.rows_w, a.kt + a.n_ext, sms);
@@ -364,6 +395,27 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
 #endif
   qlora_status st = gemm_maps(&maps, W, trans, act, ext_w, ext_act, M, r, groups.n, a.bt);
   if (st != QLORA_OK) return st;
+  maps.rank = maps.act;  // never read unless fused
+  if (fuse) {
+    a.rank_slot = gemm_rank_slot_bytes(trans, fuse->cols, fuse->r);
+    if (!trans)  // A [n r, K]: box {64 columns, n r rounded up to 16 rows (zero fill)}
+      st = encode_2d(&maps.rank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fuse->w, W->K, fuse->cols,
+                     W->K * 2ull, 64, (fuse->cols + 15) / 16 * 16, CU_TENSOR_MAP_SWIZZLE_128B);
+    else  // B [N, r]: box {r columns, 64 rows}
+      st = encode_2d(&maps.rank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fuse->w, fuse->r, W->N,
+                     fuse->r * 2ull, fuse->r, 64, swizzle_of(fuse->r * 2));
+    if (st != QLORA_OK) return st;
+    a.fuse = 1;
+    a.rank_cols = fuse->cols;
+    a.rank_r = fuse->r;
+    a.rank_groups = fuse->groups;
+    a.rank_w = static_cast<const __nv_bfloat16*>(fuse->w);
+    a.rank_saved = static_cast<__nv_bfloat16*>(fuse->saved);
+    a.rank_scaled = static_cast<__nv_bfloat16*>(fuse->scaled);
+    a.rank_scale = fuse->scale;
+    a.rank_flags = fuse->flags;
+    if (cudaMemsetAsync(fuse->flags, 0, fuse->flag_bytes, s) != cudaSuccess) return QLORA_ERR_CUDA;
+  }
   int launched = 0;
   const cudaError_t e = launch_qlora_gemm(trans, maps, a, partial ? partial_bytes / 4 : 0, s,
                                           &launched);
@@ -454,7 +506,17 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
   const float scale = alpha / static_cast<float>(r);
 
   // XA = X A^T [M, n r] (saved in bf16 unless XA_saved is NULL) and s * XA: every adapter's
-  // down-projection in one pass over X.
+  // down-projection in one pass over X -- inside the GEMM launch below when its schedule allows
+  // (whole tiles: the GEMM streams every X tile anyway), else as a launch of its own.
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (g_rank_fusion.load(std::memory_order_relaxed) && M > kGemvMaxTokens &&
+      gemm_rank_fusable(M, W->N, W->K / 64 + ext_steps(r), sms, R,
+                                              gemm_rank_slot_bytes(false, R, r))) {
+    const RankFusion f{A, R, r, single_group(W->K), XA_saved, sxa, scale,
+                       reinterpret_cast<unsigned*>(w8 + L.flags), L.flags_bytes};
+    return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s, &f);
+  }
   st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa, err, s);
   if (st != QLORA_OK) return st;
   // h = X deq(W0)^T + (s XA_g) B_g^T for the rows of each adapter g, in one launch.
@@ -494,13 +556,26 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
     st = do_lora_grad(dY, M, W->N, dyb, r, g, scale, dB, true, err, s);
     if (st != QLORA_OK) return st;
   }
-  // dYB = dY B_bd [M, n r] (bf16, for dA) and s * dYB, B_bd the block-diagonal of the B_g.
-  st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, err, s);
-  if (st != QLORA_OK) return st;
+  // dYB = dY B_bd [M, n r] (bf16, for dA) and s * dYB, B_bd the block-diagonal of the B_g --
+  // inside the dX launch when its schedule allows, else as a launch of its own.
   // dX = dY deq(W0) + (s dYB) A: one extension over all n r columns sums the adapters' terms.
-  if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
-                          L.scratch_bytes, s)) != QLORA_OK)
-    return st;
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dX && g_rank_fusion.load(std::memory_order_relaxed) &&
+      gemm_rank_fusable(M, W->K, W->N / 64 + ext_steps(R), sms, R,
+                              gemm_rank_slot_bytes(true, R, r))) {
+    const RankFusion f{B, R, r, g, dyb, sdyb, scale, reinterpret_cast<unsigned*>(w8 + L.flags),
+                       L.flags_bytes};
+    st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
+                 L.scratch_bytes, s, &f);
+    if (st != QLORA_OK) return st;
+  } else {
+    st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, err, s);
+    if (st != QLORA_OK) return st;
+    if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
+                            L.scratch_bytes, s)) != QLORA_OK)
+      return st;
+  }
   // dB_g = s dY_g^T XA_g  [N, r];  dA = s dYB^T X  [n r, K] (one launch when they match).
   if (XA_saved)
     return do_weight_grads(dY, X, XA_saved, dyb, M, W->N, W->K, r, g, scale, dA, dB, err, s);
@@ -741,6 +816,22 @@ qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count
   *grid = sc.grid;
   *partial_bytes = 4 * sc.partial_floats;
   return QLORA_OK;
+}
+
+int qlora_set_rank_fusion(int enable) {
+  return g_rank_fusion.exchange(enable ? 1 : 0, std::memory_order_relaxed);
+}
+
+int qlora_gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int rank_cols,
+                            int r, int transpose_w, int* bt) {
+  if (bt) *bt = 0;
+  if (M < 1 || rows_w < 1 || steps_per_tile < 2 || sm_count < 1 || r < 8 || r > rank_cols)
+    return 0;
+  if (!gemm_rank_fusable(M, rows_w, steps_per_tile, sm_count, rank_cols,
+                         gemm_rank_slot_bytes(transpose_w != 0, rank_cols, r)))
+    return 0;
+  if (bt) *bt = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, true).bt;
+  return 1;
 }
 
 qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream) {

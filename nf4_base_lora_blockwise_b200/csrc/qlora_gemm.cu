@@ -78,9 +78,7 @@ constexpr int kGroupThreads = 256;
 constexpr uint32_t kWBytes = 16384;         // 128 rows x 64 bf16
 constexpr uint32_t kQBytes = 4096;          // packed codes of one weight tile step
 constexpr int kRowsW = 128;                 // MMA M
-constexpr uint32_t kSmemLimit = 232448;
 constexpr int kWStages = 2 * kGroups;       // two W slots per group
-constexpr int kMaxQPerGroup = 16;
 constexpr int kAmAhead = 3;                 // owned steps the block absmax is fetched ahead
 
 struct Plan {
@@ -93,17 +91,25 @@ struct Plan {
   int qlog;      // log2 of the Q slots per dequant group
   uint32_t acc_cols;  // TMEM columns per half accumulator
   uint32_t x_bytes;   // bytes per X half-slot
+  uint32_t rank_slot; // fused down-projection: bytes of one rank-operand tile (0: not fused)
+  int rank_slots;     // tiles of its ring: dx (one per X ring step), 0 when it does not fit
   size_t smem;
 };
 
+constexpr uint32_t kSmemMax = 232448;  // dynamic shared memory of one CTA (227 KB)
+
 // Small token tiles leave shared memory for a deeper code ring: with few tokens a step is
-// short and the weight stream is the whole job, so more code tiles stay in flight.
-__host__ __device__ inline Plan make_plan(int bt, int nh) {
+// short and the weight stream is the whole job, so more code tiles stay in flight.  A fused
+// launch puts the rank operand's ring (one rank_slot-byte tile per X ring step) after the
+// barriers, giving up code-ring depth if it would not fit otherwise.
+__host__ __device__ inline Plan make_plan(int bt, int nh, uint32_t rank_slot = 0) {
   Plan p;
   p.bt = bt;
   p.nh = nh;
   p.x_bytes = static_cast<uint32_t>(bt) * 128u;
-  p.acc_cols = bt <= 16 ? 16u : (bt <= 32 ? 32u : (bt <= 64 ? 64u : (bt <= 128 ? 128u : 256u)));
+  // (Fused launches keep the accumulator at exactly bt columns: the rank window follows it.)
+  p.acc_cols = rank_slot ? static_cast<uint32_t>(bt)
+                         : (bt <= 16 ? 16u : (bt <= 32 ? 32u : (bt <= 64 ? 64u : (bt <= 128 ? 128u : 256u))));
   p.nacc = (2u * nh * p.acc_cols <= 512u) ? 2 : 1;
   p.qlog = bt <= 64 ? 4 : (bt <= 128 ? 3 : 2);
   // X slots are recycled on the W ring's empty barriers, which allows at most 4 steps of X
@@ -111,9 +117,21 @@ __host__ __device__ inline Plan make_plan(int bt, int nh) {
   p.dx = nh == 2 ? 2 : 4;
   p.dxlog = nh == 2 ? 1 : 2;
   p.sx = p.dx * nh;
-  const uint32_t sq = static_cast<uint32_t>(kGroups) << p.qlog;
-  const uint32_t fixed = 1024u + 1024u + sq * kQBytes + kWStages * kWBytes;
-  p.smem = fixed + static_cast<size_t>(p.sx) * p.x_bytes;
+  p.rank_slot = rank_slot;
+  p.rank_slots = 0;
+  for (;;) {
+    const uint32_t sq = static_cast<uint32_t>(kGroups) << p.qlog;
+    const uint32_t fixed = 1024u + 1024u + sq * kQBytes + kWStages * kWBytes;
+    p.smem = fixed + static_cast<size_t>(p.sx) * p.x_bytes;
+    if (rank_slot == 0) break;
+    const size_t ring = static_cast<size_t>(p.dx) * rank_slot;  // one tile per X ring step
+    if (p.smem + ring <= kSmemMax || p.qlog <= 1) {
+      p.rank_slots = p.smem + ring <= kSmemMax ? p.dx : 0;
+      p.smem += static_cast<size_t>(p.rank_slots) * rank_slot;
+      break;
+    }
+    --p.qlog;
+  }
   return p;
 }
 
@@ -168,17 +186,70 @@ __device__ __forceinline__ void group_sync(int g) {
 __device__ __forceinline__ int w_slot(int it) { return 2 * (it & 1) + ((it >> 1) & 1); }
 __device__ __forceinline__ uint32_t w_par(int it) { return static_cast<uint32_t>(it >> 2) & 1u; }
 
-template <bool kTransW>
+// ---------------------------------------------------------------------------------------------
+// Fused rank-r down-projection (forward X A^T, dX dY B_bd) on the tensor cores.  A token tile's
+// rank product is cut into 128-token windows, two per token half of 128 < bt <= 240 tokens:
+// rows 0-127 of the half, and rows bt-128 .. bt-1, which writes rows 128 .. bt-1.  Window w is
+// computed by the token tile's w-th tile, which runs in the first wave of tiles that reaches the
+// token tile (the host checks), so every other tile of it starts no earlier.  On each activation
+// step that tile's MMA thread adds four M = 128 MMAs: the window's rows of the activation tile
+// already in shared memory (A operand, K-major) times the step's rank-operand tile (B operand:
+// forward, A's n r rows [K-major]; dX, B's 64 rows [MN-major]), accumulated in TMEM columns past
+// the tile's accumulator.  After the last activation step the epilogue warps read the window,
+// write its rank values (bf16) and count it in the token tile's flag (one count per warp, four
+// per window), which the extension step of every tile of that token tile waits on.
+// ---------------------------------------------------------------------------------------------
+constexpr int kRankMaxCols = 32;  // n r of a fused launch
+
+struct RankWindow {
+  int has;   // this tile computes a window
+  int h;     // token half of the window
+  int w0;    // first row of the window within the half
+  int own0;  // first window row it writes (it writes rows own0 .. 127)
+  int nwin;  // windows of the token tile
+};
+
+// Windows of a token half with `toks` valid tokens.
+__host__ __device__ inline int half_windows(int toks) {
+  return toks <= 0 ? 0 : (toks <= 128 ? 1 : 2);
+}
+
+__host__ __device__ inline RankWindow rank_window(int t, int row_tiles, int M, int bt, int nh) {
+  RankWindow w;
+  const int tt = bt * nh;
+  const int tq = t / row_tiles;
+  const int rt = t - tq * row_tiles;
+  const int rest = M - tq * tt;
+  const int n0 = half_windows(rest < bt ? rest : bt);
+  const int n1 = nh == 2 ? half_windows(rest - bt < bt ? rest - bt : bt) : 0;
+  w.nwin = n0 + n1;
+  w.has = rt < w.nwin ? 1 : 0;
+  w.h = rt < n0 ? 0 : 1;
+  const int which = rt - (w.h ? n0 : 0);
+  w.w0 = which == 0 ? 0 : bt - 128;
+  w.own0 = which == 0 ? 0 : 256 - bt;
+  return w;
+}
+
+// Tiles of token tile tq in the first wave of G tiles that reaches it.
+__host__ __device__ inline int first_wave_tiles(int tq, int row_tiles, int G) {
+  const long long t0 = static_cast<long long>(tq) * row_tiles;
+  const long long wave_end = (t0 / G + 1) * G;
+  return static_cast<int>(wave_end - t0 < row_tiles ? wave_end - t0 : row_tiles);
+}
+
+template <bool kTransW, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_ext_w,
-                      const __grid_constant__ CUtensorMap tm_ext_act, const GemmArgs args) {
+                      const __grid_constant__ CUtensorMap tm_ext_act,
+                      const __grid_constant__ CUtensorMap tm_rank, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-  const Plan P = make_plan(args.bt, args.nh);
+  const Plan P = make_plan(args.bt, args.nh, kFused ? args.rank_slot : 0u);
   const int bt = P.bt, nh = P.nh, SX = P.sx, DX = P.dx, DXLOG = P.dxlog;
   const int qper = 1 << P.qlog;          // Q slots per dequant group
   const int SQ = kGroups * qper;
@@ -195,7 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* accfull = qempty + SQ;   // [2]
   uint64_t* accempty = accfull + 2;  // [2]
   uint64_t* drain = accempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* rank_full = drain + 1;  // fused: the window's MMAs have retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rank_full + 1);
+  uint8_t* rank_ring = x_ring + SX * P.x_bytes + 1024;  // fused: DX rank-operand tiles
 
   auto WS = [&](int it) { return w_ring + w_slot(it) * kWBytes; };
   auto QS = [&](int qi) { return q_ring + qi * kQBytes; };
@@ -237,6 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tile_cols = static_cast<uint32_t>(nh) * P.acc_cols;
   uint32_t ncols = static_cast<uint32_t>(P.nacc) * tile_cols;
   if (ncols < 32) ncols = 32;
+  // Fused: the rank window's columns follow the accumulator (the allocation is a power of 2).
+  const uint32_t rank_col0 = tile_cols;
+  if (kFused) ncols = 512;
+  const uint32_t rank_bytes = P.rank_slot;
   int* err = args.err;
 
   if (threadIdx.x == 0) {
@@ -254,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(accempty + b, 4);
     }
     mbar_init(drain, 1);
+    mbar_init(rank_full, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -272,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
       tma_prefetch_desc(&tm_ext_act);
+      if (kFused) tma_prefetch_desc(&tm_rank);
       int issued = 0;  // steps whose X tiles were issued
       bool ok = true;
       for (int it = 0; ok && it < n_steps;) {
@@ -279,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         segment(it, t, k0, len);
         const int tq = t / row_tiles;
         const int tok0 = tq * tile_tokens;
+        const RankWindow win = kFused ? rank_window(t, row_tiles, args.M, bt, nh) : RankWindow{};
         // Forward: the tile's adapter picks its r columns of the packed [M, n, r] operand.
         const int eg = kTransW ? 0 : row_group(args.groups, (t - tq * row_tiles) * kRowsW);
         for (int k = k0; k < k0 + len; ++k, ++it) {
@@ -288,14 +368,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          // Fused: the extension operand of this token tile is complete once all of its windows
+          // are published (acquire), and the TMA read below is ordered after that.
+          if (kFused && k == kt) {
+            if (!wait_count(args.rank_flags + tq, 4u * static_cast<unsigned>(win.nwin),
+                            kErrWaitRank, err, it)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+          }
+          // Fused, on a window's tile: the step's rank-operand tile rides on half 0's barrier.
+          const bool rank_step = win.has && k < kt;
           for (int h = 0; h < nh; ++h) {
             const int xs = x_slot(it, h);
             uint8_t* dst = x_ring + xs * P.x_bytes;
-            mbar_arrive_expect_tx(xfull + xs, P.x_bytes);
+            mbar_arrive_expect_tx(xfull + xs, P.x_bytes + (rank_step && h == 0 ? rank_bytes : 0u));
             if (k < kt)
               tma_load_2d(dst, &tm_act, xfull + xs, k * 64, tok0 + h * bt);
             else
               tma_load_3d(dst, &tm_ext_act, xfull + xs, (k - kt) * 64, eg, tok0 + h * bt);
+          }
+          if (rank_step) {
+            uint8_t* rdst = rank_ring + (it & (DX - 1)) * rank_bytes;
+            uint64_t* bar = xfull + x_slot(it, 0);
+            if (!kTransW)
+              tma_load_2d(rdst, &tm_rank, bar, k * 64, 0);  // A [n r rows, 64 k]
+            else
+              tma_load_2d(rdst, &tm_rank, bar, 0, k * 64);  // B [64 n rows, r]
           }
           issued = it + 1;
         }
@@ -363,11 +463,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t w_slot_step = kWBytes >> 4;
       const uint64_t x_slot_step = P.x_bytes >> 4;
       const uint32_t half_cols = P.acc_cols;
+      // Fused rank window: M = 128 tokens x N = the rank columns (forward: n r rounded up to 16,
+      // B K-major; dX: one adapter's r, B MN-major in rows of 2r bytes, 32B or 64B swizzle).
+      const uint32_t rank_r = static_cast<uint32_t>(args.rank_r);
+      const uint32_t rank_n =
+          kTransW ? rank_r : static_cast<uint32_t>((args.rank_cols + 15) / 16 * 16);
+      const uint32_t idesc_rank = idesc_bf16_f32(128, rank_n < 16 ? 16u : rank_n, 0u,
+                                                 kTransW ? 1u : 0u);
+      const uint32_t rank_base = smem_u32(rank_ring);
+      const uint32_t rank_pitch = 2u * rank_r;  // dX tile row bytes
+      const uint32_t rank_layout = rank_r == 16 ? 6u : 4u;
       int it = 0, seg = 0;
       bool ok = true;
       while (ok && it < n_steps) {
         int t, k0, len;
         segment(it, t, k0, len);
+        const RankWindow win = kFused ? rank_window(t, row_tiles, args.M, bt, nh) : RankWindow{};
         const int ab = P.nacc == 2 ? (seg & 1) : 0;
         const int use = P.nacc == 2 ? (seg >> 1) : seg;
         if (!mbar_wait(accempty + ab, (static_cast<uint32_t>(use) & 1u) ^ 1u, kErrWaitAcc, err,
@@ -398,6 +509,37 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (nh == 2)
                 umma_f16_ss(dtm + half_cols, ad + j * w_kstep, bd1 + j * x_kstep, idesc, acc);
             }
+            if (win.has) {
+              // The window's rows of this step's activation tile times its rank-operand tile.
+              const uint64_t wa = xdesc0 + static_cast<uint64_t>(xs + win.h) * x_slot_step +
+                                  static_cast<uint64_t>(win.w0 * 8);  // w0 rows of 128 B
+              const uint32_t rs = rank_base + static_cast<uint32_t>(it & (DX - 1)) * rank_bytes;
+              if (!kTransW) {
+                const uint64_t rb = smem_desc_sw128(rs, 16u, 1024u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  umma_f16_ss(tmem_base + rank_col0, wa + j * x_kstep, rb + j * (32u >> 4),
+                              idesc_rank, (k > 0 || j > 0) ? 1u : 0u);
+              } else {
+                // Adapter g of these 64 rows of B adds to its r columns only; its first step
+                // starts their sum.
+                const int g = row_group(args.rank_groups, k * 64);
+                int first_row = 0;
+#pragma unroll
+                for (int q = 0; q < kMaxGroups - 1; ++q)
+                  if (q + 1 < args.rank_groups.n && q + 1 <= g) first_row = args.rank_groups.end[q];
+                const uint32_t d = tmem_base + rank_col0 + static_cast<uint32_t>(g) * rank_r;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint64_t rb =
+                      smem_desc(rs + static_cast<uint32_t>(j) * 16u * rank_pitch, 0u,
+                                8u * rank_pitch, rank_layout);
+                  umma_f16_ss(d, wa + j * x_kstep, rb, idesc_rank,
+                              (k * 64 > first_row || j > 0) ? 1u : 0u);
+                }
+              }
+              if (k == kt - 1) umma_commit(rank_full);
+            }
           } else {
             const int rem = args.r_pad16 - (k - kt) * 64;
             const int nk = (rem >= 64 ? 64 : rem) / 16;
@@ -423,10 +565,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     // as fp32 to this CTA's head (0) or tail (1) partial slot of the workspace.
     const int quad = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    int seg = 0;
+    int seg = 0, nwin_done = 0;
     for (int it = 0; it < n_steps; ++seg) {
       int t, k0, len;
       segment(it, t, k0, len);
+      if (kFused) {
+        // Fused: publish this tile's rank window (if any) as soon as its MMAs retire, before the
+        // tile's extension step can run.  Lane = window row = token.
+        const RankWindow win = rank_window(t, row_tiles, args.M, bt, nh);
+        if (win.has) {
+          bool got = true;
+          if (lane == 0)
+            got = mbar_wait_sleepy(rank_full, static_cast<uint32_t>(nwin_done) & 1u, kErrWaitAcc,
+                                   err, seg);
+          if (!__shfl_sync(0xFFFFFFFFu, got, 0)) break;
+          __syncwarp();
+          tc_fence_after();
+          ++nwin_done;
+          const int wrow = quad * 32 + lane;
+          const int tq = t / row_tiles;
+          const int tok = tq * tile_tokens + win.h * bt + win.w0 + wrow;
+          const bool mine = wrow >= win.own0 && tok < args.M;
+          const int R = args.rank_cols;
+          const uint32_t tb = tmem_base + lane_base + rank_col0;
+          for (int c8 = 0; c8 < R / 8; ++c8) {
+            uint32_t v[8];
+            tmem_ld_32x32b_x8(tb + static_cast<uint32_t>(c8 * 8), v);
+            tmem_ld_wait();
+            if (mine) {
+              const long long o = static_cast<long long>(tok) * R + c8 * 8;
+#pragma unroll
+              for (int e = 0; e < 8; e += 2) {
+                const float v0 = __uint_as_float(v[e]), v1 = __uint_as_float(v[e + 1]);
+                if (args.rank_saved)
+                  *reinterpret_cast<__nv_bfloat162*>(args.rank_saved + o + e) =
+                      __floats2bfloat162_rn(v0, v1);
+                *reinterpret_cast<__nv_bfloat162*>(args.rank_scaled + o + e) =
+                    __floats2bfloat162_rn(args.rank_scale * v0, args.rank_scale * v1);
+              }
+            }
+          }
+          tc_fence_before();
+          __threadfence();
+          fence_proxy_async_global();
+          __syncwarp();
+          // Each epilogue warp counts its own 32 rows (no barrier across the warps, which a
+          // failed wait in one of them could leave waiting): a window is 4 counts.
+          if (lane == 0) atomicAdd(args.rank_flags + tq, 1u);
+        }
+      }
       const bool whole = k0 == 0 && len == total;
       const int slot = it == 0 ? 0 : 1;
       it += len;
@@ -707,8 +894,24 @@ double whole_tile_cycles(int M, int rows_w, int steps, int G, int bt, int nh) {
 
 }  // namespace
 
-GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count) {
+GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count, bool fused) {
   GemmTile t;
+  if (fused && M > 256) {
+    // The fused down-projection's windows need two halves of 128 < bt <= 240 tokens: take the
+    // cheapest such tile by the same model.
+    const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
+    double best = 0.0;
+    t.nh = 2;
+    t.bt = 240;
+    for (int bt = 240; bt >= 144; bt -= 16) {
+      const double c = whole_tile_cycles(M, rows_w, steps_per_tile, G, bt, 2);
+      if (bt == 240 || c < best) {
+        best = c;
+        t.bt = bt;
+      }
+    }
+    return t;
+  }
   if (M <= 256) {  // one half: as many tokens as there are, in steps of 16
     t.bt = M < 16 ? 16 : (M + 15) / 16 * 16;
     t.nh = 1;
@@ -752,9 +955,9 @@ cudaError_t gemm_device_sms(int* sms) {
 
 size_t gemm_smem_bytes(int bt, int nh) { return make_plan(bt, nh).smem; }
 
-GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count) {
+GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count, bool fused) {
   GemmSchedule sc;
-  const GemmTile tl = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count);
+  const GemmTile tl = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, fused);
   const int tile_tokens = tl.bt * tl.nh;
   sc.n_tiles = ((rows_w + kRowsW - 1) / kRowsW) * ((M + tile_tokens - 1) / tile_tokens);
   const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
@@ -772,6 +975,39 @@ GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count) 
   return sc;
 }
 
+bool gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int rank_cols,
+                       unsigned rank_slot) {
+  if (rank_cols < 8 || rank_cols > kRankMaxCols || rank_cols % 8 != 0 || rank_slot == 0)
+    return false;
+  if (M <= 256) return false;
+  const GemmTile tl = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, true);
+  const GemmSchedule sc = gemm_schedule(M, rows_w, steps_per_tile, sm_count, true);
+  if (sc.streamk) return false;
+  // Worth it while the fused tile costs the GEMM at most 4 % over its own choice of tile (the
+  // separate down-projection it replaces streams all of the activations once more).
+  const GemmTile own = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, false);
+  const GemmSchedule own_sc = gemm_schedule(M, rows_w, steps_per_tile, sm_count, false);
+  if (own_sc.streamk) return false;
+  const int G = sc.grid;
+  if (whole_tile_cycles(M, rows_w, steps_per_tile, G, tl.bt, tl.nh) >
+      1.04 * whole_tile_cycles(M, rows_w, steps_per_tile, G, own.bt, own.nh))
+    return false;
+  // The window's columns after the 2 bt accumulator columns, within TMEM's 512.
+  if (2 * tl.bt + (rank_cols + 15) / 16 * 16 > 512) return false;
+  const Plan p = make_plan(tl.bt, tl.nh, rank_slot);
+  if (p.rank_slots < p.dx || p.nacc != 1) return false;
+  const int tile_tokens = tl.bt * tl.nh;
+  const int row_tiles = (rows_w + kRowsW - 1) / kRowsW;
+  const int token_tiles = (M + tile_tokens - 1) / tile_tokens;
+  for (int tq = 0; tq < token_tiles; ++tq) {
+    const RankWindow w = rank_window(tq * row_tiles, row_tiles, M, tl.bt, tl.nh);
+    if (w.nwin > first_wave_tiles(tq, row_tiles, G)) return false;
+  }
+  return true;
+}
+
+size_t gemm_rank_flag_bytes(int M) { return 4 * (static_cast<size_t>(M) / 128 + 2); }
+
 size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile) {
   return 4 * gemm_schedule(M, rows_w, steps_per_tile, kGemmMaxCtas).partial_floats;
 }
@@ -783,31 +1019,29 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
   cudaError_t e = gemm_device_sms(&sms);
   if (e != cudaSuccess) return e;
   // The caller's tile (TMA boxes, smem plan) must be the one the schedule assumes.
-  const GemmTile tl = gemm_pick_tile(args.M, args.rows_w, args.kt + args.n_ext, sms);
+  const GemmTile tl = gemm_pick_tile(args.M, args.rows_w, args.kt + args.n_ext, sms, args.fuse);
   if (tl.bt != args.bt || tl.nh != args.nh) return cudaErrorInvalidValue;
-  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, sms);
+  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, sms, args.fuse);
   if (sc.streamk && (!args.partial || sc.partial_floats > partial_floats_avail)) {
     // No room for the partial sums: whole tiles, one CTA per tile.
     sc.streamk = 0;
     sc.grid = sc.n_tiles;
   }
   args.streamk = sc.streamk;
-  const size_t smem = gemm_smem_bytes(args.bt, args.nh);
-  if (!trans_w) {
-    e = cudaFuncSetAttribute(qlora_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(qlora_gemm_kernel<false>, dim3(sc.grid), dim3(kThreads), smem, stream, 1,
-                   maps.act, maps.q, maps.ext_w, maps.ext_act, args);
-    if (e != cudaSuccess) return e;
-  } else {
-    e = cudaFuncSetAttribute(qlora_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(qlora_gemm_kernel<true>, dim3(sc.grid), dim3(kThreads), smem, stream, 1,
-                   maps.act, maps.q, maps.ext_w, maps.ext_act, args);
-    if (e != cudaSuccess) return e;
-  }
+  if (args.fuse && (sc.streamk || !gemm_rank_fusable(args.M, args.rows_w, args.kt + args.n_ext,
+                                                      sms, args.rank_cols, args.rank_slot)))
+    return cudaErrorInvalidValue;
+  const size_t smem = make_plan(args.bt, args.nh, args.fuse ? args.rank_slot : 0u).smem;
+  // The fused down-projection is a separate instantiation, so the plain kernel carries none of
+  // its code.
+  auto kernel = trans_w ? (args.fuse ? qlora_gemm_kernel<true, true> : qlora_gemm_kernel<true, false>)
+                        : (args.fuse ? qlora_gemm_kernel<false, true> : qlora_gemm_kernel<false, false>);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kernel, dim3(sc.grid), dim3(kThreads), smem, stream, 1, maps.act, maps.q,
+                 maps.ext_w, maps.ext_act, maps.rank, args);
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   *launched = 1;

@@ -87,9 +87,11 @@ def test_workspace_bytes(lib):
     small = lib.qlora_workspace_bytes(64, 512, 256, 8)
     big = lib.qlora_workspace_bytes(4096, 4096, 4096, 16)
     # 4096^3 runs whole tiles and the rank-r products reduce inside their clusters, so the
-    # workspace is exactly the two bf16 rank-r activations; 64 tokens on a 512 x 256 weight
-    # run stream-K and add the GEMM's partial-sum slots.
-    assert big == 2 * 4096 * 16 * 2
+    # workspace is the two bf16 rank-r activations plus one 256-byte-aligned block of per-token-
+    # tile counters (4 bytes per 128 tokens, + 2) for the down-projection fused into the GEMM;
+    # 64 tokens on a 512 x 256 weight run stream-K and add the GEMM's partial-sum slots.
+    flags = (4 * (4096 // 128 + 2) + 255) // 256 * 256
+    assert big == 2 * 4096 * 16 * 2 + flags
     assert small > 2 * 64 * 8 * 2
 
 

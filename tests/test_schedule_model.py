@@ -198,3 +198,83 @@ def test_gemm_plan_headline_tile():
     from nf4_base_lora_blockwise_b200 import abi
     p = abi.qlora_gemm_plan(4096, 4096, 64 + 1, 148)
     assert (p["bt"], p["nh"], p["streamk"], p["grid"]) == (240, 2, 0, 148)
+
+
+def _windows(M, tq, bt, nh):
+    """The 128-token windows of token tile tq: per half with valid tokens, rows [0, 128) and,
+    past 128 valid tokens, rows [bt - 128, bt) writing rows 128 .. bt - 1.  Each window as
+    (half, first row, first row it writes)."""
+    rest = M - tq * bt * nh
+    out = []
+    for h in range(nh):
+        toks = min(bt, rest - h * bt)
+        if toks > 0:
+            out.append((h, 0, 0))
+        if toks > 128:
+            out.append((h, bt - 128, 256 - bt))
+    return out
+
+
+def _rank_ring_fits(bt, nh, slot):
+    """The GEMM's shared-memory plan with the rank operand's ring (one slot per X ring step)
+    after the W ring (4 x 16 KB), the code ring (2 << qlog tiles of 4 KB; shallower if needed),
+    the X ring (2 or 4 steps of bt x 128 B per half) and 2 KB of alignment and barriers."""
+    qlog = 4 if bt <= 64 else (3 if bt <= 128 else 2)
+    dx = 2 if nh == 2 else 4
+    while True:
+        smem = 2048 + (2 << qlog) * 4096 + 4 * 16384 + dx * nh * bt * 128
+        if smem + dx * slot <= 232448:
+            return True
+        if qlog <= 1:
+            return False
+        qlog -= 1
+
+
+def test_rank_fusion_decision_and_coverage():
+    """qlora_gemm_rank_fusable against a model of the fused down-projection's schedule.  When it
+    fuses, the launch runs whole tiles of two halves of 144..240 tokens (the accumulator's 2 bt
+    TMEM columns leave room for the window's), n r is a multiple of 8 up to 32 (dX: r = 16 or
+    32), the rank operand's ring fits in shared memory, and every token tile's windows fall on
+    its tiles in the first wave of tiles that reaches it, their written rows covering each valid
+    token exactly once.  It never fuses what the kernels cannot: n r above 32 or not a multiple
+    of 8, dX with r = 8 or 24, 256 tokens or fewer."""
+    import os
+    from nf4_base_lora_blockwise_b200 import abi
+    if not os.path.exists(abi.LIB_PATH):
+        from nf4_base_lora_blockwise_b200 import build
+        build.build()
+    rng = random.Random(23)
+    fused = 0
+    for _ in range(400):
+        M = rng.choice([17, 33, 300, 1024, 1300, 2048, 4096, 6000, 8192, 16384])
+        rows = 64 * rng.randint(2, 260)
+        steps = rng.randint(2, 200)
+        R = rng.choice([8, 16, 24, 32, 40, 64])
+        r = rng.choice([x for x in (8, 16, 24, 32) if x <= R and R % x == 0])
+        trans = rng.random() < 0.5
+        sms = rng.choice([132, 148])
+        bt = abi.qlora_gemm_rank_fusable(M, rows, steps, sms, R, r, trans)
+        if R > 32 or M <= 256 or (trans and r not in (16, 32)):
+            assert bt == 0, (M, rows, steps, R, r, trans)
+        if not bt:
+            continue
+        fused += 1
+        nh, G = 2, min(sms, 160)
+        npad = (R + 15) // 16 * 16
+        assert 144 <= bt <= 240 and bt % 16 == 0 and 2 * bt + npad <= 512
+        assert _rank_ring_fits(bt, nh, 128 * r if trans else 128 * npad)
+        row_tiles = (rows + 127) // 128
+        token_tiles = (M + bt * nh - 1) // (bt * nh)
+        assert row_tiles * token_tiles >= G  # whole tiles, one CTA per SM
+        for tq in range(token_tiles):
+            wins = _windows(M, tq, bt, nh)
+            t0 = tq * row_tiles
+            assert len(wins) <= min(row_tiles, (t0 // G + 1) * G - t0)
+            valid = min(bt * nh, M - tq * bt * nh)
+            cover = sorted(h * bt + w0 + row for h, w0, own0 in wins for row in range(own0, 128)
+                           if h * bt + w0 + row < valid)
+            assert cover == list(range(valid)), (M, tq, bt)
+    assert fused > 20
+    # The headline layer fuses in both directions: 4096 tokens, q_proj 4096 -> 4096, r = 16.
+    assert abi.qlora_gemm_rank_fusable(4096, 4096, 64 + 1, 148, 16, 16, False) == 240
+    assert abi.qlora_gemm_rank_fusable(4096, 4096, 64 + 1, 148, 16, 16, True) == 240
