@@ -233,8 +233,11 @@ QLORA_API qlora_status qlora_cross_entropy_mean(const float* token_loss, int M, 
  * With group_rows (w_is_r_by_c = 0 only): r = n r_g output columns, w = B [C, r_g] stacked by
  * adapter, and Wl is block-diagonal: rows of adapter g feed columns g r_g .. g r_g + r_g - 1.
  * The reduction over C is split across the CTAs of a thread-block cluster and summed in a fixed
- * order in distributed shared memory: no scratch is needed and ws / ws_bytes are ignored (may
- * be NULL / 0).  Results do not depend on timing. */
+ * order in distributed shared memory.  ws / ws_bytes (may be NULL / 0; 16-byte aligned): with
+ * few tokens the reduction is split further over several clusters whose fp32 partials (up to
+ * 128 r 4 bytes per 128 tokens for each cluster) go to ws and a second launch adds them in
+ * cluster order; without room in ws it stays on one cluster per 128 tokens.  Either way the
+ * results do not depend on timing. */
 QLORA_API qlora_status qlora_lora_down(const void* in, int M, int C, const void* w,
                                        int w_is_r_by_c, int r, const int* group_rows,
                                        int n_groups, float scale, void* saved, void* scaled,
@@ -260,8 +263,7 @@ QLORA_API qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W
  * small [M, r] bf16 device; written fp32 as out [C, r] (out_r_by_c = 0, e.g. dB) or
  * out [r, C] (out_r_by_c = 1, e.g. dA).  With group_rows (adapters along big's columns):
  * small is [M, n r] and column c of adapter g uses small[m, g r + j].
- * Reduced over M inside thread-block clusters like qlora_lora_down: ws / ws_bytes are ignored
- * (may be NULL / 0). */
+ * Reduced over M inside thread-block clusters: ws / ws_bytes are ignored (may be NULL / 0). */
 QLORA_API qlora_status qlora_lora_grad(const void* big, int M, int C, const void* small, int r,
                                        const int* group_rows, int n_groups, float scale,
                                        float* out, int out_r_by_c, void* ws, size_t ws_bytes,

@@ -222,18 +222,24 @@ struct RankPlan {
   SmallTile small;  // the Wl / small tile of one stage
   int box_rows_in;  // TMA box height of `in` / `big`
   int box_rows_w;   // TMA box height of Wl (A: R; B: 64 or 256) / small (64)
+  int gsplit;       // down, few tokens: clusters per row tile along the reduction (1: one),
+                    // their fp32 partials summed in order by a finalize kernel
+  size_t part_bytes;  // scratch those partials take
 };
 struct RankMaps {
   CUtensorMap big;    // in / big [M, C] bf16: box {64, 128} (down) or {64, 64} (grad), SW128
   CUtensorMap small;  // down: A [R, C] box {64, R} SW128, or B [C, rg] per small_tile(rg);
                       // grad: small [M, ld_small] per small_tile(R)
 };
-RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count);
+// scratch_bytes: workspace the plan may use for a second-level split of the reduction.
+RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count,
+                        size_t scratch_bytes = 0);
 RankPlan rank_grad_plan(int M, int C, int R, int sm_count);
+// scratch: p.part_bytes of workspace when p.gsplit > 1 (then a finalize kernel follows).
 cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int C, int R, int rg,
                              bool w_rc, const RowGroups& groups, float scale,
                              __nv_bfloat16* saved, __nv_bfloat16* scaled, int* err,
-                             cudaStream_t stream);
+                             cudaStream_t stream, float* scratch = nullptr);
 cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int C, int R,
                              int ld_small, const RowGroups& groups, float scale, float* out,
                              bool out_cr, int* err, cudaStream_t stream);

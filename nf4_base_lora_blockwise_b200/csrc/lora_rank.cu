@@ -125,6 +125,8 @@ struct RankArgs {
   float* out;             // grad: scale * G, [C, R] (out_cr) or [R, C]
   int out_cr;
   int* err;
+  int gsplit;             // down: clusters per row tile along the reduction
+  float* gpart;           // down, gsplit > 1: fp32 partials [tiles][gsplit][128][R]
 };
 
 namespace {
@@ -173,10 +175,14 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
   uint64_t* empty = full + a.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int tile = static_cast<int>(blockIdx.x) / a.split;
+  // Cluster gc of tile `tile` takes part gc of the reduction; CTA `rank` of it, its own share.
+  const int per_tile = a.split * a.gsplit;
+  const int tile = static_cast<int>(blockIdx.x) / per_tile;
+  const int gc = (static_cast<int>(blockIdx.x) / a.split) % a.gsplit;
   const int row0 = tile * kTileRows;
-  const int s0 = static_cast<int>(static_cast<long long>(a.steps) * rank / a.split);
-  const int n = static_cast<int>(static_cast<long long>(a.steps) * (rank + 1) / a.split) - s0;
+  const int part_idx = gc * a.split + static_cast<int>(rank);
+  const int s0 = static_cast<int>(static_cast<long long>(a.steps) * part_idx / per_tile);
+  const int n = static_cast<int>(static_cast<long long>(a.steps) * (part_idx + 1) / per_tile) - s0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -300,7 +306,11 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
         v.z += p[q].z;
         v.w += p[q].w;
       }
-    if (m < a.M) {
+    if (a.gsplit > 1) {
+      // This cluster's share of the reduction, for the finalize to add in cluster order.
+      float* dst = a.gpart + ((static_cast<long long>(tile) * a.gsplit + gc) * kTileRows + rl) * a.R + c4;
+      *reinterpret_cast<float4*>(dst) = v;
+    } else if (m < a.M) {
       const long long o = static_cast<long long>(m) * a.R + c4;
       if (a.saved) {
         __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
@@ -318,6 +328,42 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
     }
   }
   cluster_sync_all();  // no CTA leaves while another still reads its partial
+}
+
+// The second-level split's sum: out[m, c4 .. c4+3] adds the gsplit cluster partials of m's
+// tile in cluster order, then rounds to bf16 (saved) and scales (scaled).
+__global__ void __launch_bounds__(256) rank_down_finalize(const RankArgs a) {
+  pdl_wait();  // the partials are complete
+  pdl_trigger();
+  const int items = a.M * (a.R / 4);
+  const int it = static_cast<int>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (it >= items) return;
+  const int m = it / (a.R / 4);
+  const int c4 = (it - m * (a.R / 4)) * 4;
+  const int tile = m / kTileRows, rl = m - tile * kTileRows;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int g = 0; g < a.gsplit; ++g) {
+    const float4 p = __ldg(reinterpret_cast<const float4*>(
+        a.gpart + ((static_cast<long long>(tile) * a.gsplit + g) * kTileRows + rl) * a.R + c4));
+    v.x += p.x;
+    v.y += p.y;
+    v.z += p.z;
+    v.w += p.w;
+  }
+  const long long o = static_cast<long long>(m) * a.R + c4;
+  if (a.saved) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.saved + o) = pk;
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a.scale * v.x, a.scale * v.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(a.scale * v.z, a.scale * v.w);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(a.scaled + o) = pk;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -664,8 +710,11 @@ namespace {
 
 }  // namespace
 
-RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count) {
+RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count,
+                        size_t scratch_bytes) {
   RankPlan p;
+  p.gsplit = 1;
+  p.part_bytes = 0;
   const int row_ctas = (M + kRowRows - 1) / kRowRows;
   // (A [R, C] only: with B the 256-row box of narrow rows measured slower than the cluster kernel.)
   if (w_rc && R <= 32 && 3 * row_ctas >= 2 * sm_count) {
@@ -687,7 +736,16 @@ RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count) {
   p.rows = 0;
   const int tiles = (M + kTileRows - 1) / kTileRows;
   p.split = pick_split(tiles, C / 64, sm_count);
-  p.grid = tiles * p.split;
+  // Few tokens: too few clusters to stream `in` at full rate, so split the reduction further
+  // over gsplit clusters (at least two steps each, within two CTAs per SM) when the workspace
+  // holds their partials.
+  while (tiles * p.split * p.gsplit * 2 <= 2 * sm_count &&
+         p.split * p.gsplit * 2 * 2 <= C / 64 &&
+         static_cast<size_t>(tiles) * p.gsplit * 2 * kTileRows * R * 4 <= scratch_bytes)
+    p.gsplit *= 2;
+  if (p.gsplit > 1)
+    p.part_bytes = static_cast<size_t>(tiles) * p.gsplit * kTileRows * R * 4;
+  p.grid = tiles * p.split * p.gsplit;
   p.box_rows_in = kTileRows;
   p.small = w_rc ? SmallTile{1, 64, 128u, 7u, 128, static_cast<uint32_t>(R) * 128u}
                  : small_tile(rg);
@@ -700,6 +758,8 @@ RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count) {
 
 RankPlan rank_grad_plan(int M, int C, int R, int sm_count) {
   RankPlan p;
+  p.gsplit = 1;
+  p.part_bytes = 0;
   p.rows = 0;
   p.box_rows_in = 64;
   p.box_rows_w = 64;
@@ -712,6 +772,9 @@ RankPlan rank_grad_plan(int M, int C, int R, int sm_count) {
   p.smem = L.smem;
   return p;
 }
+
+cudaError_t launch_down_cluster(const RankMaps& maps, const RankPlan& p, int R, bool w_rc,
+                                const RankArgs& a, cudaStream_t stream);
 
 #define QLORA_RANK_DOWN_CASE(NTV)                                                              \
   case NTV:                                                                                   \
@@ -730,8 +793,10 @@ RankPlan rank_grad_plan(int M, int C, int R, int sm_count) {
 cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int C, int R, int rg,
                              bool w_rc, const RowGroups& groups, float scale,
                              __nv_bfloat16* saved, __nv_bfloat16* scaled, int* err,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, float* scratch) {
   RankArgs a = {};
+  a.gsplit = 1;
+  a.gpart = nullptr;
   a.M = M;
   a.C = C;
   a.R = R;
@@ -777,6 +842,20 @@ cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int
   a.saved = saved;
   a.scaled = scaled;
   a.err = err;
+  if (p.gsplit > 1) {
+    if (!scratch || R % 4 != 0) return cudaErrorInvalidValue;
+    a.gsplit = p.gsplit;
+    a.gpart = scratch;
+    const cudaError_t e = launch_down_cluster(maps, p, R, w_rc, a, stream);
+    if (e != cudaSuccess) return e;
+    const int items = M * (R / 4);
+    return launch_pdl(rank_down_finalize, dim3((items + 255) / 256), dim3(256), 0, stream, 1, a);
+  }
+  return launch_down_cluster(maps, p, R, w_rc, a, stream);
+}
+
+cudaError_t launch_down_cluster(const RankMaps& maps, const RankPlan& p, int R, bool w_rc,
+                                const RankArgs& a, cudaStream_t stream) {
   switch (R / 8) {
     QLORA_RANK_DOWN_CASE(1)
     QLORA_RANK_DOWN_CASE(2)

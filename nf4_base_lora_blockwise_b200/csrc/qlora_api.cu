@@ -326,13 +326,15 @@ CUtensorMapSwizzle swizzle_of(int span) {
 }
 
 // groups: the adapters packed along the rows of B (w_rc = false); r is then n r_g.
+// scratch / scratch_bytes (nullable / 0): workspace for the few-token split of the reduction.
 qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc, int r,
                           const RowGroups& groups, float scale, void* saved, void* scaled,
-                          int* err, cudaStream_t s) {
+                          int* err, cudaStream_t s, void* scratch = nullptr,
+                          size_t scratch_bytes = 0) {
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
   const int rg = w_rc ? r : r / groups.n;
-  const RankPlan p = rank_down_plan(M, C, r, rg, w_rc, sms);
+  const RankPlan p = rank_down_plan(M, C, r, rg, w_rc, sms, scratch ? scratch_bytes : 0);
   RankMaps maps;
   qlora_status st = encode_2d(&maps.big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, in, C, M, C * 2ull,
                               64, p.box_rows_in, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -346,9 +348,10 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
   if (st != QLORA_OK) return st;
   const cudaError_t e = launch_rank_down(maps, p, M, C, r, rg, w_rc, groups, scale,
                                          static_cast<__nv_bfloat16*>(saved),
-                                         static_cast<__nv_bfloat16*>(scaled), err, s);
+                                         static_cast<__nv_bfloat16*>(scaled), err, s,
+                                         static_cast<float*>(scratch));
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  count(1);
+  count(p.gsplit > 1 ? 2 : 1);
   return QLORA_OK;
 }
 
@@ -517,7 +520,9 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
                        reinterpret_cast<unsigned*>(w8 + L.flags), L.flags_bytes};
     return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s, &f);
   }
-  st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa, err, s);
+  // (The GEMM's scratch is free until the GEMM runs: the few-token split uses it first.)
+  st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa, err, s,
+                    w8 + L.scratch, L.scratch_bytes);
   if (st != QLORA_OK) return st;
   // h = X deq(W0)^T + (s XA_g) B_g^T for the rows of each adapter g, in one launch.
   return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s);
@@ -551,7 +556,8 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
   // Without a saved XA, recompute it from X (the forward's own kernel on the same inputs, so
   // bit for bit the value it would have saved) and take dB first, while small0 holds it.
   if (!XA_saved) {
-    st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, dyb, sdyb, err, s);
+    st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, dyb, sdyb, err, s,
+                      scratch, L.scratch_bytes);
     if (st != QLORA_OK) return st;
     st = do_lora_grad(dY, M, W->N, dyb, r, g, scale, dB, true, err, s);
     if (st != QLORA_OK) return st;
@@ -570,7 +576,8 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
                  L.scratch_bytes, s, &f);
     if (st != QLORA_OK) return st;
   } else {
-    st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, err, s);
+    st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, err, s, scratch,
+                      L.scratch_bytes);
     if (st != QLORA_OK) return st;
     if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
                             L.scratch_bytes, s)) != QLORA_OK)
@@ -740,15 +747,14 @@ qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_
   }
   if (!aligned16(in) || !aligned16(w) || !aligned16(scaled) || (saved && !aligned16(saved)))
     return QLORA_ERR_ALIGN;
-  (void)ws;  // the cluster reduction needs no scratch
-  (void)ws_bytes;
+  if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
   int dev;
   qlora_status st = current_device(&dev);
   if (st != QLORA_OK) return st;
   int* err;
   if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
   return do_lora_down(in, M, C, w, w_is_r_by_c != 0, r, g, scale, saved, scaled, err,
-                      static_cast<cudaStream_t>(stream));
+                      static_cast<cudaStream_t>(stream), ws, ws ? ws_bytes : 0);
 }
 
 qlora_status qlora_nf4_gemm(const void* act, const qlora_nf4_weight* W, int transpose_w,

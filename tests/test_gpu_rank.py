@@ -136,3 +136,39 @@ def test_grad_per_adapter_columns(Ns, r):
         ref[edges[g]:edges[g + 1]] = 2.0 * _f64(big)[:, edges[g]:edges[g + 1]].T @ \
             _f64(small)[:, g * r:(g + 1) * r]
     assert qlora.rel_err(_f64(out), ref) <= TOL
+
+
+@pytest.mark.parametrize("M,C,R,w_rc", [(16, 14336, 16, False), (1, 14336, 16, False),
+                                        (100, 4096, 16, True), (16, 4096, 32, True),
+                                        (128, 14336, 24, False)])
+def test_down_few_tokens_split(M, C, R, w_rc):
+    """With workspace, few tokens split the reduction over several clusters: their fp32 partials
+    go to ws and a second launch adds them in cluster order.  Same bar against the oracle, within
+    a few bf16 ulps of the single-cluster result, and bit for bit on repeat."""
+    inp = _rand((M, C), 1.0, M + C + R)
+    w = _rand((R, C) if w_rc else (C, R), 0.05, R + 3)
+    inp, w = inp.cuda(), w.cuda()
+    ws = torch.empty(8 << 20, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+
+    def run(with_ws):
+        saved = torch.empty((M, R), dtype=torch.bfloat16, device="cuda")
+        scaled = torch.empty((M, R), dtype=torch.bfloat16, device="cuda")
+        n0 = abi.qlora_launch_counter()
+        abi.qlora_lora_down(inp.data_ptr(), M, C, w.data_ptr(), 1 if w_rc else 0, R, None, 2.0,
+                            saved.data_ptr(), scaled.data_ptr(),
+                            ws.data_ptr() if with_ws else None, ws.numel() if with_ws else 0, s)
+        torch.cuda.synchronize()
+        assert linear.device_error() == 0
+        return saved, scaled, abi.qlora_launch_counter() - n0
+
+    saved, scaled, n = run(True)
+    assert n == 2, "few tokens with workspace: the split reduction and its finalize"
+    ref = _f64(inp) @ (_f64(w).T if w_rc else _f64(w))
+    assert qlora.rel_err(_f64(saved), ref) <= TOL
+    assert qlora.rel_err(_f64(scaled), 2.0 * ref) <= TOL
+    one, _, n1 = run(False)
+    assert n1 == 1
+    assert (one.float() - saved.float()).abs().max() <= 2e-2 * saved.float().abs().max()
+    again, _, _ = run(True)
+    assert torch.equal(saved, again)
