@@ -187,6 +187,23 @@ struct GemvPlan {
   size_t partial_floats;
   size_t smem;
 };
+// dX for few tokens (nf4_dx_fewtok.cu): CTAs of 256 output columns x a range of weight rows,
+// fp32 partials per row split in the workspace, a finalize adding them in order with the LoRA
+// term.  Tile maps: codes [N, K/2] u8 box {128, 64} and dY [M, N] bf16 box {64, 16 mb}, both
+// 128B-swizzled.
+constexpr int kFewTokDxMaxTokens = 32;
+struct FewTokDxPlan {
+  int gk, splits, grid;
+  int mb;             // 16-token blocks (1 or 2)
+  size_t part_bytes;  // workspace the partials need
+};
+FewTokDxPlan fewtok_dx_plan(int M, int N, int K, int sm_count);
+cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_dy,
+                                 const FewTokDxPlan& p, int M, int N, int K, const float* absmax,
+                                 const uint8_t* absmax_q8, const float* absmax_scale, int dq,
+                                 const __nv_bfloat16* sdyb, const __nv_bfloat16* A, int R,
+                                 __nv_bfloat16* dx, float* part, size_t part_bytes,
+                                 const Codebook& cb, int* err, cudaStream_t stream);
 constexpr int kGemvMaxTokens = 32;
 GemvPlan gemv_plan(int M, int N, int K, int sm_count);
 cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const float* absmax,

@@ -44,11 +44,6 @@ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
   return swz_off(row, chunk, 128u, 7u);
 }
 
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
 // ---------------------------------- cluster helpers ---------------------------------------
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;

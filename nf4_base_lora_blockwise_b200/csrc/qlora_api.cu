@@ -189,8 +189,13 @@ int ext_steps(int r) { return ((r + 15) / 16 * 16 + 63) / 64; }
 // Stream-K partial-sum bytes of the forward (rows N, K/64 steps) or dX (rows K, N/64 steps).
 size_t gemm_ws_bytes(int M, int N, int K, int r, bool trans) {
   if (!trans && M <= kGemvMaxTokens) return 4 * gemv_plan(M, N, K, kGemmMaxCtas).partial_floats;
-  return trans ? gemm_partial_bytes_bound(M, K, N / 64 + ext_steps(r))
-               : gemm_partial_bytes_bound(M, N, K / 64 + ext_steps(r));
+  if (trans) {
+    const size_t sk = gemm_partial_bytes_bound(M, K, N / 64 + ext_steps(r));
+    if (M > kFewTokDxMaxTokens) return sk;
+    const size_t ft = fewtok_dx_plan(M, N, K, kGemmMaxCtas).part_bytes;  // few-token dX partials
+    return ft > sk ? ft : sk;
+  }
+  return gemm_partial_bytes_bound(M, N, K / 64 + ext_steps(r));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -378,6 +383,27 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   }
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (trans && M <= kFewTokDxMaxTokens && partial && !fuse) {
+    // Few tokens: dX streams the weight panel by panel without the tcgen05 rings' hand-offs.
+    const FewTokDxPlan fp = fewtok_dx_plan(M, W->N, W->K, sms);
+    if (fp.part_bytes <= partial_bytes) {
+      CUtensorMap mq, md;
+      qlora_status st = encode_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->q, W->K / 2, W->N,
+                                  W->K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (st != QLORA_OK) return st;
+      st = encode_2d(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, W->N, M, W->N * 2ull, 64,
+                     16 * fp.mb, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (st != QLORA_OK) return st;
+      const cudaError_t e = launch_nf4_fewtok_dx(
+          mq, md, fp, M, W->N, W->K, W->absmax, W->absmax_q8, W->absmax_scale,
+          W->double_quant ? 1 : 0, static_cast<const __nv_bfloat16*>(ext_act),
+          static_cast<const __nv_bfloat16*>(ext_w), r, static_cast<__nv_bfloat16*>(out),
+          static_cast<float*>(partial), partial_bytes, codebook(), err, s);
+      if (e != cudaSuccess) return QLORA_ERR_CUDA;
+      count(2);
+      return QLORA_OK;
+    }
+  }
   GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms, fuse != nullptr);
   a.partial = static_cast<float*>(partial);
   GemmMaps maps;
