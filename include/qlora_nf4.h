@@ -62,7 +62,8 @@ extern "C" {
 typedef enum {
   QLORA_OK = 0,
   QLORA_ERR_NULL = 1,      /* a required pointer is NULL */
-  QLORA_ERR_SHAPE = 2,     /* M < 1, N or K not a multiple of 64, r not in {8,16,...,128} */
+  QLORA_ERR_SHAPE = 2,     /* M < 1, N or K not a multiple of 64, r out of range: [1, 128] for
+                              qlora_linear_*, multiples of 8 in [8, 128] for the other calls */
   QLORA_ERR_ALIGN = 3,     /* a device pointer is not 16-byte aligned */
   QLORA_ERR_ARCH = 4,      /* current device is not compute capability 10.0 (sm_100a) */
   QLORA_ERR_WORKSPACE = 5, /* workspace NULL or smaller than qlora_workspace_bytes() */
@@ -109,9 +110,11 @@ QLORA_API qlora_status qlora_nf4_pack(const void* W, int N, int K, int double_qu
  * entry points never materialise it).  Uses the same device routine as the GEMM mainloop. */
 QLORA_API qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, qlora_stream_t stream);
 
-/* Scratch bytes the linear entry points need for (M, N, K, r): the scaled rank-r
- * activations, the fixed-order split partials of the rank-r reductions and the stream-K
- * partial sums of the dequant GEMM (sized for any device of up to 160 SMs).  Needs no GPU. */
+/* Scratch bytes the linear entry points need for (M, N, K, r), 1 <= r <= 128: the scaled rank-r
+ * activations, the fused down-projection's counters, the few-token split partials of the rank-r
+ * reductions and the stream-K partial sums of the dequant GEMM (sized for any device of up to
+ * 160 SMs), plus, for r not a multiple of 8, the zero-padded copies described below.  Needs no
+ * GPU; 0 for an invalid shape. */
 QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
 
 /* Forward.  X [M, K], A [r, K], B [N, r] bf16 device (read); H [M, N] bf16 device (written);
@@ -120,7 +123,11 @@ QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
  * Fine-Tuning Explained", "How does Unsloth make fine-tuning faster?": recompute instead of
  * store).
  * ws: device scratch of at least qlora_workspace_bytes(M, N, K, r) bytes.
- * alpha: LoRA alpha; s = alpha / r.  r must be a multiple of 8 in [8, 128].
+ * alpha: LoRA alpha; s = alpha / r.  1 <= r <= 128.  A rank that is not a multiple of 8 runs
+ * at r rounded up to 8 on zero-padded copies of A, B (and, backward, XA_saved) in ws, the
+ * padded rows and columns contributing exact zeros; the results are those of rank r, at the
+ * cost of a few device copies per call (the tensor-memory operands need rows of a multiple of
+ * 16 bytes).
  * For M <= 32 the base product applies each block's absmax to the block's 64-deep partial sum
  * (the weight enters as bf16(code value) * absmax rather than bf16(code value * absmax)); the
  * two agree within one bf16 rounding of the weight.  Larger M and dX use the dequantised
@@ -133,7 +140,7 @@ QLORA_API qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W
  * NULL: X A^T is then recomputed from X (one more pass over X), bit-identical to the value the
  * forward would have saved, so the results do not change.
  * dX [M, K] bf16 device (written; may be NULL to skip the dX GEMM).
- * dA [r, K] and dB [N, r] fp32 device (overwritten).  ws as for the forward. */
+ * dA [r, K] and dB [N, r] fp32 device (overwritten).  ws and r as for the forward. */
 QLORA_API qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
                               const void* A, const void* B, const void* XA_saved, int M, int r,
                               float alpha, void* dX, float* dA, float* dB, void* ws,

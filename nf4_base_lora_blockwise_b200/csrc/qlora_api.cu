@@ -228,6 +228,42 @@ WsLayout ws_layout(int M, int N, int K, int r) {
   return L;
 }
 
+// A single-adapter layer of rank r that is not a multiple of 8 runs at rp = r rounded up to 8
+// (the TMA operands need rows of a multiple of 16 bytes) on zero-padded copies kept after the
+// layer's own workspace: A [rp, K], B [N, rp], XA [M, rp], and the gradients dA [rp, K] and
+// dB [N, rp] in fp32, copied back into the caller's [r, K] / [N, r].
+int pad8(int r) { return (r + 7) / 8 * 8; }
+
+struct PadLayout {
+  size_t inner, a, b, xa, da, db, total;
+};
+
+PadLayout pad_layout(int M, int N, int K, int r) {
+  PadLayout P;
+  const size_t rp = static_cast<size_t>(pad8(r));
+  P.inner = ws_layout(M, N, K, static_cast<int>(rp)).total;
+  P.a = P.inner;
+  P.b = P.a + align256(rp * K * 2);
+  P.xa = P.b + align256(static_cast<size_t>(N) * rp * 2);
+  P.da = P.xa + align256(static_cast<size_t>(M) * rp * 2);
+  P.db = P.da + align256(rp * K * 4);
+  P.total = P.db + align256(static_cast<size_t>(N) * rp * 4);
+  return P;
+}
+
+// A [r, K] -> ap [rp, K] and B [N, r] -> bp [N, rp], zero elsewhere.
+qlora_status pad_factors(const void* A, const void* B, int r, int rp, int N, int K, void* ap,
+                         void* bp, cudaStream_t s) {
+  if (cudaMemsetAsync(ap, 0, static_cast<size_t>(rp) * K * 2, s) != cudaSuccess ||
+      cudaMemcpyAsync(ap, A, static_cast<size_t>(r) * K * 2, cudaMemcpyDeviceToDevice, s) !=
+          cudaSuccess ||
+      cudaMemsetAsync(bp, 0, static_cast<size_t>(N) * rp * 2, s) != cudaSuccess ||
+      cudaMemcpy2DAsync(bp, rp * 2ull, B, r * 2ull, r * 2ull, N, cudaMemcpyDeviceToDevice, s) !=
+          cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
 // The rank-r down-projection a dequant GEMM launch computes itself (see GemmArgs::fuse).
 struct RankFusion {
   const void* w;      // forward: A [n r, K]; dX: B [N, r]
@@ -513,8 +549,9 @@ qlora_status do_weight_grads(const void* dY, const void* X, const void* XA, cons
 // rank-r operands are [M, n r] / [n r, K]; dB is [N, r]; s = alpha / r for every adapter.
 // The caller has checked W and built `g`.
 // ---------------------------------------------------------------------------------------------
+// `scale` is alpha / r of the caller's rank (the padded-rank path passes r rounded up).
 qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A, const void* B,
-                        const RowGroups& g, int M, int r, float alpha, void* H, void* XA_saved,
+                        const RowGroups& g, int M, int r, float scale, void* H, void* XA_saved,
                         void* ws, size_t ws_bytes, cudaStream_t s) {
   if (!X || !A || !B || !H) return QLORA_ERR_NULL;
   const int R = g.n * r;
@@ -532,7 +569,6 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
   if ((st = error_word_ptr(dev, &err)) != QLORA_OK) return st;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   auto* sxa = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
-  const float scale = alpha / static_cast<float>(r);
 
   // XA = X A^T [M, n r] (saved in bf16 unless XA_saved is NULL) and s * XA: every adapter's
   // down-projection in one pass over X -- inside the GEMM launch below when its schedule allows
@@ -556,7 +592,7 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
 
 qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W, const void* A,
                         const void* B, const void* XA_saved, const RowGroups& g, int M, int r,
-                        float alpha, void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                        float scale, void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
                         cudaStream_t s) {
   if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_NULL;
   const int R = g.n * r;
@@ -577,7 +613,6 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
   auto* dyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small0);
   auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
   float* scratch = reinterpret_cast<float*>(w8 + L.scratch);
-  const float scale = alpha / static_cast<float>(r);
 
   // Without a saved XA, recompute it from X (the forward's own kernel on the same inputs, so
   // bit for bit the value it would have saved) and take dB first, while small0 holds it.
@@ -705,8 +740,9 @@ qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, qlora_stream
 }
 
 size_t qlora_workspace_bytes(int M, int N, int K, int r) {
-  if (M < 1 || N < 64 || K < 64 || !rank_ok(r)) return 0;
-  return ws_layout(M, N, K, r).total;
+  if (M < 1 || N < 64 || K < 64 || r < 1 || r > 128) return 0;
+  if (rank_ok(r)) return ws_layout(M, N, K, r).total;
+  return pad_layout(M, N, K, r).total;
 }
 
 qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
@@ -714,8 +750,28 @@ qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W, const vo
                               void* ws, size_t ws_bytes, qlora_stream_t stream) {
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  return linear_fwd(X, W, A, B, single_group(W->N), M, r, alpha, H, XA_saved, ws, ws_bytes,
-                    static_cast<cudaStream_t>(stream));
+  const float scale = alpha / static_cast<float>(r);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (r < 1 || r > 128 || rank_ok(r))
+    return linear_fwd(X, W, A, B, single_group(W->N), M, r, scale, H, XA_saved, ws, ws_bytes, s);
+  // r not a multiple of 8: the layer runs at r rounded up to 8 on zero-padded copies.  (Every
+  // check the inner call makes on the caller's buffers is made here first, so nothing is
+  // enqueued before an error.)
+  if (!X || !A || !B || !H) return QLORA_ERR_NULL;
+  if (M < 1) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(H)) return QLORA_ERR_ALIGN;
+  const PadLayout P = pad_layout(M, W->N, W->K, r);
+  if (!ws || ws_bytes < P.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int rp = pad8(r);
+  if ((st = pad_factors(A, B, r, rp, W->N, W->K, w8 + P.a, w8 + P.b, s)) != QLORA_OK) return st;
+  void* xap = XA_saved ? w8 + P.xa : nullptr;
+  st = linear_fwd(X, W, w8 + P.a, w8 + P.b, single_group(W->N), M, rp, scale, H, xap, ws, P.inner,
+                  s);
+  if (st != QLORA_OK || !XA_saved) return st;
+  return cuda_status(cudaMemcpy2DAsync(XA_saved, r * 2ull, xap, rp * 2ull, r * 2ull, M,
+                                       cudaMemcpyDeviceToDevice, s));
 }
 
 qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
@@ -724,8 +780,41 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_wei
                               size_t ws_bytes, qlora_stream_t stream) {
   qlora_status st = check_weight(W);
   if (st != QLORA_OK) return st;
-  return linear_bwd(dY, X, W, A, B, XA_saved, single_group(W->N), M, r, alpha, dX, dA, dB, ws,
-                    ws_bytes, static_cast<cudaStream_t>(stream));
+  const float scale = alpha / static_cast<float>(r);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (r < 1 || r > 128 || rank_ok(r))
+    return linear_bwd(dY, X, W, A, B, XA_saved, single_group(W->N), M, r, scale, dX, dA, dB, ws,
+                      ws_bytes, s);
+  // r not a multiple of 8: zero-padded copies of A, B and XA at r rounded up to 8; dA and dB
+  // come back from padded buffers (their extra rows / columns are zero).
+  if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_NULL;
+  if (M < 1) return QLORA_ERR_SHAPE;
+  if (!aligned16(dY) || !aligned16(X) || (dX && !aligned16(dX))) return QLORA_ERR_ALIGN;
+  const PadLayout P = pad_layout(M, W->N, W->K, r);
+  if (!ws || ws_bytes < P.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int rp = pad8(r);
+  if ((st = pad_factors(A, B, r, rp, W->N, W->K, w8 + P.a, w8 + P.b, s)) != QLORA_OK) return st;
+  void* xap = nullptr;
+  if (XA_saved) {
+    xap = w8 + P.xa;
+    if (cudaMemsetAsync(xap, 0, static_cast<size_t>(M) * rp * 2, s) != cudaSuccess ||
+        cudaMemcpy2DAsync(xap, rp * 2ull, XA_saved, r * 2ull, r * 2ull, M,
+                          cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+  }
+  auto* dap = reinterpret_cast<float*>(w8 + P.da);
+  auto* dbp = reinterpret_cast<float*>(w8 + P.db);
+  st = linear_bwd(dY, X, W, w8 + P.a, w8 + P.b, xap, single_group(W->N), M, rp, scale, dX, dap,
+                  dbp, ws, P.inner, s);
+  if (st != QLORA_OK) return st;
+  if (cudaMemcpyAsync(dA, dap, static_cast<size_t>(r) * W->K * 4, cudaMemcpyDeviceToDevice, s) !=
+          cudaSuccess ||
+      cudaMemcpy2DAsync(dB, r * 4ull, dbp, rp * 4ull, r * 4ull, W->N, cudaMemcpyDeviceToDevice,
+                        s) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
 }
 
 size_t qlora_grouped_workspace_bytes(int M, int N, int K, int r, int n_groups) {
@@ -743,7 +832,8 @@ qlora_status qlora_grouped_fwd(const void* X, const qlora_nf4_weight* W, const v
   if (st != QLORA_OK) return st;
   RowGroups g;
   if ((st = make_groups(group_rows, n_groups, W->N, r, &g)) != QLORA_OK) return st;
-  return linear_fwd(X, W, A, B, g, M, r, alpha, H, XA_saved, ws, ws_bytes,
+  return linear_fwd(X, W, A, B, g, M, r, alpha / static_cast<float>(r), H, XA_saved, ws,
+                    ws_bytes,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -756,8 +846,8 @@ qlora_status qlora_grouped_bwd(const void* dY, const void* X, const qlora_nf4_we
   if (st != QLORA_OK) return st;
   RowGroups g;
   if ((st = make_groups(group_rows, n_groups, W->N, r, &g)) != QLORA_OK) return st;
-  return linear_bwd(dY, X, W, A, B, XA_saved, g, M, r, alpha, dX, dA, dB, ws, ws_bytes,
-                    static_cast<cudaStream_t>(stream));
+  return linear_bwd(dY, X, W, A, B, XA_saved, g, M, r, alpha / static_cast<float>(r), dX, dA, dB,
+                    ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_lora_down(const void* in, int M, int C, const void* w, int w_is_r_by_c, int r,

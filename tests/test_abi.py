@@ -72,8 +72,10 @@ def test_validation_codes(lib):
     assert _fwd(lib, W=_w(K=100)) == 2                 # K % 64
     assert _fwd(lib, W=_w(N=96)) == 2                  # N % 64
     assert _fwd(lib, M=0) == 2
-    assert _fwd(lib, r=12) == 2                        # r not a multiple of 8
+    assert _fwd(lib, r=0) == 2                         # r out of [1, 128]
     assert _fwd(lib, r=136) == 2
+    assert _fwd(lib, r=12, ws_bytes=16) == 5           # r = 12 (padded copies): workspace
+    assert _fwd(lib, r=12, X=FAKE + 8) == 3            # ... and alignment, before any work
     assert _fwd(lib, X=FAKE + 8) == 3                  # misaligned
     assert _fwd(lib, ws_bytes=16) == 5                 # workspace too small
     assert _fwd(lib, ws=None) == 5
@@ -83,7 +85,10 @@ def test_validation_codes(lib):
 
 def test_workspace_bytes(lib):
     assert lib.qlora_workspace_bytes(0, 128, 128, 16) == 0
-    assert lib.qlora_workspace_bytes(64, 128, 128, 12) == 0
+    assert lib.qlora_workspace_bytes(64, 128, 128, 129) == 0
+    assert lib.qlora_workspace_bytes(64, 128, 128, 0) == 0
+    # r = 12 runs at 16 on padded copies: more than the rank-16 workspace
+    assert lib.qlora_workspace_bytes(64, 128, 128, 12) > lib.qlora_workspace_bytes(64, 128, 128, 16)
     small = lib.qlora_workspace_bytes(64, 512, 256, 8)
     big = lib.qlora_workspace_bytes(4096, 4096, 4096, 16)
     # 4096^3 runs whole tiles and the rank-r products reduce inside their clusters, so the

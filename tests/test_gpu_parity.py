@@ -156,3 +156,40 @@ def test_recompute_xa_is_bit_identical(M, K, N, r):
     assert torch.equal(H, H2)
     for a, b, k in zip(saved, recomputed, ("dX", "dA", "dB")):
         assert torch.equal(a, b), k
+
+
+@pytest.mark.parametrize(
+    "M,K,N,r,dq",
+    [
+        (64, 256, 512, 1, False),      # r = 1: padded to 8
+        (17, 384, 640, 4, False),      # few-token forward and dX
+        (300, 512, 384, 12, True),     # stream-K, double-quant
+        (2048, 256, 2048, 100, False), # whole tiles, r = 100 -> 104
+        (96, 256, 128, 127, False),    # r = 127 -> 128: two extension chunks
+    ],
+)
+def test_linear_parity_any_rank(M, K, N, r, dq):
+    """Ranks that are not multiples of 8 (the C ABI takes 1 <= r <= 128): the layer runs at r
+    rounded up to 8 on zero-padded copies of A, B and XA, and hands back [M, r] / [r, K] /
+    [N, r] results; same bar against the oracle."""
+    inp, L = parity.make(M, K, N, r, seed=M * 5 + r, dy_std=1.0)
+    got = parity.run_linear(inp, L, dq=dq)
+    assert got["XA"].shape == (M, r) and got["dA"].shape == (r, K) and got["dB"].shape == (N, r)
+    parity.check_linear(inp, L, got, dq=dq)
+
+
+def test_any_rank_recompute_matches_saved():
+    """r = 12 with XA_saved NULL: the backward recomputes X A^T (into the padded copy) and gives
+    the same gradients bit for bit."""
+    inp, L = parity.make(200, 256, 384, 12, seed=77, dy_std=1.0)
+    lin = inp["linears"][0]
+    X, dY, A, B = inp["X"].cuda(), inp["dY"].cuda(), lin["A"].cuda(), lin["B"].cuda()
+    w = linear.nf4_pack(lin["W0"].cuda())
+    H, XA = linear.forward(X, w, A, B, L.alpha)
+    saved = linear.backward(dY, X, w, A, B, XA, L.alpha)
+    H2, none = linear.forward(X, w, A, B, L.alpha, save_xa=False)
+    recomputed = linear.backward(dY, X, w, A, B, None, L.alpha)
+    torch.cuda.synchronize()
+    assert none is None and torch.equal(H, H2)
+    for a, b in zip(saved, recomputed):
+        assert torch.equal(a, b)
