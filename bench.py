@@ -1105,6 +1105,16 @@ def main():
                 line["configs"][name] = measure_config(name, dev, args.config_steps,
                                                        args.warmup, peaks, flush,
                                                        not args.no_clocks)
+            # The headline workload once more with the rank-r down-projections inside the GEMM
+            # launches (qlora_set_rank_fusion; off by default), for the trade-off.
+            prev = abi.qlora_set_rank_fusion(True)
+            try:
+                fused = measure_config(w.name, dev, args.config_steps, args.warmup, peaks, flush,
+                                       not args.no_clocks)
+            finally:
+                abi.qlora_set_rank_fusion(prev)
+            fused["rank_fusion"] = True
+            line["configs"][w.name + "+rank_fusion"] = fused
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
