@@ -912,7 +912,8 @@ def measure_config(name, dev, steps, warmup, peaks, flush, clocks_on):
            "fwd_ms": round(fwd, 5), "bwd_ms": round(bwd, 5), "fwd_bwd_timing": fb_note,
            "stages_ms": {k: round(v, 5) for k, v in means.items()},
            "roofline": roofline(step, per_stage, peaks, name),
-           "graph_launches_per_step": graph.launches_per_step, "steps": steps, "clocks": clocks}
+           "graph_launches_per_step": graph.launches_per_step, "steps": steps, "clocks": clocks,
+           "side_overlap_sms": side_overlap(w)}
     if len(w.linears) == 1 and not w.mlp:
         L = w.linears[0]
         for d, t in (("fwd", fwd), ("bwd", bwd)):
@@ -926,6 +927,27 @@ def measure_config(name, dev, steps, warmup, peaks, flush, clocks_on):
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return rec
+
+
+def side_overlap(w, unpacked=False):
+    """Linears whose timed backward runs dB and dA beside the dX GEMM (qlora_set_side_overlap,
+    the library's current mode), with the SMs they get; the instrumented stage capture calls
+    the stage entry points one after another, so there they run after the GEMM."""
+    if w.ce:
+        return {}
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    groups = [[L] for L in w.linears]
+    if w.grouped:
+        groups = [list(w.linears)]
+    elif w.mlp and not unpacked:
+        groups = [list(w.linears[:2]), [w.linears[2]]]
+    out = {}
+    for g in groups:
+        N, K, R = sum(L.N for L in g), g[0].K, sum(L.r for L in g)
+        s = abi.qlora_backward_side_sms(w.M, N, K, R, sms, -1)
+        if s:
+            out["+".join(L.name for L in g)] = s
+    return out
 
 
 def workload_config(w, unpacked=False):
@@ -1086,7 +1108,10 @@ def main():
                             "qlora_linear_bwd and the SwiGLU glue) with no interior events; "
                             "per-stage times come from a second capture of the same work as its "
                             "stage entry points with an event between every two stages, replayed "
-                            "after the timed region"),
+                            "after the timed region; for the linears in side_overlap_sms the timed "
+                            "backward runs lora_grad_dB / lora_grad_dA beside gemm_dx on that many "
+                            "SMs (the stage capture runs them after it)"),
+            "side_overlap_sms": side_overlap(w, args.unpacked),
             "instrumented_ms_per_step": (round(instrumented_ms, 5) if instrumented_ms else None),
             "roofline": roofline(step, per_stage, peaks, w.name),
             "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

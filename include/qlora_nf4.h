@@ -309,6 +309,32 @@ QLORA_API int qlora_gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int
  * counterpart on the pages (a scheduling choice of this implementation). */
 QLORA_API int qlora_set_rank_fusion(int enable);
 
+/* Host-only, process-wide: where dB and dA of qlora_linear_bwd / qlora_grouped_bwd run when
+ * XA_saved and dX are given and the dX GEMM runs whole tiles.  They can run on a few SMs taken
+ * from the GEMM (qlora_backward_side_sms) while the GEMM runs on the rest, on a stream the library
+ * owns, forked from the caller's stream after dY B and joined back before the call returns
+ * (two events; inside a stream capture they become graph edges, so the captured graph has the
+ * same fork and join).  0: never (dB and dA after the GEMM); 1 (the default): when the
+ * launcher's schedule model expects that to be faster and the shape is one where it measured
+ * faster (qlora_backward_side_sms); 2: always, with the model's best split.
+ * Every output has the same bits in all three modes: the side kernel sums each reduction in the
+ * same step ranges and order as the cluster kernels that run otherwise.  If the side stream
+ * cannot be created the work runs after the GEMM.  Concurrent calls on one device take turns at
+ * the fork/join (a mutex).  Returns the previous mode.  No counterpart on the pages (a
+ * scheduling choice of this implementation). */
+QLORA_API int qlora_set_side_overlap(int mode);
+
+/* Host-only, no GPU needed: the number of SMs (even, 2..32) qlora_linear_bwd /
+ * qlora_grouped_bwd give to dB and dA beside the dX GEMM, for M tokens, W0 [N, K] and
+ * R = n r packed rank columns on a device of sm_count SMs, under side-overlap mode `mode`
+ * (0, 1, 2 as in qlora_set_side_overlap; -1: the current setting); 0 when they run after the
+ * GEMM.  The split minimises the launcher's schedule model of max(GEMM on the other SMs, dY
+ * and X streamed at ~26 GB/s per SM); mode 1 takes it only when that model beats running them
+ * after the GEMM, R <= 32 and dY (2 M N bytes) is at most 48 MiB (larger ranks or operands
+ * measured slower beside the GEMM on a B200); modes 1 and 2 give 0 for stream-K shapes,
+ * M <= 256 and fewer than 64 SMs. */
+QLORA_API int qlora_backward_side_sms(int M, int N, int K, int R, int sm_count, int mode);
+
 /* Number of kernels this library has launched in this process so far (all devices). */
 QLORA_API uint64_t qlora_launch_counter(void);
 

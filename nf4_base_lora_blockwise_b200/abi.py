@@ -42,6 +42,8 @@ EXPORTS = (
     "qlora_gemm_plan",
     "qlora_gemm_rank_fusable",
     "qlora_set_rank_fusion",
+    "qlora_set_side_overlap",
+    "qlora_backward_side_sms",
     "qlora_selftest_bounded_wait",
 )
 
@@ -123,6 +125,8 @@ def _lib():
                                      ctypes.POINTER(_SZ)]),
             "qlora_gemm_rank_fusable": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
             "qlora_set_rank_fusion": (_I, [_I]),
+            "qlora_set_side_overlap": (_I, [_I]),
+            "qlora_backward_side_sms": (_I, [_I, _I, _I, _I, _I, _I]),
             "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
                                        _VP]),
@@ -301,6 +305,19 @@ def qlora_set_rank_fusion(enable):
     """Fuse the rank-r down-projections into the GEMM launches (process-wide); returns the
     previous setting."""
     return bool(_lib().qlora_set_rank_fusion(int(bool(enable))))
+
+
+def qlora_set_side_overlap(mode):
+    """Where dB and dA of the backward run (process-wide): 0 after the dX GEMM, 1 beside it on
+    SMs taken from it when the schedule model expects that to pay (default), 2 beside it
+    whenever the GEMM runs whole tiles.  Returns the previous mode."""
+    return int(_lib().qlora_set_side_overlap(int(mode)))
+
+
+def qlora_backward_side_sms(M, N, K, R, sm_count, mode=-1):
+    """SMs the backward gives to dB / dA beside the dX GEMM for M tokens, W0 [N, K] and R packed
+    rank columns under side-overlap mode `mode` (-1: the current setting); 0: after the GEMM."""
+    return int(_lib().qlora_backward_side_sms(M, N, K, R, sm_count, int(mode)))
 
 
 def qlora_launch_counter():

@@ -11,11 +11,12 @@
 
 namespace qlora {
 
-// Launch `kernel` as a programmatic dependent of the previous kernel on the stream (its CTAs
-// call pdl_wait() before touching global memory), optionally as clusters of `cluster` CTAs.
+// Launch `kernel`, as a programmatic dependent of the previous kernel on the stream when `pdl`
+// (its CTAs call pdl_wait() before touching global memory), optionally as clusters of
+// `cluster` CTAs.
 template <typename... Params, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
-                              cudaStream_t stream, int cluster, Args... args) {
+inline cudaError_t launch_kernel(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, bool pdl, int cluster, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -23,9 +24,11 @@ inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, 
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int n = 0;
-  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[n].val.programmaticStreamSerializationAllowed = 1;
-  ++n;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   if (cluster > 1) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
     attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
@@ -36,6 +39,12 @@ inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, 
   cfg.attrs = attr;
   cfg.numAttrs = static_cast<unsigned>(n);
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, int cluster, Args... args) {
+  return launch_kernel(kernel, grid, block, smem, stream, true, cluster, args...);
 }
 
 // ------------------------------ adapters packed along the output rows -----------------------
@@ -110,6 +119,9 @@ struct GemmArgs {
   float rank_scale;
   unsigned* rank_flags;         // [token tiles], zero before the launch
   unsigned rank_slot;           // bytes of one rank-operand tile (gemm_rank_slot_bytes)
+  // SMs the launch may use (0: all of them); the rest are left to a kernel running beside it.
+  // The tile (bt, nh) must be the one gemm_pick_tile gives for that many SMs.
+  int sm_limit;
 };
 
 struct GemmMaps {
@@ -144,6 +156,13 @@ inline unsigned gemm_rank_slot_bytes(bool trans_w, int rank_cols, int r) {
   if (trans_w) return (r == 16 || r == 32) ? 128u * static_cast<unsigned>(r) : 0u;
   return 128u * static_cast<unsigned>((rank_cols + 15) / 16 * 16);
 }
+// SMs to hand to `side_bytes` of streaming work (dB and dA) that runs beside a whole-tile
+// launch of this shape: the count s (even, 2..32) minimising the schedule model's
+// max(launch on sm_count - s SMs with its tile re-picked, side_bytes at ~26 GB/s per SM),
+// or 0 when running the work after the launch is modelled no slower (always 0 for stream-K
+// shapes and M <= 256).  force: the best s even then.  *us: the modelled duration of both.
+int gemm_side_sms(int M, int rows_w, int steps_per_tile, int sm_count, double side_bytes,
+                  bool force, double* us);
 // Counters the fused down-projection needs in the workspace (zeroed before each launch).
 size_t gemm_rank_flag_bytes(int M);
 // Partial-sum bytes any device (at most kGemmMaxCtas SMs) may need for this shape.
@@ -268,6 +287,16 @@ cudaError_t launch_rank_grad_pair(const RankMaps& m1, const RankPlan& p1, int M,
                                   const RankMaps& m2, const RankPlan& p2, int C2, int ld2,
                                   const RowGroups& g2, float* out2, bool cr2, float scale,
                                   int* err, cudaStream_t stream);
+
+// dB and dA of one backward (the second problem may be absent: m2 == nullptr) on `ctas` CTAs,
+// one per SM, beside another kernel: each CTA walks whole tiles, summing a tile's reduction in
+// the step ranges of the cluster plan p1 / p2, so the results are bit for bit those of
+// launch_rank_grad with the same plans.  Launched as a plain (not programmatic) dependent.
+cudaError_t launch_rank_grad_side(const RankMaps& m1, const RankPlan& p1, int M, int C1, int R1,
+                                  int ld1, const RowGroups& g1, float* out1, bool cr1,
+                                  const RankMaps* m2, const RankPlan* p2, int C2, int R2,
+                                  int ld2, const RowGroups& g2, float* out2, bool cr2,
+                                  float scale, int* err, int ctas, cudaStream_t stream);
 
 // ------------------------------ LM-head cross-entropy ---------------------------------------
 // count = number of labels in [0, V); z [rows, V] bf16 (V % 8 == 0) -> loss [rows] and, with

@@ -83,12 +83,13 @@ struct RankLayout {
 
 __host__ __device__ inline uint32_t partial_pitch(int R) { return static_cast<uint32_t>(R + 4); }
 
-__host__ __device__ inline RankLayout rank_layout(uint32_t small_bytes, int R, int budget) {
+__host__ __device__ inline RankLayout rank_layout(uint32_t small_bytes, int R, int budget,
+                                                  int max_stages = 8) {
   RankLayout L;
   L.small_bytes = (small_bytes + 1023u) & ~1023u;
   L.stage_bytes = kBigTileBytes + L.small_bytes;
   int st = static_cast<int>((static_cast<uint32_t>(budget) - 2048u) / L.stage_bytes);
-  L.stages = st < 2 ? 2 : (st > 8 ? 8 : st);
+  L.stages = st < 2 ? 2 : (st > max_stages ? max_stages : st);
   const uint32_t ring = static_cast<uint32_t>(L.stages) * L.stage_bytes;
   const uint32_t part = static_cast<uint32_t>(kTileRows) * partial_pitch(R) * 4u;
   L.ring_bytes = ring > part ? ring : part;
@@ -517,6 +518,141 @@ __global__ void __launch_bounds__(kRankThreads, NT <= 8 ? 2 : 1)
     }
   }
   cluster_sync_all();
+}
+
+// ------------------------------------------------------------------------------------------
+// grad beside another kernel (rank_grad_loop_kernel): a few CTAs, one per SM, each walking
+// whole tiles -- CTA b of a problem takes tiles b, b + nb, ... -- so the launch occupies only
+// the SMs it is given while a GEMM holds the rest.  A tile's reduction over M runs in the same
+// S contiguous step ranges as the cluster kernel's S CTAs: each range is summed on its own and
+// the range sums are added in range order, exactly the cluster kernel's arithmetic, so both
+// kernels give the same bits.  The ring runs on across tiles (the copies of the next tile
+// overlap the end of this one) and each tile is written straight from the accumulators.
+// ------------------------------------------------------------------------------------------
+template <int NT>
+__global__ void __launch_bounds__(kRankThreads, 1)
+    rank_grad_loop_kernel(const __grid_constant__ CUtensorMap tm_big1,
+                          const __grid_constant__ CUtensorMap tm_small1,
+                          const __grid_constant__ RankArgs a1,
+                          const __grid_constant__ CUtensorMap tm_big2,
+                          const __grid_constant__ CUtensorMap tm_small2,
+                          const __grid_constant__ RankArgs a2, int grid1) {
+  const bool second = static_cast<int>(blockIdx.x) >= grid1;
+  const RankArgs& a = second ? a2 : a1;
+  const CUtensorMap& tm_big = second ? tm_big2 : tm_big1;
+  const CUtensorMap& tm_small = second ? tm_small2 : tm_small1;
+  const int bid = second ? static_cast<int>(blockIdx.x) - grid1 : static_cast<int>(blockIdx.x);
+  const int nb = second ? static_cast<int>(gridDim.x) - grid1 : grid1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + a.ring_bytes);
+  uint64_t* empty = full + a.stages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = (a.C + kTileRows - 1) / kTileRows;
+  const int my_tiles = bid < tiles ? (tiles - bid + nb - 1) / nb : 0;
+  const int n = my_tiles * a.steps;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_wait();  // the previous kernel's outputs are complete
+  pdl_trigger();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_big);
+      tma_prefetch_desc(&tm_small);
+      // The big operand is read once here: evict-first, so the stream does not push out of L2
+      // the activation tiles the GEMM beside this kernel keeps re-reading.
+      const uint64_t once = l2_policy_evict_first();
+      rank_produce(a, ring, full, empty, n, [&](int i, uint8_t* dst, uint64_t* bar) {
+        const int ti = i / a.steps;
+        const int c0 = (bid + ti * nb) * kTileRows;
+        const int m0 = (i - ti * a.steps) * 64;
+        const int j0 = row_group(a.groups, c0) * a.R;
+        tma_load_2d_hint(dst, &tm_big, bar, c0, m0, once);
+        tma_load_2d_hint(dst + 8192, &tm_big, bar, c0 + 64, m0, once);
+        uint8_t* sm = dst + kBigTileBytes;
+        tma_load_2d(sm, &tm_small, bar, j0, m0);
+        if (a.small_blocks == 2) tma_load_2d(sm + 8192, &tm_small, bar, j0 + 64, m0);
+      });
+    }
+    return;
+  }
+  bool failed = false;
+  const int q = lane >> 3, i8 = lane & 7;
+  const int cl = 16 * warp + (q & 1) * 8;
+  const uint32_t cblk = static_cast<uint32_t>(cl >> 6) * 8192u;
+  const uint32_t cch = static_cast<uint32_t>(cl & 63) >> 3;
+  const int r_lo = 16 * warp + (lane >> 2);
+  int i = 0;  // ring position (steps consumed by this CTA)
+  for (int ti = 0; ti < my_tiles; ++ti) {
+    const int c0 = (bid + ti * nb) * kTileRows;
+    float tot[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) tot[t][0] = tot[t][1] = tot[t][2] = tot[t][3] = 0.f;
+    for (int rq = 0; rq < a.split; ++rq) {
+      const int s0 = static_cast<int>(static_cast<long long>(a.steps) * rq / a.split);
+      const int s1 = static_cast<int>(static_cast<long long>(a.steps) * (rq + 1) / a.split);
+      float acc[NT][4];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+      for (int s = s0; s < s1; ++s, ++i) {
+        const int st = i % a.stages;
+        if (!failed)
+          failed = !mbar_wait_warp(full + st, static_cast<uint32_t>(i / a.stages) & 1u,
+                                   kErrWaitFull, a.err, i);
+        if (!failed) {
+          const uint32_t bb = smem_u32(ring + st * a.stage_bytes);
+          const uint32_t sb = bb + kBigTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            uint32_t af[4];
+            const int tok = 16 * kk + i8 + (q >> 1) * 8;
+            ldsm_x4_t(af, bb + cblk + sw128_off(tok, cch));
+            const int l = lane & 15;
+            const int k = 16 * kk + (l & 7) + ((l >> 3) << 3);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              uint32_t b[2];
+              ldsm_x2_t(b, sb + small_off(a, k, static_cast<uint32_t>(t)));
+              mma16816(acc[t], af, b[0], b[1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + st);
+      }
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tot[t][e] += acc[t][e];
+    }
+    if (failed) continue;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int col = t * 8 + (lane & 3) * 2;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = c0 + r_lo + 8 * h;
+        if (c >= a.C) continue;
+        const float v0 = a.scale * tot[t][2 * h], v1 = a.scale * tot[t][2 * h + 1];
+        if (a.out_cr)  // out [C, R]
+          *reinterpret_cast<float2*>(a.out + static_cast<long long>(c) * a.R + col) =
+              make_float2(v0, v1);
+        else {  // out [R, C]
+          a.out[static_cast<long long>(col) * a.C + c] = v0;
+          a.out[static_cast<long long>(col + 1) * a.C + c] = v1;
+        }
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -955,6 +1091,91 @@ cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int
   const RankArgs a = grad_args(p, M, C, R, ld_small, groups, scale, out, out_cr, err, &ok);
   if (!ok) return cudaErrorInvalidValue;
   return launch_grad_any(R, maps, a, p.grid, maps, a, 0, p.split, p.smem, stream);
+}
+
+namespace {
+
+// The side kernel has an SM to itself: a deeper ring than the cluster kernel's two CTAs per SM.
+constexpr int kSideBudget = 220 * 1024;
+constexpr int kSideMaxStages = 12;
+
+RankArgs side_args(const RankPlan& p, int M, int C, int R, int ld_small, const RowGroups& groups,
+                   float scale, float* out, bool out_cr, int* err, bool* ok, size_t* smem) {
+  RankArgs a = grad_args(p, M, C, R, ld_small, groups, scale, out, out_cr, err, ok);
+  const RankLayout L = rank_layout(p.small.bytes, R, kSideBudget, kSideMaxStages);
+  a.stages = L.stages;
+  a.stage_bytes = L.stage_bytes;
+  a.small_bytes = L.small_bytes;
+  a.ring_bytes = L.ring_bytes;
+  *ok = *ok && L.small_bytes == p.small.bytes;
+  *smem = L.smem;
+  return a;
+}
+
+template <int NT>
+cudaError_t launch_side_nt(const RankMaps& m1, const RankArgs& a1, int grid1, const RankMaps& m2,
+                           const RankArgs& a2, int grid2, size_t smem, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(rank_grad_loop_kernel<NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_kernel(rank_grad_loop_kernel<NT>, dim3(static_cast<unsigned>(grid1 + grid2)),
+                       dim3(kRankThreads), smem, stream, false, 1, m1.big, m1.small, a1, m2.big,
+                       m2.small, a2, grid1);
+}
+
+cudaError_t launch_side_any(int R, const RankMaps& m1, const RankArgs& a1, int grid1,
+                            const RankMaps& m2, const RankArgs& a2, int grid2, size_t smem,
+                            cudaStream_t stream) {
+  switch (R / 8) {
+#define QLORA_RANK_SIDE_CASE(NTV) \
+  case NTV:                       \
+    return launch_side_nt<NTV>(m1, a1, grid1, m2, a2, grid2, smem, stream);
+    QLORA_RANK_SIDE_CASE(1)
+    QLORA_RANK_SIDE_CASE(2)
+    QLORA_RANK_SIDE_CASE(3)
+    QLORA_RANK_SIDE_CASE(4)
+    QLORA_RANK_SIDE_CASE(5)
+    QLORA_RANK_SIDE_CASE(6)
+    QLORA_RANK_SIDE_CASE(7)
+    QLORA_RANK_SIDE_CASE(8)
+    QLORA_RANK_SIDE_CASE(9)
+    QLORA_RANK_SIDE_CASE(10)
+    QLORA_RANK_SIDE_CASE(11)
+    QLORA_RANK_SIDE_CASE(12)
+    QLORA_RANK_SIDE_CASE(13)
+    QLORA_RANK_SIDE_CASE(14)
+    QLORA_RANK_SIDE_CASE(15)
+    QLORA_RANK_SIDE_CASE(16)
+#undef QLORA_RANK_SIDE_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rank_grad_side(const RankMaps& m1, const RankPlan& p1, int M, int C1, int R1,
+                                  int ld1, const RowGroups& g1, float* out1, bool cr1,
+                                  const RankMaps* m2, const RankPlan* p2, int C2, int R2,
+                                  int ld2, const RowGroups& g2, float* out2, bool cr2,
+                                  float scale, int* err, int ctas, cudaStream_t stream) {
+  bool ok = true;
+  size_t smem1 = 0, smem2 = 0;
+  const RankArgs a1 = side_args(p1, M, C1, R1, ld1, g1, scale, out1, cr1, err, &ok, &smem1);
+  if (!ok) return cudaErrorInvalidValue;
+  if (!m2) {
+    if (ctas < 1) return cudaErrorInvalidValue;
+    return launch_side_any(R1, m1, a1, ctas, m1, a1, 0, smem1, stream);
+  }
+  // Two problems in one launch need one instance (same rank); CTAs split by their bytes.
+  if (!p2 || R2 != R1 || ctas < 2) return cudaErrorInvalidValue;
+  const RankArgs a2 = side_args(*p2, M, C2, R2, ld2, g2, scale, out2, cr2, err, &ok, &smem2);
+  if (!ok) return cudaErrorInvalidValue;
+  int grid1 = static_cast<int>((static_cast<long long>(ctas) * C1 + (C1 + C2) / 2) / (C1 + C2));
+  grid1 = grid1 < 1 ? 1 : (grid1 > ctas - 1 ? ctas - 1 : grid1);
+  return launch_side_any(R1, m1, a1, grid1, *m2, a2, ctas - grid1,
+                         smem1 > smem2 ? smem1 : smem2, stream);
 }
 
 bool rank_grad_pair_ok(const RankPlan& p1, int R1, const RankPlan& p2, int R2) {

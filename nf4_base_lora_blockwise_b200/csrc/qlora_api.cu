@@ -309,6 +309,7 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& gro
   a.rank_scale = 0.f;
   a.rank_flags = nullptr;
   a.rank_slot = 0;
+  a.sm_limit = 0;
   return a;
 }
 
@@ -352,6 +353,41 @@ std::atomic<uint64_t> g_launches{0};
 // measured slower than the separate launches).
 std::atomic<int> g_rank_fusion{0};
 void count(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------------------------------------
+// Work beside the dX GEMM.  When the GEMM runs whole tiles, dB and dA can run on a few SMs
+// taken from it (gemm_side_sms) while it runs on the rest, on a stream this library
+// owns, forked from and joined back to the caller's stream with events (inside a stream
+// capture the fork and the join become graph edges).  qlora_set_side_overlap: 0 never,
+// 1 (default) when the schedule model expects it to be faster than running them after the
+// GEMM, 2 always (with the model's best split) when the GEMM runs whole tiles.
+// ---------------------------------------------------------------------------------------------
+struct SideExec {
+  std::mutex mu;  // one fork/join sequence at a time per device (the events are shared)
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ready = false, broken = false;
+};
+SideExec g_side[64];
+constexpr double kSideMaxActBytes = 48.0 * 1024 * 1024;  // dY bytes the GEMM keeps in L2
+std::mutex g_side_init_mu;
+std::atomic<int> g_side_overlap{1};
+SideExec* side_exec(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_side_init_mu);
+  SideExec& se = g_side[dev];
+  if (!se.ready && !se.broken) {
+    if (cudaStreamCreateWithFlags(&se.stream, cudaStreamNonBlocking) == cudaSuccess &&
+        cudaEventCreateWithFlags(&se.fork, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&se.join, cudaEventDisableTiming) == cudaSuccess)
+      se.ready = true;
+    else {
+      se.broken = true;
+      (void)cudaGetLastError();
+    }
+  }
+  return se.ready ? &se : nullptr;
+}
 
 // ---------------------------------------------------------------------------------------------
 // Stage bodies (validated by their callers).
@@ -401,7 +437,7 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
                      const void* ext_act, int M, int r, const RowGroups& groups, void* out,
                      int* err, void* partial, size_t partial_bytes, cudaStream_t s,
-                     const RankFusion* fuse = nullptr) {
+                     const RankFusion* fuse = nullptr, int sm_limit = 0) {
   if (!trans && M <= kGemvMaxTokens && partial) {
     // Few tokens: the register-direct kernel streams the weight without the tcgen05 rings.
     const cudaError_t e = launch_nf4_gemv_fwd(
@@ -440,11 +476,14 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
       return QLORA_OK;
     }
   }
+  if (sm_limit > 0 && sm_limit < sms && !fuse) sms = sm_limit;
+  else sm_limit = 0;
   GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms, fuse != nullptr);
   a.partial = static_cast<float*>(partial);
+  a.sm_limit = sm_limit;
   GemmMaps maps;
 #ifdef QLORA_CTA_PAIRS
-  if (!fuse && gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
+  if (!fuse && !sm_limit && gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
     // Enough whole tiles for every SM pair: M = 256 MMAs over CTA pairs (each CTA loads half of
     // every activation block, so the tensor maps' boxes are bt / 2 tokens high).
     const GemmTile t2 = gemm2_pick_tile(M, a.rows_w, a.kt + a.n_ext, sms);
@@ -515,6 +554,73 @@ qlora_status do_lora_grad(const void* big, int M, int C, const void* small, int 
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   count(1);
   return QLORA_OK;
+}
+
+// SMs the dX GEMM of a backward gives to dB and dA (0: they run after it), for W [N, K] with
+// n r = R rank columns, under side-overlap mode `mode`.
+int side_sms(int M, int N, int K, int R, int sms, int mode) {
+  if (mode == 0 || M < 1 || N < 64 || K < 64 || R < 1) return 0;
+  // Measured on a B200, where the model alone is too hopeful: with n r > 32 the side kernel is
+  // bound by its mma.sync work, not its stream (proj_70b_dq, r = 64: 5.25 -> 8.34 ms per
+  // step), and when dY (which the GEMM re-reads once per row tile) is too big to stay in L2 the
+  // side stream's DRAM traffic costs the GEMM more than the side saves (mlp_8b +1.5 %, 16384
+  // tokens +2.4 %; q_proj, dY 32 MiB: 0.349 -> 0.327 ms).
+  if (mode == 1 && (R > 32 || 2.0 * M * N > kSideMaxActBytes)) return 0;
+  double us = 0.0;
+  // dB streams dY [M, N], dA streams X [M, K].
+  const double bytes = 2.0 * M * (static_cast<double>(N) + K);
+  return gemm_side_sms(M, K, N / 64 + ext_steps(R), sms, bytes, mode == 2, &us);
+}
+
+// dX = dY deq(W0) + (s dYB) A on all but `spare` SMs, with dB_g = s dY_g^T XA_g and
+// dA = s dYB^T X on those `spare` SMs at the same time (a side stream forked after dYB).  The
+// side kernels sum in the cluster kernels' order, so every output has the bits of the serial
+// path.  *done = false when the side stream is unavailable (nothing enqueued).
+qlora_status gemm_with_side_grads(const void* dY, const void* X, const void* XA, const void* dYB,
+                                  const void* sdYB, const qlora_nf4_weight* W, const void* A,
+                                  const RowGroups& g, int M, int r, float scale, void* dX,
+                                  float* dA, float* dB, int* err, void* scratch,
+                                  size_t scratch_bytes, cudaStream_t s, int dev, int sms,
+                                  int spare, bool* done) {
+  *done = false;
+  SideExec* se = side_exec(dev);
+  if (!se) return QLORA_OK;
+  const int R = g.n * r, N = W->N, K = W->K;
+  const RankPlan pB = rank_grad_plan(M, N, r, sms);
+  const RankPlan pA = rank_grad_plan(M, K, R, sms);
+  RankMaps mB, mA;
+  qlora_status st = grad_maps(&mB, pB, dY, M, N, XA, R);
+  if (st != QLORA_OK) return st;
+  if ((st = grad_maps(&mA, pA, X, M, K, dYB, R)) != QLORA_OK) return st;
+  std::lock_guard<std::mutex> lk(se->mu);
+  if (cudaEventRecord(se->fork, s) != cudaSuccess ||
+      cudaStreamWaitEvent(se->stream, se->fork, 0) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  *done = true;
+  cudaError_t e;
+  if (r == R) {  // one launch: both problems share the kernel instance
+    e = launch_rank_grad_side(mB, pB, M, N, r, R, g, dB, true, &mA, &pA, K, R, R,
+                              single_group(K), dA, false, scale, err, spare, se->stream);
+    if (e == cudaSuccess) count(1);
+  } else {
+    e = launch_rank_grad_side(mB, pB, M, N, r, R, g, dB, true, nullptr, nullptr, 0, 0, 0, g,
+                              nullptr, false, scale, err, spare, se->stream);
+    if (e == cudaSuccess) {
+      count(1);
+      e = launch_rank_grad_side(mA, pA, M, K, R, R, single_group(K), dA, false, nullptr, nullptr,
+                                0, 0, 0, g, nullptr, false, scale, err, spare, se->stream);
+      if (e == cudaSuccess) count(1);
+    }
+  }
+  st = e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  if (st == QLORA_OK)
+    st = do_gemm(dY, W, true, A, sdYB, M, R, single_group(K), dX, err, scratch, scratch_bytes, s,
+                 nullptr, sms - spare);
+  // Join whatever was enqueued, so the caller's stream (or capture) waits for the side work.
+  if (cudaEventRecord(se->join, se->stream) != cudaSuccess ||
+      cudaStreamWaitEvent(s, se->join, 0) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return st;
 }
 
 // dB = s dY^T XA (per adapter) and dA = s dYB^T X of one backward, in one launch when their
@@ -640,6 +746,16 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
     st = do_lora_down(dY, M, W->N, B, false, R, g, scale, dyb, sdyb, err, s, scratch,
                       L.scratch_bytes);
     if (st != QLORA_OK) return st;
+    const int spare = (dX && XA_saved)
+                          ? side_sms(M, W->N, W->K, R, sms,
+                                     g_side_overlap.load(std::memory_order_relaxed))
+                          : 0;
+    if (spare > 0) {
+      bool done = false;
+      st = gemm_with_side_grads(dY, X, XA_saved, dyb, sdyb, W, A, g, M, r, scale, dX, dA, dB, err,
+                                scratch, L.scratch_bytes, s, dev, sms, spare, &done);
+      if (st != QLORA_OK || done) return st;
+    }
     if (dX && (st = do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
                             L.scratch_bytes, s)) != QLORA_OK)
       return st;
@@ -942,6 +1058,16 @@ qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count
 
 int qlora_set_rank_fusion(int enable) {
   return g_rank_fusion.exchange(enable ? 1 : 0, std::memory_order_relaxed);
+}
+
+int qlora_set_side_overlap(int mode) {
+  return g_side_overlap.exchange(mode < 0 ? 0 : (mode > 2 ? 2 : mode), std::memory_order_relaxed);
+}
+
+int qlora_backward_side_sms(int M, int N, int K, int R, int sm_count, int mode) {
+  if (sm_count < 1) return 0;
+  if (mode < 0) mode = qlora::g_side_overlap.load(std::memory_order_relaxed);
+  return qlora::side_sms(M, N, K, R, sm_count, mode > 2 ? 2 : mode);
 }
 
 int qlora_gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int rank_cols,

@@ -576,8 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (win.has) {
           bool got = true;
           if (lane == 0)
-            got = mbar_wait_sleepy(rank_full, static_cast<uint32_t>(nwin_done) & 1u, kErrWaitAcc,
-                                   err, seg);
+            got = mbar_wait(rank_full, static_cast<uint32_t>(nwin_done) & 1u, kErrWaitAcc, err,
+                            seg);
           if (!__shfl_sync(0xFFFFFFFFu, got, 0)) break;
           __syncwarp();
           tc_fence_after();
@@ -621,8 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int use = P.nacc == 2 ? (seg >> 1) : seg;
       bool got = true;
       if (lane == 0)
-        got = mbar_wait_sleepy(accfull + ab, static_cast<uint32_t>(use) & 1u, kErrWaitAcc, err,
-                               seg);
+        got = mbar_wait(accfull + ab, static_cast<uint32_t>(use) & 1u, kErrWaitAcc, err, seg);
       if (!__shfl_sync(0xFFFFFFFFu, got, 0)) break;
       __syncwarp();  // lane 0's acquire, passed on to the warp
       tc_fence_after();
@@ -880,6 +879,14 @@ namespace {
 // the commit; and when one accumulator fills TMEM (more than 256 token columns) the epilogue's
 // drain, ~37 cycles per token column, is exposed at every tile switch instead of overlapping
 // the next tile's mainloop.
+// Measured on a B200 (4096-token q_proj backward): one CTA of the side kernel, alone on its SM
+// with a 12-stage TMA ring, streams ~26 GB/s while the GEMM holds the other SMs (the SM's
+// outstanding-miss limit, not HBM); the cluster kernels on the whole GPU ~2.2 TB/s.
+constexpr double kSideBytesPerUsPerSm = 26e3;
+constexpr double kSerialBytesPerUs = 2.2e6;
+constexpr double kClockMhz = 1965.0;  // cycles of the model per microsecond
+constexpr int kSideMaxSms = 32;
+
 double whole_tile_cycles(int M, int rows_w, int steps, int G, int bt, int nh) {
   const int tt = bt * nh;
   const long long tiles =
@@ -1006,6 +1013,37 @@ bool gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int 
   return true;
 }
 
+int gemm_side_sms(int M, int rows_w, int steps_per_tile, int sm_count, double side_bytes,
+                  bool force, double* us) {
+  const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
+  *us = 0.0;
+  if (M <= 256 || G < 64 || side_bytes <= 0.0 ||
+      gemm_schedule(M, rows_w, steps_per_tile, G).streamk)
+    return 0;
+  const GemmTile t0 = gemm_pick_tile(M, rows_w, steps_per_tile, G);
+  const double alone = whole_tile_cycles(M, rows_w, steps_per_tile, G, t0.bt, t0.nh) / kClockMhz;
+  int best = 0;
+  double best_us = 0.0;
+  for (int spare = 2; spare <= kSideMaxSms; spare += 2) {
+    const int g = G - spare;
+    if (gemm_schedule(M, rows_w, steps_per_tile, g).streamk) break;
+    const GemmTile t = gemm_pick_tile(M, rows_w, steps_per_tile, g);
+    const double gemm = whole_tile_cycles(M, rows_w, steps_per_tile, g, t.bt, t.nh) / kClockMhz;
+    const double side = side_bytes / (spare * kSideBytesPerUsPerSm);
+    const double both = gemm > side ? gemm : side;
+    if (best == 0 || both < best_us) {
+      best = spare;
+      best_us = both;
+    }
+  }
+  // After the launch instead: the cluster kernels stream at ~2.2 TB/s on the whole GPU, plus
+  // ~5 us for their launch and tail.
+  const double serial = alone + side_bytes / kSerialBytesPerUs + 5.0;
+  if (best == 0 || (!force && best_us > 0.97 * serial)) return 0;
+  *us = best_us;
+  return best;
+}
+
 size_t gemm_rank_flag_bytes(int M) { return 4 * (static_cast<size_t>(M) / 128 + 2); }
 
 size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile) {
@@ -1018,6 +1056,10 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
   int sms = 0;
   cudaError_t e = gemm_device_sms(&sms);
   if (e != cudaSuccess) return e;
+  if (args.sm_limit > 0 && args.sm_limit < sms) {
+    if (args.fuse) return cudaErrorInvalidValue;  // its windows assume every SM's first wave
+    sms = args.sm_limit;
+  }
   // The caller's tile (TMA boxes, smem plan) must be the one the schedule assumes.
   const GemmTile tl = gemm_pick_tile(args.M, args.rows_w, args.kt + args.n_ext, sms, args.fuse);
   if (tl.bt != args.bt || tl.nh != args.nh) return cudaErrorInvalidValue;

@@ -278,3 +278,45 @@ def test_rank_fusion_decision_and_coverage():
     # The headline layer fuses in both directions: 4096 tokens, q_proj 4096 -> 4096, r = 16.
     assert abi.qlora_gemm_rank_fusable(4096, 4096, 64 + 1, 148, 16, 16, False) == 240
     assert abi.qlora_gemm_rank_fusable(4096, 4096, 64 + 1, 148, 16, 16, True) == 240
+
+
+def test_backward_side_sms():
+    """SMs the backward gives to dB / dA beside the dX GEMM (qlora_backward_side_sms, host
+    only): an even count in [2, 32] or 0; 0 in mode 0, for stream-K shapes and M <= 256; mode 1
+    gives either 0 or mode 2's split, and 0 for R > 32 or dY above 48 MiB; with s SMs given
+    away the GEMM's plan on the rest is still whole tiles on every remaining SM; and the q_proj
+    backward (4096 tokens, 4096 x 4096, r 16) gives 20 of 148 SMs, so the GEMM runs its 256
+    tiles of 512 tokens two per CTA on 128 CTAs."""
+    from nf4_base_lora_blockwise_b200 import abi
+    assert abi.qlora_backward_side_sms(4096, 4096, 4096, 16, 148, 1) == 20
+    p = abi.qlora_gemm_plan(4096, 4096, 64 + 1, 128)
+    assert (p["bt"] * p["nh"], p["streamk"], p["grid"]) == (512, 0, 128)
+    assert abi.qlora_backward_side_sms(4096, 4096, 4096, 16, 148, 0) == 0
+    assert abi.qlora_backward_side_sms(4096, 4096, 4096, 64, 148, 1) == 0   # R > 32
+    assert abi.qlora_backward_side_sms(4096, 4096, 4096, 64, 148, 2) > 0
+    assert abi.qlora_backward_side_sms(8192, 4096, 14336, 16, 148, 1) == 0  # dY 64 MiB
+    assert abi.qlora_backward_side_sms(256, 4096, 4096, 16, 148, 2) == 0
+    assert abi.qlora_backward_side_sms(4096, 4096, 4096, 16, 32, 2) == 0    # too few SMs
+    rng = random.Random(23)
+    seen = 0
+    for _ in range(300):
+        M = rng.choice([128, 256, 300, 1024, 2048, 3000, 4096, 8192, 16384])
+        N, K = 64 * rng.randint(1, 460), 128 * rng.randint(1, 230)
+        R = rng.choice([8, 16, 32, 64])
+        sms = rng.choice([132, 148, 160])
+        s = abi.qlora_backward_side_sms(M, N, K, R, sms, 2)
+        assert s == 0 or (s % 2 == 0 and 2 <= s <= 32)
+        s1 = abi.qlora_backward_side_sms(M, N, K, R, sms, 1)
+        assert s1 in (0, s)
+        if R > 32 or 2 * M * N > 48 * 2**20:
+            assert s1 == 0
+        steps = N // 64 + ((R + 15) // 16 * 16 + 63) // 64
+        full = abi.qlora_gemm_plan(M, K, steps, sms)
+        if M <= 256 or full["streamk"]:
+            assert s == 0
+        if s == 0:
+            continue
+        seen += 1
+        part = abi.qlora_gemm_plan(M, K, steps, sms - s)
+        assert part["streamk"] == 0 and part["grid"] == sms - s
+    assert seen > 20
