@@ -38,7 +38,6 @@ constexpr int kGvWarps = 8;
 constexpr int kGvThreads = 32 * kGvWarps;
 constexpr int kGvRows = 16 * kGvWarps;  // weight rows per tile
 constexpr int kGvBlk = 4;               // 64-blocks per pipeline stage
-constexpr int kGvStages = 3;
 
 __device__ __forceinline__ uint32_t gv_saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
