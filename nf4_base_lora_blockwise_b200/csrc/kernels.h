@@ -198,6 +198,19 @@ cudaError_t launch_qlora_gemm2(bool trans_w, const GemmMaps& maps, const GemmArg
 // h[M, N] = X[M, K] . deq(W0)^T + ext_act[M, g(n), r] . ext_w[N, r]^T for M <= 32 (g(n) the
 // adapter of row n): stream-K over (128-row tile, 64-block) units with fp32 partial slots and
 // a fixed-order finalize.
+// The rank-r down-projection of a few-token layer left as fp32 partials for its consumer to
+// add (rank_down_plan's second-level split, gsplit > 1, one row tile: M <= 128): the consumer
+// sums part[g][m][j] over g in order -- rank_down_finalize's arithmetic, so the same bits --
+// and uses bf16(scale * sum) as the LoRA term's rank-r activation.
+struct RankFold {
+  const float* part;     // [gsplit][128][R] fp32
+  int gsplit;
+  int R;                 // n r columns
+  float scale;           // alpha / r
+  __nv_bfloat16* saved;  // [M, R]: bf16(sum), written by the consumer (nullable)
+};
+constexpr int kFoldMaxR = 128;
+
 struct GemvPlan {
   int tt;                 // token tiles of 8
   long long units;
@@ -222,7 +235,25 @@ cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_
                                  const uint8_t* absmax_q8, const float* absmax_scale, int dq,
                                  const __nv_bfloat16* sdyb, const __nv_bfloat16* A, int R,
                                  __nv_bfloat16* dx, float* part, size_t part_bytes,
-                                 const Codebook& cb, int* err, cudaStream_t stream);
+                                 const Codebook& cb, int* err, cudaStream_t stream,
+                                 bool finalize = true);
+// The few-token layer backward's last launch, after the main dX kernel ran without its
+// finalize (or alone, with dx null): dY B summed from the down-projection's partials (fold),
+// dX from the main kernel's split partials (xpart, splits) plus (s dYB) A, dA = s dYB^T X and
+// dB_g = s dY_g^T XA_g, each summed over the M <= 32 tokens in order in fp32.
+struct FewTokTail {
+  RankFold fold;             // dY B partials (fold.R = n r; fold.saved unused)
+  const __nv_bfloat16* X;    // [M, K]
+  const __nv_bfloat16* dY;   // [M, N]
+  const __nv_bfloat16* XA;   // [M, n r]
+  const __nv_bfloat16* A;    // [n r, K]
+  RowGroups groups;          // adapters along W0's rows; r columns of XA each
+  int r;
+  float* dA;                 // [n r, K]
+  float* dB;                 // [N, r]
+};
+cudaError_t launch_fewtok_bwd_tail(const FewTokTail& tail, const float* xpart, int splits, int M,
+                                   int N, int K, __nv_bfloat16* dx, cudaStream_t stream);
 constexpr int kGemvMaxTokens = 32;
 GemvPlan gemv_plan(int M, int N, int K, int sm_count);
 cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const float* absmax,
@@ -230,7 +261,8 @@ cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const 
                                 int N, int K, const __nv_bfloat16* ext_act,
                                 const __nv_bfloat16* ext_w, int r, const RowGroups& groups,
                                 __nv_bfloat16* out, float* partial, size_t partial_floats,
-                                const Codebook& cb, cudaStream_t stream);
+                                const Codebook& cb, cudaStream_t stream,
+                                const RankFold* fold = nullptr);
 
 // ------------------------------ rank-r products (TMA ring, mma.sync, cluster reduction) ------
 // down: out[m, j] = sum_c in[m, c] Wl(j, c), Wl = A [R, C] (w_rc) or B [C, rg] (block-diagonal
@@ -271,11 +303,13 @@ struct RankMaps {
 RankPlan rank_down_plan(int M, int C, int R, int rg, bool w_rc, int sm_count,
                         size_t scratch_bytes = 0);
 RankPlan rank_grad_plan(int M, int C, int R, int sm_count);
-// scratch: p.part_bytes of workspace when p.gsplit > 1 (then a finalize kernel follows).
+// scratch: p.part_bytes of workspace when p.gsplit > 1 (then a finalize kernel follows, unless
+// !finalize: the partials' consumer adds them itself, see RankFold).
 cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int C, int R, int rg,
                              bool w_rc, const RowGroups& groups, float scale,
                              __nv_bfloat16* saved, __nv_bfloat16* scaled, int* err,
-                             cudaStream_t stream, float* scratch = nullptr);
+                             cudaStream_t stream, float* scratch = nullptr,
+                             bool finalize = true);
 cudaError_t launch_rank_grad(const RankMaps& maps, const RankPlan& p, int M, int C, int R,
                              int ld_small, const RowGroups& groups, float scale, float* out,
                              bool out_cr, int* err, cudaStream_t stream);

@@ -924,7 +924,7 @@ cudaError_t launch_down_cluster(const RankMaps& maps, const RankPlan& p, int R, 
 cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int C, int R, int rg,
                              bool w_rc, const RowGroups& groups, float scale,
                              __nv_bfloat16* saved, __nv_bfloat16* scaled, int* err,
-                             cudaStream_t stream, float* scratch) {
+                             cudaStream_t stream, float* scratch, bool finalize) {
   RankArgs a = {};
   a.gsplit = 1;
   a.gpart = nullptr;
@@ -978,7 +978,7 @@ cudaError_t launch_rank_down(const RankMaps& maps, const RankPlan& p, int M, int
     a.gsplit = p.gsplit;
     a.gpart = scratch;
     const cudaError_t e = launch_down_cluster(maps, p, R, w_rc, a, stream);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || !finalize) return e;
     const int items = M * (R / 4);
     return launch_pdl(rank_down_finalize, dim3((items + 255) / 256), dim3(256), 0, stream, 1, a);
   }

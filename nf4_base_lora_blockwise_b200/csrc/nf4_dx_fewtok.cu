@@ -264,7 +264,156 @@ __global__ void __launch_bounds__(128) nf4_dx_fewtok_finalize(const FtArgs a,
       __floats2bfloat162_rn(v0 + l0, v1 + l1);
 }
 
+// The few-token backward's last kernel: every block first sums dY B for all tokens from the
+// down-projection's partials (in split order, rounded to bf16 -- rank_down_finalize's
+// arithmetic) or loads XA, then takes one job by block range:
+//   [0, nx)          dX pairs, as nf4_dx_fewtok_finalize with s dYB from shared memory
+//   [nx, nx + na)    dA[j, k] = s sum_m dYB[m, j] X[m, k]        (two columns k per thread)
+//   [nx + na, ...)   dB[n, j] = s sum_m dY[m, n] XA[m, g(n) r + j]  (eight columns j per thread)
+// The sums over the M <= 32 tokens run in token order in fp32.
+struct FtTail {
+  const float* dpart;  // dY B partials [gsplit][128][R]
+  int gsplit;
+  int R, r;            // n r packed columns; r per adapter
+  float scale;
+  const float* xpart;  // dX split partials [splits][M][K] (nx == 0: none)
+  int splits;
+  int M, N, K;
+  const __nv_bfloat16* X;
+  const __nv_bfloat16* dY;
+  const __nv_bfloat16* XA;
+  const __nv_bfloat16* A;
+  RowGroups groups;
+  __nv_bfloat16* dx;
+  float* dA;
+  float* dB;
+  int nx, na;
+};
+
+__global__ void __launch_bounds__(128) nf4_fewtok_bwd_tail(const FtTail t) {
+  __shared__ float s_rank[kFewTokDxMaxTokens * kFoldMaxR];
+  pdl_wait();  // the partials are complete
+  pdl_trigger();
+  const int b = static_cast<int>(blockIdx.x);
+  const int job = b < t.nx ? 0 : (b < t.nx + t.na ? 1 : 2);
+  const int mr = t.M * t.R;
+  if (job < 2) {  // job 0: s dYB (the LoRA term of dX); job 1: dYB
+    for (int i = threadIdx.x; i < mr; i += blockDim.x) {
+      const int m = i / t.R, j = i - m * t.R;
+      float v = 0.f;
+      for (int g = 0; g < t.gsplit; ++g)
+        v += __ldg(t.dpart + (static_cast<long long>(g) * 128 + m) * t.R + j);
+      s_rank[i] = __bfloat162float(__float2bfloat16_rn(job == 0 ? t.scale * v : v));
+    }
+  } else {
+    for (int i = threadIdx.x; i < mr; i += blockDim.x) s_rank[i] = __bfloat162float(t.XA[i]);
+  }
+  __syncthreads();
+  const long long idx = static_cast<long long>(job == 0 ? b : (job == 1 ? b - t.nx
+                                                                          : b - t.nx - t.na)) *
+                            blockDim.x + threadIdx.x;
+  if (job == 0) {
+    if (idx >= static_cast<long long>(t.M) * (t.K / 2)) return;
+    const int m = static_cast<int>(idx / (t.K / 2));
+    const int k = static_cast<int>(idx - static_cast<long long>(m) * (t.K / 2)) * 2;
+    float v0 = 0.f, v1 = 0.f;
+    const long long stride = static_cast<long long>(t.M) * t.K;
+    const float* pp = t.xpart + static_cast<long long>(m) * t.K + k;
+    int s = 0;
+    for (; s + 8 <= t.splits; s += 8) {  // eight loads in flight, added in split order
+      float2 p[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        p[j] = __ldg(reinterpret_cast<const float2*>(pp + (s + j) * stride));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v0 += p[j].x;
+        v1 += p[j].y;
+      }
+    }
+    for (; s < t.splits; ++s) {
+      const float2 p = __ldg(reinterpret_cast<const float2*>(pp + s * stride));
+      v0 += p.x;
+      v1 += p.y;
+    }
+    float l0 = 0.f, l1 = 0.f;
+    const float* e = s_rank + m * t.R;
+    for (int j = 0; j < t.R; ++j) {
+      const __nv_bfloat162 w =
+          *reinterpret_cast<const __nv_bfloat162*>(t.A + static_cast<long long>(j) * t.K + k);
+      l0 += e[j] * __low2float(w);
+      l1 += e[j] * __high2float(w);
+    }
+    *reinterpret_cast<__nv_bfloat162*>(t.dx + static_cast<long long>(m) * t.K + k) =
+        __floats2bfloat162_rn(v0 + l0, v1 + l1);
+  } else if (job == 1) {
+    if (idx >= static_cast<long long>(t.R) * (t.K / 2)) return;
+    const int j = static_cast<int>(idx / (t.K / 2));
+    const int k = static_cast<int>(idx - static_cast<long long>(j) * (t.K / 2)) * 2;
+    float a0 = 0.f, a1 = 0.f;
+    for (int m = 0; m < t.M; ++m) {
+      const float d = s_rank[m * t.R + j];
+      const float2 x = __bfloat1622float2(
+          *reinterpret_cast<const __nv_bfloat162*>(t.X + static_cast<long long>(m) * t.K + k));
+      a0 = fmaf(d, x.x, a0);
+      a1 = fmaf(d, x.y, a1);
+    }
+    *reinterpret_cast<float2*>(t.dA + static_cast<long long>(j) * t.K + k) =
+        make_float2(t.scale * a0, t.scale * a1);
+  } else {
+    const int groups8 = t.r / 8;
+    if (idx >= static_cast<long long>(t.N) * groups8) return;
+    const int n = static_cast<int>(idx / groups8);
+    const int j0 = static_cast<int>(idx - static_cast<long long>(n) * groups8) * 8;
+    const float* xa = s_rank + row_group(t.groups, n) * t.r + j0;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int m = 0; m < t.M; ++m) {
+      const float d = __bfloat162float(t.dY[static_cast<long long>(m) * t.N + n]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(d, xa[m * t.R + i], acc[i]);
+    }
+    float4* o = reinterpret_cast<float4*>(t.dB + static_cast<long long>(n) * t.r + j0);
+    o[0] = make_float4(t.scale * acc[0], t.scale * acc[1], t.scale * acc[2], t.scale * acc[3]);
+    o[1] = make_float4(t.scale * acc[4], t.scale * acc[5], t.scale * acc[6], t.scale * acc[7]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_fewtok_bwd_tail(const FewTokTail& tl, const float* xpart, int splits, int M,
+                                   int N, int K, __nv_bfloat16* dx, cudaStream_t stream) {
+  const int R = tl.groups.n * tl.r;
+  if (M < 1 || M > kFewTokDxMaxTokens || R != tl.fold.R || R > kFoldMaxR || tl.r % 8 ||
+      K % 2 || !tl.fold.part || tl.fold.gsplit < 1 || (dx && (!xpart || splits < 1)))
+    return cudaErrorInvalidValue;
+  FtTail t;
+  t.dpart = tl.fold.part;
+  t.gsplit = tl.fold.gsplit;
+  t.R = R;
+  t.r = tl.r;
+  t.scale = tl.fold.scale;
+  t.xpart = xpart;
+  t.splits = splits;
+  t.M = M;
+  t.N = N;
+  t.K = K;
+  t.X = tl.X;
+  t.dY = tl.dY;
+  t.XA = tl.XA;
+  t.A = tl.A;
+  t.groups = tl.groups;
+  t.dx = dx;
+  t.dA = tl.dA;
+  t.dB = tl.dB;
+  const long long per = 128;
+  t.nx = dx ? static_cast<int>((static_cast<long long>(M) * (K / 2) + per - 1) / per) : 0;
+  t.na = static_cast<int>((static_cast<long long>(R) * (K / 2) + per - 1) / per);
+  const long long nb = (static_cast<long long>(N) * (tl.r / 8) + per - 1) / per;
+  return launch_pdl(nf4_fewtok_bwd_tail, dim3(static_cast<unsigned>(t.nx + t.na + nb)),
+                    dim3(128), 0, stream, 1, t);
+}
 
 FewTokDxPlan fewtok_dx_plan(int M, int N, int K, int sm_count) {
   FewTokDxPlan p;
@@ -285,7 +434,8 @@ cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_
                                  const uint8_t* absmax_q8, const float* absmax_scale, int dq,
                                  const __nv_bfloat16* sdyb, const __nv_bfloat16* A, int R,
                                  __nv_bfloat16* dx, float* part, size_t part_bytes,
-                                 const Codebook& cb, int* err, cudaStream_t stream) {
+                                 const Codebook& cb, int* err, cudaStream_t stream,
+                                 bool finalize) {
   if (M < 1 || M > kFewTokDxMaxTokens || N % kFtRows || K % 64 || p.part_bytes > part_bytes ||
       !part)
     return cudaErrorInvalidValue;
@@ -317,7 +467,7 @@ cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_
       e = launch_pdl(nf4_dx_fewtok_kernel<2>, dim3(p.grid), dim3(kFtThreads), ft_smem_bytes(2),
                      stream, 1, tm_q, tm_dy, a);
   }
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || !finalize) return e;
   const long long pairs = static_cast<long long>(M) * (K / 2);
   return launch_pdl(nf4_dx_fewtok_finalize, dim3(static_cast<unsigned>((pairs + 127) / 128)),
                     dim3(128), 0, stream, 1, a, sdyb, A, R, dx);

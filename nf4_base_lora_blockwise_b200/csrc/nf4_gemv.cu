@@ -287,15 +287,29 @@ __global__ void __launch_bounds__(kGvThreads, 2)
 //                    + sum_j ext_act[tok, g, j] * ext_w[row, j] ),  g = the row tile's adapter
 // Grid (row tiles, tokens), one row per thread.  Thread 0 finds the CTAs whose ranges cover
 // the row tile (one 64-bit division each) and shares them through shared memory.
+// With fold.part, the token's scaled rank-r activations are summed here from the
+// down-projection's partials (and row tile 0 writes the saved bf16 sums) instead of being read
+// from ext_act.
 __global__ void __launch_bounds__(kGvRows) nf4_gemv_finalize(
     const float* __restrict__ partial, int M, int N, int K, long long U, int G, int max_seg,
     int Mp, const __nv_bfloat16* __restrict__ ext_act, const __nv_bfloat16* __restrict__ ext_w,
-    int r, const RowGroups groups, __nv_bfloat16* __restrict__ out) {
+    int r, const RowGroups groups, __nv_bfloat16* __restrict__ out, const RankFold fold) {
   __shared__ int s_first, s_last, s_seg0;
+  __shared__ float s_ea[kFoldMaxR];
   pdl_wait();  // the segment partial sums are complete
   pdl_trigger();
   const int KB = K / 64;
   const int rt = blockIdx.x, tok = blockIdx.y;
+  if (fold.part) {
+    for (int j = threadIdx.x; j < fold.R; j += blockDim.x) {
+      float v = 0.f;
+      for (int g = 0; g < fold.gsplit; ++g)
+        v += __ldg(fold.part + (static_cast<long long>(g) * 128 + tok) * fold.R + j);
+      if (rt == 0 && fold.saved)
+        fold.saved[static_cast<long long>(tok) * fold.R + j] = __float2bfloat16_rn(v);
+      s_ea[j] = __bfloat162float(__float2bfloat16_rn(fold.scale * v));
+    }
+  }
   if (threadIdx.x == 0) {
     const long long us = static_cast<long long>(rt) * KB, ue = us + KB;
     // CTA holding unit u: the largest b with floor(b U / G) <= u.
@@ -325,9 +339,24 @@ __global__ void __launch_bounds__(kGvRows) nf4_gemv_finalize(
       if (b + i <= b_last) v += p[i];
   }
   float e = 0.f;
+  const __nv_bfloat16* ew = ext_w + static_cast<long long>(row) * r;
+  if (fold.part) {
+    const float* ea = s_ea + row_group(groups, rt * kGvRows) * r;
+    for (int j = 0; j < r; j += 8) {
+      const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(ew + j));
+      const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&w4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 w = __bfloat1622float2(w2[i]);
+        e = fmaf(ea[j + 2 * i], w.x, e);
+        e = fmaf(ea[j + 2 * i + 1], w.y, e);
+      }
+    }
+    out[static_cast<long long>(tok) * N + row] = __float2bfloat16_rn(v + e);
+    return;
+  }
   const __nv_bfloat16* ea = ext_act + static_cast<long long>(tok) * groups.n * r +
                             row_group(groups, rt * kGvRows) * r;
-  const __nv_bfloat16* ew = ext_w + static_cast<long long>(row) * r;
   for (int j = 0; j < r; j += 8) {
     const uint4 a4 = *reinterpret_cast<const uint4*>(ea + j);
     const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(ew + j));
@@ -369,7 +398,7 @@ cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const 
                                 int N, int K, const __nv_bfloat16* ext_act,
                                 const __nv_bfloat16* ext_w, int r, const RowGroups& groups,
                                 __nv_bfloat16* out, float* partial, size_t partial_floats,
-                                const Codebook& cb, cudaStream_t stream) {
+                                const Codebook& cb, cudaStream_t stream, const RankFold* fold) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -412,9 +441,15 @@ cudaError_t launch_nf4_gemv_fwd(const __nv_bfloat16* X, const uint8_t* q, const 
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  RankFold f = {};
+  if (fold) {
+    if (!fold->part || fold->R > kFoldMaxR || fold->R != groups.n * r || fold->gsplit < 1 || M > 128)
+      return cudaErrorInvalidValue;
+    f = *fold;
+  }
   return launch_pdl(nf4_gemv_finalize, dim3((N + kGvRows - 1) / kGvRows, M), dim3(kGvRows), 0,
                     stream, 1, static_cast<const float*>(partial), M, N, K, p.units, p.grid,
-                    p.max_seg, 8 * p.tt, ext_act, ext_w, r, groups, out);
+                    p.max_seg, 8 * p.tt, ext_act, ext_w, r, groups, out, f);
 }
 
 }  // namespace qlora

@@ -206,12 +206,14 @@ size_t gemm_ws_bytes(int M, int N, int K, int r, bool trans) {
 //                 the call before the launch that counts them
 //   [3]  scratch  fp32 partial sums of the dequant GEMM (stream-K slots, or the few-token
 //                 kernel's segment slots), written and read within one launch pair
+//   [4]  rpart    (M <= 32) fp32 partials of the rank-r down-projection, added by the
+//                 few-token kernels' last launch (RankFold, FewTokTail)
 // The rank-r products reduce inside their clusters and need no scratch.
 // ---------------------------------------------------------------------------------------------
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-  size_t small0, small1, flags, flags_bytes, scratch, scratch_bytes, total;
+  size_t small0, small1, flags, flags_bytes, scratch, scratch_bytes, rpart, rpart_bytes, total;
 };
 
 WsLayout ws_layout(int M, int N, int K, int r) {
@@ -224,7 +226,12 @@ WsLayout ws_layout(int M, int N, int K, int r) {
   L.flags_bytes = align256(gemm_rank_flag_bytes(M));
   L.scratch = L.flags + L.flags_bytes;
   L.scratch_bytes = align256(gemm);
-  L.total = L.scratch + L.scratch_bytes;
+  // Few tokens: the down-projection's second-level partials, left for the few-token kernels'
+  // last launch to add (one row tile; at most one cluster per SM, up to kGemmMaxCtas).
+  L.rpart = L.scratch + L.scratch_bytes;
+  L.rpart_bytes =
+      M <= kGemvMaxTokens ? align256(static_cast<size_t>(kGemmMaxCtas) * 128 * r * 4) : 0;
+  L.total = L.rpart + L.rpart_bytes;
   return L;
 }
 
@@ -407,11 +414,15 @@ CUtensorMapSwizzle swizzle_of(int span) {
 qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc, int r,
                           const RowGroups& groups, float scale, void* saved, void* scaled,
                           int* err, cudaStream_t s, void* scratch = nullptr,
-                          size_t scratch_bytes = 0) {
+                          size_t scratch_bytes = 0, void* fold_part = nullptr,
+                          size_t fold_bytes = 0) {
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
   const int rg = w_rc ? r : r / groups.n;
   const RankPlan p = rank_down_plan(M, C, r, rg, w_rc, sms, scratch ? scratch_bytes : 0);
+  // fold_part: the same plan, its second-level partials left in fold_part for the consumer to
+  // add (no finalize launch); the caller has checked down_foldable.
+  if (fold_part && (p.gsplit < 2 || p.part_bytes > fold_bytes)) return QLORA_ERR_WORKSPACE;
   RankMaps maps;
   qlora_status st = encode_2d(&maps.big, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, in, C, M, C * 2ull,
                               64, p.box_rows_in, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -423,13 +434,23 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
     st = encode_2d(&maps.small, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, rg, C, rg * 2ull,
                    p.small.box_w, p.box_rows_w, swizzle_of(p.small.swizzle));
   if (st != QLORA_OK) return st;
-  const cudaError_t e = launch_rank_down(maps, p, M, C, r, rg, w_rc, groups, scale,
-                                         static_cast<__nv_bfloat16*>(saved),
-                                         static_cast<__nv_bfloat16*>(scaled), err, s,
-                                         static_cast<float*>(scratch));
+  const cudaError_t e = launch_rank_down(
+      maps, p, M, C, r, rg, w_rc, groups, scale, static_cast<__nv_bfloat16*>(saved),
+      static_cast<__nv_bfloat16*>(scaled), err, s,
+      static_cast<float*>(fold_part ? fold_part : scratch), fold_part == nullptr);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  count(p.gsplit > 1 ? 2 : 1);
+  count(p.gsplit > 1 && !fold_part ? 2 : 1);
   return QLORA_OK;
+}
+
+// Whether do_lora_down of this shape can leave its partials for the consumer (fold_part): the
+// plan do_lora_down takes with scratch_bytes splits the reduction over clusters (gsplit > 1)
+// into a single row tile, and the partials fit fold_bytes.
+bool down_foldable(int M, int C, int r, int rg, bool w_rc, int sms, size_t scratch_bytes,
+                   size_t fold_bytes, int* gsplit) {
+  const RankPlan p = rank_down_plan(M, C, r, rg, w_rc, sms, scratch_bytes);
+  *gsplit = p.gsplit;
+  return M <= 128 && r <= kFoldMaxR && !p.rows && p.gsplit > 1 && p.part_bytes <= fold_bytes;
 }
 
 // `partial` / `partial_bytes`: scratch for the stream-K partial sums (whole tiles if too small).
@@ -437,21 +458,24 @@ qlora_status do_lora_down(const void* in, int M, int C, const void* w, bool w_rc
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
                      const void* ext_act, int M, int r, const RowGroups& groups, void* out,
                      int* err, void* partial, size_t partial_bytes, cudaStream_t s,
-                     const RankFusion* fuse = nullptr, int sm_limit = 0) {
+                     const RankFusion* fuse = nullptr, int sm_limit = 0,
+                     const RankFold* fold = nullptr, const FewTokTail* tail = nullptr) {
+  // fold (few-token forward) / tail (few-token dX): the few-token kernels' last launch adds the
+  // down-projection's partials itself (the caller has checked that those kernels apply).
   if (!trans && M <= kGemvMaxTokens && partial) {
     // Few tokens: the register-direct kernel streams the weight without the tcgen05 rings.
     const cudaError_t e = launch_nf4_gemv_fwd(
         static_cast<const __nv_bfloat16*>(act), W->q, W->absmax, W->absmax_q8, W->absmax_scale,
         W->double_quant ? 1 : 0, M, W->N, W->K, static_cast<const __nv_bfloat16*>(ext_act),
         static_cast<const __nv_bfloat16*>(ext_w), r, groups, static_cast<__nv_bfloat16*>(out),
-        static_cast<float*>(partial), partial_bytes / 4, codebook(), s);
+        static_cast<float*>(partial), partial_bytes / 4, codebook(), s, fold);
     if (e == cudaSuccess) {
       count(2);
       return QLORA_OK;
     }
     // cudaErrorInvalidValue: the scratch is too small for its partials (nothing was launched,
     // so no error is pending); use the tcgen05 kernel instead.
-    if (e != cudaErrorInvalidValue) return QLORA_ERR_CUDA;
+    if (e != cudaErrorInvalidValue || fold) return QLORA_ERR_CUDA;
   }
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -470,12 +494,17 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
           mq, md, fp, M, W->N, W->K, W->absmax, W->absmax_q8, W->absmax_scale,
           W->double_quant ? 1 : 0, static_cast<const __nv_bfloat16*>(ext_act),
           static_cast<const __nv_bfloat16*>(ext_w), r, static_cast<__nv_bfloat16*>(out),
-          static_cast<float*>(partial), partial_bytes, codebook(), err, s);
+          static_cast<float*>(partial), partial_bytes, codebook(), err, s, tail == nullptr);
       if (e != cudaSuccess) return QLORA_ERR_CUDA;
+      if (tail &&
+          launch_fewtok_bwd_tail(*tail, static_cast<float*>(partial), fp.splits, M, W->N, W->K,
+                                 static_cast<__nv_bfloat16*>(out), s) != cudaSuccess)
+        return QLORA_ERR_CUDA;
       count(2);
       return QLORA_OK;
     }
   }
+  if (tail) return QLORA_ERR_WORKSPACE;  // the caller checked the few-token plan fits
   if (sm_limit > 0 && sm_limit < sms && !fuse) sms = sm_limit;
   else sm_limit = 0;
   GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms, fuse != nullptr);
@@ -688,6 +717,21 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
                        reinterpret_cast<unsigned*>(w8 + L.flags), L.flags_bytes};
     return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s, &f);
   }
+  // Few tokens: the few-token kernel's finalize adds X A^T's partials itself and writes the
+  // saved XA (one launch fewer; the same bits).
+  int gsplit = 0;
+  if (M <= kGemvMaxTokens &&
+      gemv_plan(M, W->N, W->K, std::min(sms, kGemmMaxCtas)).partial_floats * 4 <=
+          L.scratch_bytes &&
+      down_foldable(M, W->K, R, R, true, sms, L.scratch_bytes, L.rpart_bytes, &gsplit)) {
+    st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, nullptr, nullptr, err, s,
+                      w8 + L.scratch, L.scratch_bytes, w8 + L.rpart, L.rpart_bytes);
+    if (st != QLORA_OK) return st;
+    const RankFold f{reinterpret_cast<const float*>(w8 + L.rpart), gsplit, R, scale,
+                     static_cast<__nv_bfloat16*>(XA_saved)};
+    return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s,
+                   nullptr, 0, &f);
+  }
   // (The GEMM's scratch is free until the GEMM runs: the few-token split uses it first.)
   st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, XA_saved, sxa, err, s,
                     w8 + L.scratch, L.scratch_bytes);
@@ -720,6 +764,44 @@ qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W
   auto* sdyb = reinterpret_cast<__nv_bfloat16*>(w8 + L.small1);
   float* scratch = reinterpret_cast<float*>(w8 + L.scratch);
 
+  // Few tokens: dY B left as partials, the few-token dX kernel, and one last launch that adds
+  // the partials and computes dX, dA and dB (XA recomputed first when it was not saved, with
+  // the forward's own plan, so the same bits).
+  {
+    int fsms = 0, gsplit = 0;
+    if (gemm_device_sms(&fsms) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (M <= kFewTokDxMaxTokens &&
+        (!dX || fewtok_dx_plan(M, W->N, W->K, fsms).part_bytes <= L.scratch_bytes) &&
+        down_foldable(M, W->N, R, r, false, fsms, L.scratch_bytes, L.rpart_bytes, &gsplit)) {
+      const void* xa = XA_saved;
+      if (!xa) {
+        st = do_lora_down(X, M, W->K, A, true, R, single_group(W->K), scale, dyb, sdyb, err, s,
+                          scratch, L.scratch_bytes);
+        if (st != QLORA_OK) return st;
+        xa = dyb;
+      }
+      st = do_lora_down(dY, M, W->N, B, false, R, g, scale, nullptr, nullptr, err, s, scratch,
+                        L.scratch_bytes, w8 + L.rpart, L.rpart_bytes);
+      if (st != QLORA_OK) return st;
+      FewTokTail t;
+      t.fold = RankFold{reinterpret_cast<const float*>(w8 + L.rpart), gsplit, R, scale, nullptr};
+      t.X = static_cast<const __nv_bfloat16*>(X);
+      t.dY = static_cast<const __nv_bfloat16*>(dY);
+      t.XA = static_cast<const __nv_bfloat16*>(xa);
+      t.A = static_cast<const __nv_bfloat16*>(A);
+      t.groups = g;
+      t.r = r;
+      t.dA = dA;
+      t.dB = dB;
+      if (dX)
+        return do_gemm(dY, W, true, A, sdyb, M, R, single_group(W->K), dX, err, scratch,
+                       L.scratch_bytes, s, nullptr, 0, nullptr, &t);
+      if (launch_fewtok_bwd_tail(t, nullptr, 0, M, W->N, W->K, nullptr, s) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+      count(1);
+      return QLORA_OK;
+    }
+  }
   // Without a saved XA, recompute it from X (the forward's own kernel on the same inputs, so
   // bit for bit the value it would have saved) and take dB first, while small0 holds it.
   if (!XA_saved) {
