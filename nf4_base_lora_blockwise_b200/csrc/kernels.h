@@ -230,8 +230,11 @@ struct FewTokDxPlan {
   size_t part_bytes;  // workspace the partials need
 };
 FewTokDxPlan fewtok_dx_plan(int M, int N, int K, int sm_count);
+// tm_am (nullable): fp32 absmax [N, K/64] in boxes {4, 64}, taken when the absmax is not
+// double-quantised and K % 256 == 0 (the stage's block scales then arrive with its codes).
 cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_dy,
-                                 const FewTokDxPlan& p, int M, int N, int K, const float* absmax,
+                                 const CUtensorMap* tm_am, const FewTokDxPlan& p, int M, int N,
+                                 int K, const float* absmax,
                                  const uint8_t* absmax_q8, const float* absmax_scale, int dq,
                                  const __nv_bfloat16* sdyb, const __nv_bfloat16* A, int R,
                                  __nv_bfloat16* dx, float* part, size_t part_bytes,

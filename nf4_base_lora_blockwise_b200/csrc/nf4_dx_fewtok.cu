@@ -31,8 +31,11 @@ constexpr int kFtCols = 256;              // output columns per CTA
 constexpr uint32_t kFtCodeBytes = kFtRows * kFtCols / 2;  // 8 KB of codes per stage
 constexpr uint32_t kFtDecBytes = kFtRows * kFtCols * 2;   // 32 KB decoded bf16 tile
 
+constexpr uint32_t kFtAmBytes = kFtRows * 4 * 4;  // block scales: 64 rows x 4 blocks, fp32
+// A ring slot: the codes, dY [16 mb tokens, 64 rows], and (fp32 absmax, K % 256 == 0) the
+// stage's block scales.
 __host__ __device__ constexpr uint32_t ft_slot_bytes(int mb) {
-  return kFtCodeBytes + static_cast<uint32_t>(mb) * 2048u;  // + dY [16 mb tokens, 64 rows]
+  return kFtCodeBytes + static_cast<uint32_t>(mb) * 2048u + kFtAmBytes;
 }
 // TMA ring depth: 4 stages, 3 with 32 tokens, so two CTAs fit on an SM either way.
 __host__ __device__ constexpr int ft_stages(int mb) { return mb == 1 ? 4 : 3; }
@@ -52,6 +55,7 @@ struct FtArgs {
   float* part;     // [splits, M, K] fp32
   int* err;
   Codebook cb;
+  int am_tma;      // the block scales arrive in the ring slot (else per-thread loads)
 };
 
 // grid (gk x splits): CTA b takes output columns 256 (b % gk) .. and the row steps of split
@@ -59,7 +63,8 @@ struct FtArgs {
 template <int MB>
 __global__ void __launch_bounds__(kFtThreads, 2)
     nf4_dx_fewtok_kernel(const __grid_constant__ CUtensorMap tm_q,
-                         const __grid_constant__ CUtensorMap tm_dy, const FtArgs a) {
+                         const __grid_constant__ CUtensorMap tm_dy,
+                         const __grid_constant__ CUtensorMap tm_am, const FtArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -90,14 +95,16 @@ __global__ void __launch_bounds__(kFtThreads, 2)
     uint8_t* dst = ring + (i % kFtStages) * kSlot;
     uint64_t* bar = full + (i % kFtStages);
     const int n0 = (st0 + i) * kFtRows;
-    mbar_arrive_expect_tx(bar, kSlot);
+    mbar_arrive_expect_tx(bar, kFtCodeBytes + MB * 2048u + (a.am_tma ? kFtAmBytes : 0u));
     tma_load_2d(dst, &tm_q, bar, k0 / 2, n0);
     tma_load_2d(dst + kFtCodeBytes, &tm_dy, bar, n0, 0);
+    if (a.am_tma) tma_load_2d(dst + kFtCodeBytes + MB * 2048u, &tm_am, bar, kg * 4, n0);
     issued = i + 1;
   };
   if (tid == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_dy);
+    if (a.am_tma) tma_prefetch_desc(&tm_am);
     for (int i = 0; i < n_st && i < kFtStages; ++i) issue(i);
   }
 
@@ -105,7 +112,7 @@ __global__ void __launch_bounds__(kFtThreads, 2)
   const int drow = tid >> 2, dj = tid & 3;
   const int kb = kg * 4 + dj;
   auto absmax_of = [&](int i) -> float {
-    if (i >= n_st || kb >= a.kblocks) return 0.f;  // past K: zero weight
+    if (a.am_tma || i >= n_st || kb >= a.kblocks) return 0.f;  // past K: zero weight
     const long long n = static_cast<long long>(st0 + i) * kFtRows + drow;
     return nf4_block_absmax(a.absmax, a.absmax_q8, a.absmax_scale, a.dq, n * a.kblocks + kb);
   };
@@ -138,8 +145,11 @@ __global__ void __launch_bounds__(kFtThreads, 2)
       const uint32_t cph = static_cast<uint32_t>(drow) & 7u;
       const uint4 c0 = *reinterpret_cast<const uint4*>(codes + (((2u * dj) ^ cph) << 4));
       const uint4 c1 = *reinterpret_cast<const uint4*>(codes + (((2u * dj + 1u) ^ cph) << 4));
+      const float scale = a.am_tma ? reinterpret_cast<const float*>(
+                                         ring + slot * kSlot + kFtCodeBytes + MB * 2048u)[tid]
+                                   : am;
       Nf4Lut lut;
-      nf4_build_lut(a.cb, am, lut);
+      nf4_build_lut(a.cb, scale, lut);
       uint8_t* row = d + drow * (kFtCols * 2);
       const uint32_t ph = static_cast<uint32_t>(drow) & 7u;
       const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -430,7 +440,8 @@ FewTokDxPlan fewtok_dx_plan(int M, int N, int K, int sm_count) {
 }
 
 cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_dy,
-                                 const FewTokDxPlan& p, int M, int N, int K, const float* absmax,
+                                 const CUtensorMap* tm_am, const FewTokDxPlan& p, int M, int N,
+                                 int K, const float* absmax,
                                  const uint8_t* absmax_q8, const float* absmax_scale, int dq,
                                  const __nv_bfloat16* sdyb, const __nv_bfloat16* A, int R,
                                  __nv_bfloat16* dx, float* part, size_t part_bytes,
@@ -453,19 +464,21 @@ cudaError_t launch_nf4_fewtok_dx(const CUtensorMap& tm_q, const CUtensorMap& tm_
   a.part = part;
   a.err = err;
   a.cb = cb;
+  a.am_tma = (tm_am && !dq && K % 256 == 0) ? 1 : 0;
+  const CUtensorMap& am_map = a.am_tma ? *tm_am : tm_q;  // (never read without am_tma)
   cudaError_t e;
   if (p.mb == 1) {
     e = cudaFuncSetAttribute(nf4_dx_fewtok_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(ft_smem_bytes(1)));
     if (e == cudaSuccess)
       e = launch_pdl(nf4_dx_fewtok_kernel<1>, dim3(p.grid), dim3(kFtThreads), ft_smem_bytes(1),
-                     stream, 1, tm_q, tm_dy, a);
+                     stream, 1, tm_q, tm_dy, am_map, a);
   } else {
     e = cudaFuncSetAttribute(nf4_dx_fewtok_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(ft_smem_bytes(2)));
     if (e == cudaSuccess)
       e = launch_pdl(nf4_dx_fewtok_kernel<2>, dim3(p.grid), dim3(kFtThreads), ft_smem_bytes(2),
-                     stream, 1, tm_q, tm_dy, a);
+                     stream, 1, tm_q, tm_dy, am_map, a);
   }
   if (e != cudaSuccess || !finalize) return e;
   const long long pairs = static_cast<long long>(M) * (K / 2);

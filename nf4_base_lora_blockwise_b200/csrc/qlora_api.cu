@@ -490,8 +490,16 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
       st = encode_2d(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, W->N, M, W->N * 2ull, 64,
                      16 * fp.mb, CU_TENSOR_MAP_SWIZZLE_128B);
       if (st != QLORA_OK) return st;
+      // fp32 block scales [N, K/64] in boxes of 4 blocks x 64 rows (rows of K/64 * 4 bytes:
+      // a multiple of 16 when K % 256 == 0).
+      CUtensorMap ma;
+      const bool am_tma = !W->double_quant && W->K % 256 == 0 && aligned16(W->absmax);
+      if (am_tma && (st = encode_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, W->absmax, W->K / 64,
+                                    W->N, (W->K / 64) * 4ull, 4, 64,
+                                    CU_TENSOR_MAP_SWIZZLE_NONE)) != QLORA_OK)
+        return st;
       const cudaError_t e = launch_nf4_fewtok_dx(
-          mq, md, fp, M, W->N, W->K, W->absmax, W->absmax_q8, W->absmax_scale,
+          mq, md, am_tma ? &ma : nullptr, fp, M, W->N, W->K, W->absmax, W->absmax_q8, W->absmax_scale,
           W->double_quant ? 1 : 0, static_cast<const __nv_bfloat16*>(ext_act),
           static_cast<const __nv_bfloat16*>(ext_w), r, static_cast<__nv_bfloat16*>(out),
           static_cast<float*>(partial), partial_bytes, codebook(), err, s, tail == nullptr);
