@@ -113,8 +113,10 @@ QLORA_API qlora_status qlora_nf4_dequant(const qlora_nf4_weight* W, void* Wd, ql
 /* Scratch bytes the linear entry points need for (M, N, K, r), 1 <= r <= 128: the scaled rank-r
  * activations, the fused down-projection's counters, the few-token split partials of the rank-r
  * reductions and the stream-K partial sums of the dequant GEMM (sized for any device of up to
- * 160 SMs), plus, for r not a multiple of 8, the zero-padded copies described below.  Needs no
- * GPU; 0 for an invalid shape. */
+ * 160 SMs), for M <= 32 a region where the down-projection leaves its split partials for the
+ * few-token kernels' last launch to add (so each direction is three launches), plus, for r not
+ * a multiple of 8, the zero-padded copies described below.  Needs no GPU; 0 for an invalid
+ * shape. */
 QLORA_API size_t qlora_workspace_bytes(int M, int N, int K, int r);
 
 /* Forward.  X [M, K], A [r, K], B [N, r] bf16 device (read); H [M, N] bf16 device (written);
@@ -140,7 +142,11 @@ QLORA_API qlora_status qlora_linear_fwd(const void* X, const qlora_nf4_weight* W
  * NULL: X A^T is then recomputed from X (one more pass over X), bit-identical to the value the
  * forward would have saved, so the results do not change.
  * dX [M, K] bf16 device (written; may be NULL to skip the dX GEMM).
- * dA [r, K] and dB [N, r] fp32 device (overwritten).  ws and r as for the forward. */
+ * dA [r, K] and dB [N, r] fp32 device (overwritten).  ws and r as for the forward.
+ * With XA_saved and dX given, dA and dB may be computed on a library-owned stream beside the dX
+ * GEMM (qlora_set_side_overlap); the call joins it back to `stream` before returning, so the
+ * outputs are ordered on `stream` as usual.  For M <= 32, dA and dB are computed in the
+ * few-token dX kernel's last launch, summed over the tokens in order in fp32. */
 QLORA_API qlora_status qlora_linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
                               const void* A, const void* B, const void* XA_saved, int M, int r,
                               float alpha, void* dX, float* dA, float* dB, void* ws,
