@@ -35,7 +35,7 @@
 //   warp 0      X producer: activation tiles, then the scaled rank-r tile (s*XA or s*dYB)
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma and commits slots back
 //   warp 2      Q producer: packed code tiles
-//   warp 3      idle
+//   warp 3      with two token halves, lane 0 issues half 1's MMAs (warp 1 then issues half 0's)
 //   warps 4-7   epilogue: TMEM -> registers -> bf16 -> global
 //   warps 8-23  two dequant groups of 8 warps; group g owns the pipeline steps it = g mod 2
 //               (counted across tiles) and W slots 2g, 2g+1.  Each thread turns half of one
@@ -315,22 +315,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (kFused) ncols = 512;
   const uint32_t rank_bytes = P.rank_slot;
   int* err = args.err;
+  // Two token halves: warp 1 issues half 0's MMAs and warp 3 half 1's, each thread waiting only
+  // for its own half's X tile and committing its own MMAs (the halves' accumulators are
+  // disjoint TMEM columns), so the empty and accumulator barriers take one commit from each.
+  // A lone MMA thread's serial chain of barrier operations and issues idles the tensor pipe
+  // between steps.  (Fused launches keep one issuer: the window MMAs read either half.)
+  const bool dual = !kFused && nh == 2;
+  const uint32_t n_issuers = dual ? 2u : 1u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) mbar_init(xfull + s, 1);
     for (int s = 0; s < SW; ++s) {
       mbar_init(wfull + s, 1);
-      mbar_init(wempty + s, 1);
+      mbar_init(wempty + s, n_issuers);  // one commit per MMA-issuing thread
     }
     for (int s = 0; s < SQ; ++s) {
       mbar_init(qfull + s, 1);
       mbar_init(qempty + s, kGroupThreads / 32);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(accfull + b, 1);
+      mbar_init(accfull + b, n_issuers);
       mbar_init(accempty + b, 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, n_issuers);
     mbar_init(rank_full, 1);
     fence_barrier_init();
   }
@@ -447,12 +454,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     static_cast<uint32_t>(v >> P.qlog) & 1u, kErrWaitDrain, err, v);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer -------------------------------------------
-    // One thread issues everything, so the loop keeps its per-step work to a few adds: ring
-    // positions advance incrementally and the smem descriptors are precomputed, the start
-    // address (bits 0-13, >> 4) being the only field that moves.
+  } else if (warp == 1 || (warp == 3 && dual)) {
+    // ------------------------------ MMA issuer(s) ----------------------------------------
+    // The issuing thread keeps its per-step work to a few adds: ring positions advance
+    // incrementally and the smem descriptors are precomputed, the start address (bits 0-13,
+    // >> 4) being the only field that moves.  h_lo .. h_hi - 1: the token halves it issues.
     if (lane == 0) {
+      const int h_lo = dual ? (warp == 1 ? 0 : 1) : 0;
+      const int h_hi = dual ? h_lo + 1 : nh;
       const uint32_t idesc =
           idesc_bf16_f32(128, static_cast<uint32_t>(bt), kTransW ? 1u : 0u, 0u);
       const uint64_t wdesc0 = kTransW ? smem_desc_sw128(smem_u32(w_ring), 8192u, 1024u)
@@ -490,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ws = w_slot(it);
           const int xs = (it & (DX - 1)) * nh;
           bool got = mbar_wait(wfull + ws, w_par(it), kErrWaitDequant, err, it);
-          if (got) got = mbar_wait(xfull + xs, x_par(it), kErrWaitFull, err, it);
-          if (got && nh == 2) got = mbar_wait(xfull + xs + 1, x_par(it), kErrWaitFull, err, it);
+          for (int h = h_lo; got && h < h_hi; ++h)
+            got = mbar_wait(xfull + xs + h, x_par(it), kErrWaitFull, err, it);
           if (!got) {
             ok = false;
             break;
@@ -502,12 +511,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd1 = bd0 + x_slot_step;
           const uint32_t acc0 = k > k0 ? 1u : 0u;  // the segment's first step starts the sum
           if (k < kt) {
+            if (dual) {  // this thread's half only
+              const uint32_t dh = dtm + static_cast<uint32_t>(h_lo) * half_cols;
+              const uint64_t bh = h_lo ? bd1 : bd0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t acc = j > 0 ? 1u : acc0;
-              umma_f16_ss(dtm, ad + j * w_kstep, bd0 + j * x_kstep, idesc, acc);
-              if (nh == 2)
-                umma_f16_ss(dtm + half_cols, ad + j * w_kstep, bd1 + j * x_kstep, idesc, acc);
+              for (int j = 0; j < 4; ++j)
+                umma_f16_ss(dh, ad + j * w_kstep, bh + j * x_kstep, idesc, j > 0 ? 1u : acc0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t acc = j > 0 ? 1u : acc0;
+                umma_f16_ss(dtm, ad + j * w_kstep, bd0 + j * x_kstep, idesc, acc);
+                if (nh == 2)
+                  umma_f16_ss(dtm + half_cols, ad + j * w_kstep, bd1 + j * x_kstep, idesc, acc);
+              }
             }
             if (win.has) {
               // The window's rows of this step's activation tile times its rank-operand tile.
@@ -545,9 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nk = (rem >= 64 ? 64 : rem) / 16;
             for (int j = 0; j < nk; ++j) {
               const uint32_t acc = j > 0 ? 1u : acc0;
-              umma_f16_ss(dtm, ad + j * w_kstep, bd0 + j * x_kstep, idesc, acc);
-              if (nh == 2)
-                umma_f16_ss(dtm + half_cols, ad + j * w_kstep, bd1 + j * x_kstep, idesc, acc);
+              for (int h = h_lo; h < h_hi; ++h)
+                umma_f16_ss(dtm + static_cast<uint32_t>(h) * half_cols, ad + j * w_kstep,
+                            (h ? bd1 : bd0) + j * x_kstep, idesc, acc);
             }
           }
           umma_commit(wempty + ws);  // releases the W slot and, DX steps on, the X slots

@@ -12,7 +12,9 @@ Each run checks three things:
 * no slot is overwritten while reads of its previous contents are pending.
 
 The protocol modelled:
-* per step, the MMA thread waits for W-full and X-full and commits W-empty;
+* per step, the MMA thread waits for W-full and X-full and commits W-empty; with two token
+  halves two MMA threads share the work (each waits for W-full and its own half's X-full and
+  commits W-empty and the accumulator's full barrier, which then count two commits);
 * X slots are refilled after the W-empty of the step DX earlier;
 * Q and W slots are owned per dequant group;
 * on a LoRA extension step every warp of the owning group waits for the slot's release,
@@ -60,14 +62,16 @@ class Fail(Exception):
     pass
 
 
-def simulate(kt, n_ext, nh, qper, nacc, g0, n_steps, seed, all_warps_on_ext=True):
+def simulate(kt, n_ext, nh, qper, nacc, g0, n_steps, seed, all_warps_on_ext=True, dual=True):
     total = kt + n_ext
     DX = 2 if nh == 2 else 4
     SX, SW, NG, NW = DX * nh, 4, 2, 8
+    issuers = [(0, 1), (1, 2)] if (dual and nh == 2) else [(0, nh)]
+    ni = len(issuers)
     xf = [Bar(1) for _ in range(SX)]
-    wf, we = [Bar(1) for _ in range(SW)], [Bar(1) for _ in range(SW)]
+    wf, we = [Bar(1) for _ in range(SW)], [Bar(ni) for _ in range(SW)]
     qf, qe = [Bar(1) for _ in range(NG * qper)], [Bar(NW) for _ in range(NG * qper)]
-    af, ae = [Bar(1) for _ in range(2)], [Bar(4) for _ in range(2)]
+    af, ae = [Bar(ni) for _ in range(2)], [Bar(4) for _ in range(2)]
     xtag, wtag, qtag = [None] * SX, [None] * SW, [None] * (NG * qper)
     xreads, wreads = [0] * SX, [0] * SW
     tma, tensor = [], []
@@ -119,20 +123,20 @@ def simulate(kt, n_ext, nh, qper, nacc, g0, n_steps, seed, all_warps_on_ext=True
                 qf[s].complete_tx(10)
             tma.append(land)
 
-    def mma():
+    def mma(h_lo, h_hi):
         it = 0
         for si, (k0, ln) in enumerate(segs):
             ab, use = (si & 1, si >> 1) if nacc == 2 else (0, si)
             yield from wait(ae[ab], (use & 1) ^ 1)
             for _ in range(ln):
                 ws = w_slot(it)
-                xs = [(it % DX) * nh + h for h in range(nh)]
+                xs = [(it % DX) * nh + h for h in range(h_lo, h_hi)]
                 yield from wait(wf[ws], w_par(it))
                 for s in xs:
                     yield from wait(xf[s], (it // DX) & 1)
                 if wtag[ws] != it:
                     raise Fail(f"MMA step {it}: W slot {ws} holds {wtag[ws]}")
-                for h, s in enumerate(xs):
+                for h, s in zip(range(h_lo, h_hi), xs):
                     if xtag[s] != (it, h):
                         raise Fail(f"MMA step {it}: X slot {s} holds {xtag[s]}")
                 wreads[ws] += 1
@@ -197,7 +201,8 @@ def simulate(kt, n_ext, nh, qper, nacc, g0, n_steps, seed, all_warps_on_ext=True
                     wf[ws].complete_tx(7)
                 tma.append(land)
 
-    roles = [x_producer(), q_producer(), mma()] + [epilogue() for _ in range(4)]
+    roles = [x_producer(), q_producer()] + [mma(lo, hi) for lo, hi in issuers]
+    roles += [epilogue() for _ in range(4)]
     roles += [dequant(g, w) for g in range(NG) for w in range(NW)]
     rng = random.Random(seed)
     idle = 0
@@ -240,6 +245,14 @@ def _cases(n, seed=7):
 def test_protocol_randomised(case):
     kt, n_ext, nh, qper, nacc, g0, n_steps, seed = case
     assert simulate(kt, n_ext, nh, qper, nacc, g0, n_steps, seed) == "ok"
+
+
+@pytest.mark.parametrize("case", list(_cases(40, seed=11)))
+def test_protocol_one_mma_thread(case):
+    """The single-issuer protocol (fused launches, one token half) passes the same checks
+    with two token halves too."""
+    kt, n_ext, nh, qper, nacc, g0, n_steps, seed = case
+    assert simulate(kt, n_ext, nh, qper, nacc, g0, n_steps, seed, dual=False) == "ok"
 
 
 def test_model_catches_extension_step_aliasing():
