@@ -164,18 +164,21 @@ __global__ void __launch_bounds__(kThreads2, 1)
   while (ncols < tile_cols) ncols <<= 1;
   int* err = args.err;
 
+  // Two token blocks: warp 1 of the first CTA issues block 0's MMAs and warp 3 block 1's, so
+  // every commit barrier takes one (multicast) commit from each issuer.
+  const uint32_t n_issuers = nh == 2 ? 2u : 1u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW; ++s) {
       mbar_init(full + s, 4);
-      mbar_init(wempty + s, 1);
+      mbar_init(wempty + s, n_issuers);
     }
     for (int s = 0; s < SQ; ++s) {
       mbar_init(qfull + s, 1);
       mbar_init(qempty + s, kGroupThreads2 / 32);
     }
-    mbar_init(accfull, 1);
+    mbar_init(accfull, n_issuers);
     mbar_init(accempty, 8);
-    mbar_init(drain, 1);
+    mbar_init(drain, n_issuers);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -256,9 +259,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     static_cast<uint32_t>(v >> P.qlog) & 1u, kErrWaitDrain, err, v);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer (first CTA) --------------------------------
+  } else if (warp == 1 || (warp == 3 && nh == 2)) {
+    // ------------------------------ MMA issuers (first CTA) -------------------------------
     if (lane == 0 && lead) {
+      const int h_lo = nh == 2 ? (warp == 1 ? 0 : 1) : 0;
+      const int h_hi = nh == 2 ? h_lo + 1 : nh;
       const uint32_t idesc =
           idesc_bf16_f32(256, static_cast<uint32_t>(bt), kTransW ? 1u : 0u, 0u);
       const uint64_t wdesc0 = kTransW ? smem_desc_sw128(smem_u32(w_ring), 8192u, 1024u)
@@ -290,7 +295,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
                                        16);
           for (int j = 0; j < nk; ++j) {
             const uint32_t acc = (k > 0 || j > 0) ? 1u : 0u;
-            for (int h = 0; h < nh; ++h)
+            for (int h = h_lo; h < h_hi; ++h)
               umma_f16_ss_pair(tmem_base + static_cast<uint32_t>(h) * P.acc_cols,
                                ad + j * w_kstep,
                                bd0 + static_cast<uint64_t>(h) * x_slot_step + j * x_kstep, idesc,
