@@ -288,8 +288,9 @@ class CeState:
 class Step:
     """One step of a workload: its linears' states and the ordered (name, call) stages."""
 
-    def __init__(self, w, dev, seed, unpacked=False):
+    def __init__(self, w, dev, seed, unpacked=False, glu_fused=False):
         self.w = w
+        self.glu_fused = glu_fused  # packed MLP: SwiGLU in the gate/up GEMM's epilogue
         self.share_x = False
         self.pglue = None
         self.ce = None
@@ -410,6 +411,16 @@ class Step:
         if self.pglue is not None:
             sgu, sd = self.pglue
             M, I = self.a.shape
+            if self.glu_fused:
+                # qlora_grouped_fwd_swiglu as one stage: X A^T, then the GEMM that also writes
+                # the SwiGLU output (attributed to the GEMM).
+                fused = [(f"{sgu.L.name}.gemm_fwd", lambda: abi.qlora_grouped_fwd_swiglu(
+                    p(sgu.X), sgu.cw, p(sgu.A), p(sgu.B), M, sgu.L.r, sgu.L.alpha, p(sgu.H),
+                    p(sgu.XA), p(self.a), p(sgu.ws), sgu.ws.numel(), stream))]
+                return (fused + sd.fwd_stages(stream) + sd.bwd_stages(stream)
+                        + [("swiglu.bwd", lambda: abi.qlora_swiglu_packed_bwd(
+                            p(sgu.H), p(sd.dX), p(sgu.dY), M, I, stream))]
+                        + sgu.bwd_stages(stream))
             return (sgu.fwd_stages(stream)
                     + [("swiglu.fwd", lambda: abi.qlora_swiglu_packed_fwd(p(sgu.H), p(self.a), M,
                                                                           I, stream))]
@@ -440,8 +451,12 @@ class Step:
             return
         if self.pglue is not None:
             sgu, sd = self.pglue
-            sgu.forward()
-            linear.swiglu_packed_forward(sgu.H, a=self.a)
+            if self.glu_fused:
+                linear.gate_up_swiglu_forward(sgu.X, sgu.w, sgu.A, sgu.B, sgu.L.alpha, GU=sgu.H,
+                                              XA=sgu.XA, act=self.a, ws=sgu.ws)
+            else:
+                sgu.forward()
+                linear.swiglu_packed_forward(sgu.H, a=self.a)
             sd.forward()
             sd.backward()
             linear.swiglu_packed_backward(sgu.H, sd.dX, dgu=sgu.dY)
@@ -873,12 +888,12 @@ def is_fwd_stage(name):
     return st in ("lora_down_fwd", "gemm_fwd", "fwd")
 
 
-def measure_config(name, dev, steps, warmup, peaks, flush, clocks_on):
+def measure_config(name, dev, steps, warmup, peaks, flush, clocks_on, glu_fused=False):
     """tokens/s, step TFLOP/s, forward and backward times (and, for one linear, their GB/s of
     minimum traffic), the dominant stage's roofline and the clocks, for one workload timed as
     the headline is: CUDA-graph replays with L2 flushed before each."""
     w = synth.workload(name)
-    step = Step(w, dev, seed=0)
+    step = Step(w, dev, seed=0, glu_fused=glu_fused)
     stream = torch.cuda.current_stream()
     run_steps(step, warmup, stream, flush, record=False)
     graph = GraphStep(step)
@@ -1140,6 +1155,12 @@ def main():
                 abi.qlora_set_rank_fusion(prev)
             fused["rank_fusion"] = True
             line["configs"][w.name + "+rank_fusion"] = fused
+            # The MLP block with the SwiGLU in the gate/up GEMM's epilogue
+            # (qlora_grouped_fwd_swiglu; the default step runs the packed SwiGLU kernel).
+            glu = measure_config("mlp_8b", dev, args.config_steps, args.warmup, peaks, flush,
+                                 not args.no_clocks, glu_fused=True)
+            glu["swiglu_fusion"] = True
+            line["configs"]["mlp_8b+swiglu_fusion"] = glu
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

@@ -177,6 +177,22 @@ QLORA_API qlora_status qlora_grouped_fwd(const void* X, const qlora_nf4_weight* 
                                float alpha, void* H, void* XA_saved, void* ws, size_t ws_bytes,
                                qlora_stream_t stream);
 
+/* The packed gate/up forward with its SwiGLU ("Unsloth vs QLoRA vs Liger-Kernel", section 2:
+ * the SwiGLU MLP among the hand-derived fused ops): qlora_grouped_fwd with group_rows {I, I}
+ * (gate rows [0, I) of W, up rows [I, 2I); I = W->N / 2), writing GU [M, 2I] (g, u) as that
+ * call writes H, and also act [M, I] = silu(g) * u (bf16 g and u, fp32 math, bf16 result: the
+ * bits qlora_swiglu_packed_fwd gives on GU).  Where the dequant GEMM runs whole tiles (M > 32,
+ * enough tiles for every SM, I % 128 == 0, rank fusion not used) each CTA takes a gate tile and
+ * then the up tile of the same rows and tokens, and the up tile's epilogue computes act from
+ * the g it has just written: no separate launch and no second read of GU.  Otherwise the call
+ * is qlora_grouped_fwd followed by qlora_swiglu_packed_fwd.  The workspace is
+ * qlora_grouped_workspace_bytes(M, W->N, K, r, 2).  Requirements as for qlora_grouped_fwd with
+ * n_groups = 2 (I a multiple of 128); act must be 16-byte aligned. */
+QLORA_API qlora_status qlora_grouped_fwd_swiglu(const void* X, const qlora_nf4_weight* W,
+                                                const void* A, const void* B, int M, int r,
+                                                float alpha, void* GU, void* XA_saved, void* act,
+                                                void* ws, size_t ws_bytes, qlora_stream_t stream);
+
 QLORA_API qlora_status qlora_grouped_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,
                                const void* A, const void* B, const void* XA_saved,
                                const int* group_rows, int n_groups, int M, int r, float alpha,

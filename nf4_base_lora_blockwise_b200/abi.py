@@ -31,6 +31,7 @@ EXPORTS = (
     "qlora_device_error",
     "qlora_grouped_workspace_bytes",
     "qlora_grouped_fwd",
+    "qlora_grouped_fwd_swiglu",
     "qlora_grouped_bwd",
     "qlora_swiglu_packed_fwd",
     "qlora_swiglu_packed_bwd",
@@ -130,6 +131,8 @@ def _lib():
             "qlora_grouped_fwd": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _SZ,
                                        _VP]),
+            "qlora_grouped_fwd_swiglu": (_I, [_VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _I, _I,
+                                              _F, _VP, _VP, _VP, _VP, _SZ, _VP]),
             "qlora_grouped_bwd": (_I, [_VP, _VP, ctypes.POINTER(Nf4Weight), _VP, _VP, _VP,
                                        ctypes.POINTER(_I), _I, _I, _I, _F, _VP, _VP, _VP, _VP,
                                        _SZ, _VP]),
@@ -200,6 +203,13 @@ def qlora_grouped_fwd(X, weight, A, B, group_rows, M, r, alpha, H, XA_saved, ws,
     _check("qlora_grouped_fwd", _lib().qlora_grouped_fwd(X, ctypes.byref(weight), A, B, rows, n,
                                                          M, r, float(alpha), H, XA_saved, ws,
                                                          ws_bytes, stream))
+
+
+def qlora_grouped_fwd_swiglu(X, weight, A, B, M, r, alpha, GU, XA_saved, act, ws, ws_bytes,
+                             stream):
+    _check("qlora_grouped_fwd_swiglu",
+           _lib().qlora_grouped_fwd_swiglu(X, ctypes.byref(weight), A, B, M, r, float(alpha), GU,
+                                           XA_saved, act, ws, ws_bytes, stream))
 
 
 def qlora_grouped_bwd(dY, X, weight, A, B, XA_saved, group_rows, M, r, alpha, dX, dA, dB, ws,

@@ -122,6 +122,13 @@ struct GemmArgs {
   // SMs the launch may use (0: all of them); the rest are left to a kernel running beside it.
   // The tile (bt, nh) must be the one gemm_pick_tile gives for that many SMs.
   int sm_limit;
+  // SwiGLU on a packed gate/up layer (whole tiles, forward, unfused rank; 0 / null: off):
+  // rows [0, glu_I) of W0 are the gate rows and [glu_I, 2 glu_I) the up rows (glu_I % 128 == 0).
+  // CTA b takes (gate row tile j, token tile) pairs b, b + G, ..., each as the gate tile followed
+  // by the matching up tile, and the up tile's epilogue adds glu_out[M, glu_I] =
+  // silu(g) * u from the g it wrote one tile earlier (bf16 g and u, fp32 math).
+  __nv_bfloat16* glu_out;
+  int glu_I;
 };
 
 struct GemmMaps {
@@ -178,6 +185,9 @@ struct GemmTile {
 GemmTile gemm_pick_tile(int M, int rows_w, int steps_per_tile, int sm_count, bool fused = false);
 cudaError_t gemm_device_sms(int* sms);  // SMs of the current device (cached)
 size_t gemm_smem_bytes(int bt, int nh);
+// Whether a forward launch of the packed gate/up layer [2 I, K] on M tokens can add the SwiGLU
+// output in its epilogue (GemmArgs::glu_out): whole tiles on sm_count SMs, I % 128 == 0.
+bool gemm_glu_ok(int M, int I, int steps_per_tile, int sm_count);
 // Falls back to whole tiles when stream-K is chosen but `partial` is null or smaller than the
 // schedule needs (partial_floats_avail).  *launched = kernels enqueued (1, or 2 with stream-K).
 cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,

@@ -317,6 +317,8 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& gro
   a.rank_flags = nullptr;
   a.rank_slot = 0;
   a.sm_limit = 0;
+  a.glu_out = nullptr;
+  a.glu_I = 0;
   return a;
 }
 
@@ -455,11 +457,18 @@ bool down_foldable(int M, int C, int r, int rg, bool w_rc, int sms, size_t scrat
 
 // `partial` / `partial_bytes`: scratch for the stream-K partial sums (whole tiles if too small).
 // groups (forward only): adapters packed along W0's rows, each with r columns of ext_act.
+// SwiGLU output of a packed gate/up forward (GemmArgs::glu_out): a [M, I] bf16.
+struct GluOut {
+  void* a;
+  int I;
+};
+
 qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, const void* ext_w,
                      const void* ext_act, int M, int r, const RowGroups& groups, void* out,
                      int* err, void* partial, size_t partial_bytes, cudaStream_t s,
                      const RankFusion* fuse = nullptr, int sm_limit = 0,
-                     const RankFold* fold = nullptr, const FewTokTail* tail = nullptr) {
+                     const RankFold* fold = nullptr, const FewTokTail* tail = nullptr,
+                     const GluOut* glu = nullptr) {
   // fold (few-token forward) / tail (few-token dX): the few-token kernels' last launch adds the
   // down-projection's partials itself (the caller has checked that those kernels apply).
   if (!trans && M <= kGemvMaxTokens && partial) {
@@ -518,6 +527,10 @@ qlora_status do_gemm(const void* act, const qlora_nf4_weight* W, bool trans, con
   GemmArgs a = gemm_args(W, M, r, groups, trans, out, err, sms, fuse != nullptr);
   a.partial = static_cast<float*>(partial);
   a.sm_limit = sm_limit;
+  if (glu) {  // the caller checked gemm_glu_ok
+    a.glu_out = static_cast<__nv_bfloat16*>(glu->a);
+    a.glu_I = glu->I;
+  }
   GemmMaps maps;
 #ifdef QLORA_CTA_PAIRS
   if (!fuse && !sm_limit && gemm2_applies(M, a.rows_w, a.kt + a.n_ext, sms, groups)) {
@@ -695,7 +708,8 @@ qlora_status do_weight_grads(const void* dY, const void* X, const void* XA, cons
 // `scale` is alpha / r of the caller's rank (the padded-rank path passes r rounded up).
 qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A, const void* B,
                         const RowGroups& g, int M, int r, float scale, void* H, void* XA_saved,
-                        void* ws, size_t ws_bytes, cudaStream_t s) {
+                        void* ws, size_t ws_bytes, cudaStream_t s,
+                        const GluOut* glu = nullptr) {
   if (!X || !A || !B || !H) return QLORA_ERR_NULL;
   const int R = g.n * r;
   if (M < 1 || !rank_ok(r) || !rank_ok(R)) return QLORA_ERR_SHAPE;
@@ -718,7 +732,7 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
   // (whole tiles: the GEMM streams every X tile anyway), else as a launch of its own.
   int sms = 0;
   if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
-  if (g_rank_fusion.load(std::memory_order_relaxed) && M > kGemvMaxTokens &&
+  if (!glu && g_rank_fusion.load(std::memory_order_relaxed) && M > kGemvMaxTokens &&
       gemm_rank_fusable(M, W->N, W->K / 64 + ext_steps(r), sms, R,
                                               gemm_rank_slot_bytes(false, R, r))) {
     const RankFusion f{A, R, r, single_group(W->K), XA_saved, sxa, scale,
@@ -745,7 +759,8 @@ qlora_status linear_fwd(const void* X, const qlora_nf4_weight* W, const void* A,
                     w8 + L.scratch, L.scratch_bytes);
   if (st != QLORA_OK) return st;
   // h = X deq(W0)^T + (s XA_g) B_g^T for the rows of each adapter g, in one launch.
-  return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s);
+  return do_gemm(X, W, false, B, sxa, M, r, g, H, err, w8 + L.scratch, L.scratch_bytes, s,
+                 nullptr, 0, nullptr, nullptr, glu);
 }
 
 qlora_status linear_bwd(const void* dY, const void* X, const qlora_nf4_weight* W, const void* A,
@@ -1041,6 +1056,33 @@ qlora_status qlora_grouped_fwd(const void* X, const qlora_nf4_weight* W, const v
   return linear_fwd(X, W, A, B, g, M, r, alpha / static_cast<float>(r), H, XA_saved, ws,
                     ws_bytes,
                     static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_grouped_fwd_swiglu(const void* X, const qlora_nf4_weight* W, const void* A,
+                                      const void* B, int M, int r, float alpha, void* GU,
+                                      void* XA_saved, void* act, void* ws, size_t ws_bytes,
+                                      qlora_stream_t stream) {
+  qlora_status st = check_weight(W);
+  if (st != QLORA_OK) return st;
+  if (!act) return QLORA_ERR_NULL;
+  if (!aligned16(act)) return QLORA_ERR_ALIGN;
+  if (W->N < 16 || W->N % 16) return QLORA_ERR_SHAPE;
+  const int I = W->N / 2;
+  const int rows[2] = {I, I};
+  RowGroups g;
+  if ((st = make_groups(rows, 2, W->N, r, &g)) != QLORA_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int sms = 0;
+  if (gemm_device_sms(&sms) != cudaSuccess) return QLORA_ERR_CUDA;
+  const float scale = alpha / static_cast<float>(r);
+  if (M > kGemvMaxTokens && rank_ok(r) && gemm_glu_ok(M, I, W->K / 64 + ext_steps(r), sms)) {
+    const GluOut glu{act, I};
+    return linear_fwd(X, W, A, B, g, M, r, scale, GU, XA_saved, ws, ws_bytes, s, &glu);
+  }
+  // Otherwise the packed SwiGLU kernel after the layer: the same bits.
+  if ((st = linear_fwd(X, W, A, B, g, M, r, scale, GU, XA_saved, ws, ws_bytes, s)) != QLORA_OK)
+    return st;
+  return qlora_swiglu_packed_fwd(GU, act, M, I, stream);
 }
 
 qlora_status qlora_grouped_bwd(const void* dY, const void* X, const qlora_nf4_weight* W,

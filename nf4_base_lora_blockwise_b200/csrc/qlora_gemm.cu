@@ -140,6 +140,8 @@ struct StepMap {
   int total;       // steps per tile
   int streamk;     // 0: whole tiles b, b + G, ...; 1: contiguous range [g0, g0 + n_steps)
   long long g0;    // stream-K: first global step of this CTA
+  int glu_rt;      // SwiGLU pairs: gate row tiles (half of row_tiles); 0: off
+  int row_tiles;
   __device__ __forceinline__ void at(int it, int& t, int& k) const {
     if (streamk) {
       const long long g = g0 + it;
@@ -147,7 +149,14 @@ struct StepMap {
       k = static_cast<int>(g - static_cast<long long>(t) * total);
     } else {
       const int lt = it / total;
-      t = static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x);
+      if (glu_rt) {
+        // Local tiles 2 i and 2 i + 1: pair q = b + i G, its gate row tile, then its up row tile.
+        const int q = static_cast<int>(blockIdx.x) + (lt >> 1) * static_cast<int>(gridDim.x);
+        const int tq = q / glu_rt;
+        t = tq * row_tiles + (q - tq * glu_rt) + (lt & 1) * glu_rt;
+      } else {
+        t = static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x);
+      }
       k = it - lt * total;
     }
   }
@@ -158,11 +167,36 @@ struct StepMap {
 struct StepCursor {
   int t, k;
   int row0;  // first weight row (or output feature, dX) of tile t
+  int lt, j, tq;  // SwiGLU pairs: local tile, gate row tile and token tile of its pair
   __device__ __forceinline__ void set(const StepMap& m, int it, int row_tiles) {
     m.at(it, t, k);
     row0 = (t % row_tiles) * kRowsW;
+    if (m.glu_rt) {
+      lt = it / m.total;
+      const int q = static_cast<int>(blockIdx.x) + (lt >> 1) * static_cast<int>(gridDim.x);
+      tq = q / m.glu_rt;
+      j = q - tq * m.glu_rt;
+    }
   }
   __device__ __forceinline__ void advance(const StepMap& m, int row_tiles) {
+    if (m.glu_rt) {  // paired tiles: the next pair is G pairs on, walked without dividing
+      k += 2;
+      if (k >= m.total) {
+        k -= m.total;
+        ++lt;
+        if ((lt & 1) == 0) {
+          j += static_cast<int>(gridDim.x);
+          while (j >= m.glu_rt) {
+            j -= m.glu_rt;
+            ++tq;
+          }
+        }
+        const int rt = j + (lt & 1) * m.glu_rt;
+        t = tq * row_tiles + rt;
+        row0 = rt * kRowsW;
+      }
+      return;
+    }
     k += 2;
     if (k >= m.total) {
       k -= m.total;
@@ -238,7 +272,7 @@ __host__ __device__ inline int first_wave_tiles(int tq, int row_tiles, int G) {
   return static_cast<int>(wave_end - t0 < row_tiles ? wave_end - t0 : row_tiles);
 }
 
-template <bool kTransW, bool kFused>
+template <bool kTransW, bool kFused, bool kGlu = false>
 __global__ void __launch_bounds__(kThreads, 1)
     qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_q,
@@ -288,8 +322,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   StepMap map;
   map.total = total;
   map.streamk = args.streamk;
+  map.row_tiles = row_tiles;
+  map.glu_rt = (kGlu && !args.streamk) ? args.glu_I / kRowsW : 0;
   int n_steps;
-  if (args.streamk) {
+  if (map.glu_rt) {
+    map.g0 = 0;
+    const int pairs = map.glu_rt * (n_tiles / row_tiles);
+    const int my_pairs = static_cast<int>(blockIdx.x) < pairs
+                             ? (pairs - 1 - static_cast<int>(blockIdx.x)) /
+                                       static_cast<int>(gridDim.x) + 1
+                             : 0;
+    n_steps = 2 * my_pairs * total;
+  } else if (args.streamk) {
     const long long T = static_cast<long long>(n_tiles) * total;
     map.g0 = sk_start(blockIdx.x, T, gridDim.x);
     n_steps = static_cast<int>(sk_start(blockIdx.x + 1, T, gridDim.x) - map.g0);
@@ -649,7 +693,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* part = args.partial +
                     ((static_cast<long long>(blockIdx.x) * 2 + slot) * tile_tokens) * kRowsW;
       // (Two separate loops: a branch inside the drain loop measurably slows the bf16 path.)
-      if (whole) {
+      if (kGlu && whole && map.glu_rt && (t % row_tiles) >= map.glu_rt) {
+        // Up tile of a SwiGLU pair: u as usual, and a = silu(g) u from the g this thread wrote
+        // for the same tokens and the gate row (row - I) one tile earlier: bf16 g and u, fp32
+        // math in the packed SwiGLU kernel's order, so a has that kernel's bits.
+        const int I = args.glu_I;
+        const long long ld = args.rows_w;
+        for (int h = 0; h < nh; ++h) {
+          const uint32_t tb = tmem_base + lane_base + static_cast<uint32_t>(ab) * tile_cols +
+                              static_cast<uint32_t>(h) * P.acc_cols;
+          // g of 16 tokens is loaded ahead of their u (16 independent L2 reads in flight).
+          for (int c32 = 0; c32 < bt / 8; c32 += 2) {
+            const int tk0 = tok0 + h * bt + c32 * 8;
+            __nv_bfloat16 gq[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              gq[j] = (c32 * 8 + j < bt && tk0 + j < args.M)
+                          ? args.out[static_cast<long long>(tk0 + j) * ld + row - I]
+                          : __float2bfloat16_rn(0.f);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              if (c32 + q >= bt / 8) break;
+              uint32_t v[8];
+              tmem_ld_32x32b_x8(tb + static_cast<uint32_t>((c32 + q) * 8), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int tok = tk0 + q * 8 + j;
+                if (tok < args.M) {
+                  const __nv_bfloat16 ub = __float2bfloat16_rn(__uint_as_float(v[j]));
+                  args.out[static_cast<long long>(tok) * ld + row] = ub;
+                  const float g = __bfloat162float(gq[q * 8 + j]);
+                  args.glu_out[static_cast<long long>(tok) * I + row - I] =
+                      __float2bfloat16_rn(g * (1.f / (1.f + expf(-g))) * __bfloat162float(ub));
+                }
+              }
+            }
+          }
+        }
+      } else if (whole) {
         for (int h = 0; h < nh; ++h) {
           const uint32_t tb = tmem_base + lane_base + static_cast<uint32_t>(ab) * tile_cols +
                               static_cast<uint32_t>(h) * P.acc_cols;
@@ -979,6 +1061,11 @@ cudaError_t gemm_device_sms(int* sms) {
 
 size_t gemm_smem_bytes(int bt, int nh) { return make_plan(bt, nh).smem; }
 
+bool gemm_glu_ok(int M, int I, int steps_per_tile, int sm_count) {
+  if (I < kRowsW || I % kRowsW) return false;
+  return !gemm_schedule(M, 2 * I, steps_per_tile, sm_count, false).streamk;
+}
+
 GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count, bool fused) {
   GemmSchedule sc;
   const GemmTile tl = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, fused);
@@ -1087,14 +1174,20 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
     sc.grid = sc.n_tiles;
   }
   args.streamk = sc.streamk;
+  if (args.glu_I > 0 && (trans_w || args.fuse || sc.streamk || !args.glu_out ||
+                         args.glu_I % kRowsW || args.rows_w != 2 * args.glu_I))
+    return cudaErrorInvalidValue;
   if (args.fuse && (sc.streamk || !gemm_rank_fusable(args.M, args.rows_w, args.kt + args.n_ext,
                                                       sms, args.rank_cols, args.rank_slot)))
     return cudaErrorInvalidValue;
   const size_t smem = make_plan(args.bt, args.nh, args.fuse ? args.rank_slot : 0u).smem;
   // The fused down-projection is a separate instantiation, so the plain kernel carries none of
   // its code.
+  // The SwiGLU epilogue is a third instance (forward, unfused), so the others carry none of it.
   auto kernel = trans_w ? (args.fuse ? qlora_gemm_kernel<true, true> : qlora_gemm_kernel<true, false>)
-                        : (args.fuse ? qlora_gemm_kernel<false, true> : qlora_gemm_kernel<false, false>);
+                        : (args.fuse ? qlora_gemm_kernel<false, true>
+                                     : (args.glu_I > 0 ? qlora_gemm_kernel<false, false, true>
+                                                       : qlora_gemm_kernel<false, false>));
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;

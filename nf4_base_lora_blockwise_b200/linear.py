@@ -153,6 +153,31 @@ def grouped_forward(X, w: NF4Weight, A, B, group_rows, alpha, H=None, XA=None, w
     return H, (XA if save_xa else None)
 
 
+def gate_up_swiglu_forward(X, w: NF4Weight, A, B, alpha, GU=None, XA=None, act=None, ws=None,
+                           save_xa=True):
+    """Packed gate/up forward with its SwiGLU (qlora_grouped_fwd_swiglu): w NF4 [2I, K] (gate
+    rows, then up rows); A [2r, K]; B [2I, r].  Returns (GU [M, 2I], XA [M, 2r] or None,
+    act [M, I] = silu(g) * u)."""
+    M = X.shape[0]
+    r = A.shape[0] // 2
+    I = w.N // 2
+    _need(X, torch.bfloat16, (M, w.K), "X")
+    _need(A, torch.bfloat16, (2 * r, w.K), "A")
+    _need(B, torch.bfloat16, (w.N, r), "B")
+    if GU is None:
+        GU = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    if XA is None and save_xa:
+        XA = torch.empty((M, 2 * r), dtype=torch.bfloat16, device=X.device)
+    if act is None:
+        act = torch.empty((M, I), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = alloc_grouped_workspace(M, w.N, w.K, r, 2, X.device)
+    abi.qlora_grouped_fwd_swiglu(X.data_ptr(), w.c_struct(), A.data_ptr(), B.data_ptr(), M, r,
+                                 alpha, GU.data_ptr(), _ptr(XA) if save_xa else None,
+                                 act.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
+    return GU, (XA if save_xa else None), act
+
+
 def grouped_backward(dY, X, w: NF4Weight, A, B, XA, group_rows, alpha, need_dx=True, dX=None,
                      dA=None, dB=None, ws=None):
     """Backward of grouped_forward.  Returns (dX or None, dA fp32 [n r, K], dB fp32 [N, r])."""
