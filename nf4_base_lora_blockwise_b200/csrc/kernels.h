@@ -129,7 +129,6 @@ struct GemmArgs {
   // silu(g) * u from the g it wrote one tile earlier (bf16 g and u, fp32 math).
   __nv_bfloat16* glu_out;
   int glu_I;
-  int whole_rounds;  // set by the launcher: whole-tile rounds before the stream-K part
 };
 
 struct GemmMaps {
@@ -147,17 +146,13 @@ struct GemmMaps {
 constexpr int kGemmMaxCtas = 160;
 struct GemmSchedule {
   int n_tiles;
-  int streamk;       // 1: stream-K over the tiles from whole_rounds * grid on
-  int whole_rounds;  // rounds of whole tiles b, b + G, ... before the stream-K part (hybrid)
+  int streamk;
   int grid;
   size_t partial_floats;  // workspace the stream-K partials need
 };
 // fused: the tile a launch with the fused down-projection uses (two halves of 144..240 tokens).
-// hybrid: when the last round of whole tiles would be at most 60 % full, run the full rounds
-// whole and split the remaining tiles stream-K over every CTA (launches that need whole tiles,
-// with SMs left to a side kernel, fused or with the SwiGLU epilogue, pass false).
 GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count,
-                           bool fused = false, bool hybrid = true);
+                           bool fused = false);
 // Whether a launch of this shape can fuse a rank-`rank_cols` down-projection (whole tiles, every
 // token tile's 16-token blocks spread over its first wave of tiles at most 2 per tile).
 bool gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int rank_cols,

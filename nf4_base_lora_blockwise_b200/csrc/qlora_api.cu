@@ -319,7 +319,6 @@ GemmArgs gemm_args(const qlora_nf4_weight* W, int M, int r, const RowGroups& gro
   a.sm_limit = 0;
   a.glu_out = nullptr;
   a.glu_I = 0;
-  a.whole_rounds = 0;
   return a;
 }
 
@@ -1183,7 +1182,7 @@ qlora_status qlora_gemm_plan(int M, int rows_w, int steps_per_tile, int sm_count
   const GemmSchedule sc = gemm_schedule(M, rows_w, steps_per_tile, sm_count);
   *bt = t.bt;
   *nh = t.nh;
-  *streamk = sc.streamk ? (sc.whole_rounds > 0 ? 2 : 1) : 0;
+  *streamk = sc.streamk;
   *grid = sc.grid;
   *partial_bytes = 4 * sc.partial_floats;
   return QLORA_OK;

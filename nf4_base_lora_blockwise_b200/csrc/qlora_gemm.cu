@@ -138,18 +138,15 @@ __host__ __device__ inline Plan make_plan(int bt, int nh, uint32_t rank_slot = 0
 // Where the CTA's it-th reduction step lies: tile t and step k within the tile.
 struct StepMap {
   int total;       // steps per tile
-  int streamk;     // 0: whole tiles b, b + G, ...; 1: contiguous range [g0, ...) (after wr
-                   // rounds of whole tiles b, b + G, ... when wr > 0)
-  long long g0;    // stream-K: first step of this CTA in the stream-K part's step space
-  int wr;          // whole-tile rounds before the stream-K part
+  int streamk;     // 0: whole tiles b, b + G, ...; 1: contiguous range [g0, g0 + n_steps)
+  long long g0;    // stream-K: first global step of this CTA
   int glu_rt;      // SwiGLU pairs: gate row tiles (half of row_tiles); 0: off
   int row_tiles;
   __device__ __forceinline__ void at(int it, int& t, int& k) const {
-    if (streamk && it >= wr * total) {
-      const long long g = g0 + (it - wr * total);
-      const int ts = static_cast<int>(g / total);
-      t = wr * static_cast<int>(gridDim.x) + ts;
-      k = static_cast<int>(g - static_cast<long long>(ts) * total);
+    if (streamk) {
+      const long long g = g0 + it;
+      t = static_cast<int>(g / total);
+      k = static_cast<int>(g - static_cast<long long>(t) * total);
     } else {
       const int lt = it / total;
       if (glu_rt) {
@@ -171,9 +168,7 @@ struct StepCursor {
   int t, k;
   int row0;  // first weight row (or output feature, dX) of tile t
   int lt, j, tq;  // SwiGLU pairs: local tile, gate row tile and token tile of its pair
-  int it;
-  __device__ __forceinline__ void set(const StepMap& m, int it_, int row_tiles) {
-    it = it_;
+  __device__ __forceinline__ void set(const StepMap& m, int it, int row_tiles) {
     m.at(it, t, k);
     row0 = (t % row_tiles) * kRowsW;
     if (m.glu_rt) {
@@ -184,11 +179,6 @@ struct StepCursor {
     }
   }
   __device__ __forceinline__ void advance(const StepMap& m, int row_tiles) {
-    it += 2;
-    if (m.streamk && m.wr > 0 && it >= m.wr * m.total && it - 2 < m.wr * m.total + m.total) {
-      set(m, it, row_tiles);  // into (or just past the start of) the stream-K part: once a CTA
-      return;
-    }
     if (m.glu_rt) {  // paired tiles: the next pair is G pairs on, walked without dividing
       k += 2;
       if (k >= m.total) {
@@ -210,7 +200,7 @@ struct StepCursor {
     k += 2;
     if (k >= m.total) {
       k -= m.total;
-      t += (m.streamk && it >= m.wr * m.total) ? 1 : static_cast<int>(gridDim.x);
+      t += m.streamk ? 1 : static_cast<int>(gridDim.x);
       row0 = (t % row_tiles) * kRowsW;
     }
   }
@@ -331,8 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // This CTA's reduction steps: whole tiles, or one contiguous stream-K range.
   StepMap map;
   map.total = total;
-  map.streamk = kGlu ? 0 : args.streamk;  // the SwiGLU instance runs whole tiles only
-  map.wr = map.streamk ? args.whole_rounds : 0;
+  map.streamk = args.streamk;
   map.row_tiles = row_tiles;
   map.glu_rt = (kGlu && !args.streamk) ? args.glu_I / kRowsW : 0;
   int n_steps;
@@ -344,11 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        static_cast<int>(gridDim.x) + 1
                              : 0;
     n_steps = 2 * my_pairs * total;
-  } else if (map.streamk) {
-    const long long T =
-        static_cast<long long>(n_tiles - map.wr * static_cast<int>(gridDim.x)) * total;
+  } else if (args.streamk) {
+    const long long T = static_cast<long long>(n_tiles) * total;
     map.g0 = sk_start(blockIdx.x, T, gridDim.x);
-    n_steps = map.wr * total + static_cast<int>(sk_start(blockIdx.x + 1, T, gridDim.x) - map.g0);
+    n_steps = static_cast<int>(sk_start(blockIdx.x + 1, T, gridDim.x) - map.g0);
   } else {
     map.g0 = 0;
     const int my_tiles = static_cast<int>(blockIdx.x) < n_tiles
@@ -688,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const bool whole = k0 == 0 && len == total;
-      const int slot = it == map.wr * total ? 0 : 1;  // head of the stream-K range, or its tail
+      const int slot = it == 0 ? 0 : 1;
       it += len;
       const int ab = P.nacc == 2 ? (seg & 1) : 0;
       const int use = P.nacc == 2 ? (seg >> 1) : seg;
@@ -932,14 +920,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(256) qlora_gemm_finalize(const float* __restrict__ partial,
                                                            int M, int rows_w, int tile_tokens,
                                                            int total, long long T, int G,
-                                                           int t_off,
                                                            __nv_bfloat16* __restrict__ out) {
   pdl_wait();  // the GEMM's partial sums are complete
   pdl_trigger();
   const int row_tiles = (rows_w + kRowsW - 1) / kRowsW;
-  // Tile t_off + blockIdx.y; the stream-K step space (T steps) starts at tile t_off.
-  const int t = t_off + static_cast<int>(blockIdx.y);
-  const long long gs = static_cast<long long>(blockIdx.y) * total;
+  const int t = blockIdx.y;
+  const long long gs = static_cast<long long>(t) * total;
   // CTA holding global step g: the largest b with floor(b T / G) <= g.
   auto owner = [&](long long g) { return static_cast<int>(((g + 1) * G - 1) / T); };
   const int b_first = owner(gs);
@@ -1077,28 +1063,16 @@ size_t gemm_smem_bytes(int bt, int nh) { return make_plan(bt, nh).smem; }
 
 bool gemm_glu_ok(int M, int I, int steps_per_tile, int sm_count) {
   if (I < kRowsW || I % kRowsW) return false;
-  // Only where a plain launch runs whole tiles too, so both give the same bits.
-  return !gemm_schedule(M, 2 * I, steps_per_tile, sm_count).streamk;
+  return !gemm_schedule(M, 2 * I, steps_per_tile, sm_count, false).streamk;
 }
 
-GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count, bool fused,
-                           bool hybrid) {
+GemmSchedule gemm_schedule(int M, int rows_w, int steps_per_tile, int sm_count, bool fused) {
   GemmSchedule sc;
   const GemmTile tl = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, fused);
   const int tile_tokens = tl.bt * tl.nh;
   sc.n_tiles = ((rows_w + kRowsW - 1) / kRowsW) * ((M + tile_tokens - 1) / tile_tokens);
   const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
-  sc.whole_rounds = 0;
-  const int rem = sc.n_tiles % G;
-  if (sc.n_tiles >= G && hybrid && !fused && rem > 0 && rem * 10 <= G * 6 &&
-      static_cast<long long>(rem) * steps_per_tile >= G) {
-    // The last round would leave most CTAs idle: run the full rounds whole, then cut the
-    // remaining tiles' steps evenly over every CTA (each CTA at least one step, as the
-    // finalize's owner arithmetic assumes).
-    sc.streamk = 1;
-    sc.whole_rounds = sc.n_tiles / G;
-    sc.grid = G;
-  } else if (sc.n_tiles >= G) {
+  if (sc.n_tiles >= G) {
     sc.streamk = 0;
     sc.grid = G;
   } else {
@@ -1123,7 +1097,7 @@ bool gemm_rank_fusable(int M, int rows_w, int steps_per_tile, int sm_count, int 
   // Worth it while the fused tile costs the GEMM at most 4 % over its own choice of tile (the
   // separate down-projection it replaces streams all of the activations once more).
   const GemmTile own = gemm_pick_tile(M, rows_w, steps_per_tile, sm_count, false);
-  const GemmSchedule own_sc = gemm_schedule(M, rows_w, steps_per_tile, sm_count, false, false);
+  const GemmSchedule own_sc = gemm_schedule(M, rows_w, steps_per_tile, sm_count, false);
   if (own_sc.streamk) return false;
   const int G = sc.grid;
   if (whole_tile_cycles(M, rows_w, steps_per_tile, G, tl.bt, tl.nh) >
@@ -1147,8 +1121,6 @@ int gemm_side_sms(int M, int rows_w, int steps_per_tile, int sm_count, double si
                   bool force, double* us) {
   const int G = sm_count < kGemmMaxCtas ? sm_count : kGemmMaxCtas;
   *us = 0.0;
-  // Only where the GEMM alone runs whole tiles (not stream-K, nor the hybrid), so the outputs
-  // have the same bits with and without the side kernel.
   if (M <= 256 || G < 64 || side_bytes <= 0.0 ||
       gemm_schedule(M, rows_w, steps_per_tile, G).streamk)
     return 0;
@@ -1158,7 +1130,7 @@ int gemm_side_sms(int M, int rows_w, int steps_per_tile, int sm_count, double si
   double best_us = 0.0;
   for (int spare = 2; spare <= kSideMaxSms; spare += 2) {
     const int g = G - spare;
-    if (gemm_schedule(M, rows_w, steps_per_tile, g, false, false).streamk) break;
+    if (gemm_schedule(M, rows_w, steps_per_tile, g).streamk) break;
     const GemmTile t = gemm_pick_tile(M, rows_w, steps_per_tile, g);
     const double gemm = whole_tile_cycles(M, rows_w, steps_per_tile, g, t.bt, t.nh) / kClockMhz;
     const double side = side_bytes / (spare * kSideBytesPerUsPerSm);
@@ -1179,10 +1151,7 @@ int gemm_side_sms(int M, int rows_w, int steps_per_tile, int sm_count, double si
 size_t gemm_rank_flag_bytes(int M) { return 4 * (static_cast<size_t>(M) / 128 + 2); }
 
 size_t gemm_partial_bytes_bound(int M, int rows_w, int steps_per_tile) {
-  // Pure stream-K shapes only: a hybrid launch uses the partial slots when the workspace has
-  // them (for instance from the other direction of the same layer) and runs whole tiles
-  // otherwise, so the workspace size does not grow for shapes that run whole tiles.
-  return 4 * gemm_schedule(M, rows_w, steps_per_tile, kGemmMaxCtas, false, false).partial_floats;
+  return 4 * gemm_schedule(M, rows_w, steps_per_tile, kGemmMaxCtas).partial_floats;
 }
 
 cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
@@ -1198,19 +1167,13 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
   // The caller's tile (TMA boxes, smem plan) must be the one the schedule assumes.
   const GemmTile tl = gemm_pick_tile(args.M, args.rows_w, args.kt + args.n_ext, sms, args.fuse);
   if (tl.bt != args.bt || tl.nh != args.nh) return cudaErrorInvalidValue;
-  // Whole tiles for launches that leave SMs to a side kernel, fuse the down-projection or add
-  // the SwiGLU epilogue; otherwise a part-full last round goes stream-K (hybrid).
-  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, sms, args.fuse,
-                                  args.sm_limit == 0 && args.glu_I == 0 && !args.fuse);
+  GemmSchedule sc = gemm_schedule(args.M, args.rows_w, args.kt + args.n_ext, sms, args.fuse);
   if (sc.streamk && (!args.partial || sc.partial_floats > partial_floats_avail)) {
-    // No room for the partial sums: whole tiles (one CTA per tile when there are fewer tiles
-    // than SMs).
+    // No room for the partial sums: whole tiles, one CTA per tile.
     sc.streamk = 0;
-    if (sc.whole_rounds == 0) sc.grid = sc.n_tiles;
-    sc.whole_rounds = 0;
+    sc.grid = sc.n_tiles;
   }
   args.streamk = sc.streamk;
-  args.whole_rounds = sc.whole_rounds;
   if (args.glu_I > 0 && (trans_w || args.fuse || sc.streamk || !args.glu_out ||
                          args.glu_I % kRowsW || args.rows_w != 2 * args.glu_I))
     return cudaErrorInvalidValue;
@@ -1236,13 +1199,12 @@ cudaError_t launch_qlora_gemm(bool trans_w, const GemmMaps& maps, GemmArgs args,
   *launched = 1;
   if (!sc.streamk) return e;
   const int total = args.kt + args.n_ext;
-  const int t_off = sc.whole_rounds * sc.grid;  // tiles the whole rounds wrote
-  const long long T = static_cast<long long>(sc.n_tiles - t_off) * total;
+  const long long T = static_cast<long long>(sc.n_tiles) * total;
   const int tile_elems = args.bt * args.nh * kRowsW;
-  const dim3 fgrid((tile_elems / 4 + 255) / 256, sc.n_tiles - t_off);
+  const dim3 fgrid((tile_elems / 4 + 255) / 256, sc.n_tiles);
   e = launch_pdl(qlora_gemm_finalize, fgrid, dim3(256), 0, stream, 1,
                  static_cast<const float*>(args.partial), args.M, args.rows_w,
-                 args.bt * args.nh, total, T, sc.grid, t_off, args.out);
+                 args.bt * args.nh, total, T, sc.grid, args.out);
   if (e == cudaSuccess) *launched = 2;
   return e;
 }

@@ -7,9 +7,8 @@ just written.  Checked here:
 * GU, the saved XA and act have the bits of qlora_grouped_fwd followed by
   qlora_swiglu_packed_fwd (the path the call falls back to), on whole-tile shapes with ragged
   token tails, at the MLP workload's full size, and on a double-quantised weight;
-* where a plain launch of the layer runs whole tiles, the call takes one launch fewer than that
-  sequence (no SwiGLU launch); shapes the epilogue does not serve (stream-K, the hybrid
-  schedule, few tokens) fall back to it;
+* the fused shapes take one launch fewer than that sequence (no SwiGLU launch), and shapes the
+  epilogue cannot serve (stream-K, few tokens) fall back to it;
 * act meets the oracle's SwiGLU on the GPU's own g and u (max|err| / max|ref| <= 1e-2), and the
   packed layer's GU meets the oracle's forward per adapter (the parity bar, 2e-2).
 """
@@ -50,13 +49,6 @@ def _launches(fn):
     return out, abi.qlora_launch_counter() - n0
 
 
-def _whole(M, K, I, r):
-    """Whether a plain forward of the packed layer runs whole tiles on this device."""
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    steps = K // 64 + ((r + 15) // 16 * 16 + 63) // 64
-    return M > 32 and abi.qlora_gemm_plan(M, 2 * I, steps, sms)["streamk"] == 0
-
-
 def _both(M, K, I, r, seed, dq=False):
     X, w, A, B, W0 = _inputs(M, K, I, r, seed, dq)
     alpha = 2.0 * r
@@ -72,18 +64,14 @@ def _both(M, K, I, r, seed, dq=False):
     return ref, n_ref, n_got, (X, w, A, B, W0, alpha)
 
 
-@pytest.mark.parametrize("M,K,I,r,dq,fused", [
-    (4096, 1024, 2048, 16, False, True),   # whole tiles (288 tiles of 480 tokens on 148 SMs)
-    (3900, 1024, 3072, 16, False, True),   # ragged last token tile (448-token tiles)
-    (4000, 1536, 2048, 32, True, True),    # double-quantised absmax, r = 32
-    (2048, 1024, 4096, 16, False, False),  # the hybrid schedule alone: falls back, same bits
+@pytest.mark.parametrize("M,K,I,r,dq", [
+    (2048, 1024, 4096, 16, False),   # whole tiles, 480-token tiles
+    (1900, 512, 4096, 16, False),    # ragged last token tile
+    (2304, 768, 3072, 32, True),     # double-quantised absmax, r = 32
 ])
-def test_fused_equals_layer_then_swiglu(M, K, I, r, dq, fused):
-    whole = _whole(M, K, I, r)
+def test_fused_equals_layer_then_swiglu(M, K, I, r, dq):
     _, n_ref, n_got, _ = _both(M, K, I, r, seed=M + I, dq=dq)
-    assert n_got == n_ref - (1 if whole else 0), "the SwiGLU goes in the epilogue on whole tiles"
-    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
-        assert whole == fused, "the shape exercises the path it is meant to on a 148-SM B200"
+    assert n_got == n_ref - 1, "the SwiGLU is in the GEMM epilogue, not a launch of its own"
 
 
 @pytest.mark.parametrize("M,K,I,r", [
@@ -96,8 +84,7 @@ def test_fallback_equals_layer_then_swiglu(M, K, I, r):
 
 
 def test_fused_meets_the_oracle():
-    M, K, I, r = 4096, 1024, 2048, 16
-    assert _whole(M, K, I, r) or torch.cuda.get_device_properties(0).multi_processor_count != 148
+    M, K, I, r = 2048, 512, 2048 + 2048, 16
     (GU, XA, act), _, n_got, (X, w, A, B, W0, alpha) = _both(M, K, I, r, seed=3)
     rows = np.concatenate([np.arange(0, M, 61), [M - 1]])
     g, u = qlora.split_cols(parity.f32(GU)[rows], [I, I])
@@ -117,6 +104,5 @@ def test_full_size_mlp_gate_up():
     """The MLP workload's packed gate/up layer (4096 -> 2 x 14336, 8192 tokens, r = 16)."""
     w = synth.workload("mlp_8b")
     gate = w.linears[0]
-    whole = _whole(w.M, gate.K, gate.N, gate.r)
     _, n_ref, n_got, _ = _both(w.M, gate.K, gate.N, gate.r, seed=11)
-    assert n_got == n_ref - (1 if whole else 0)
+    assert n_got == n_ref - 1

@@ -72,63 +72,6 @@ def test_stream_k_partition():
             assert ks == total
 
 
-def test_hybrid_partition():
-    """Whole rounds, then stream-K over the remaining tiles (the kernel's hybrid schedule):
-    every (tile, step) is computed exactly once; the whole rounds and whole stream-K segments
-    are written directly; the finalize, walking the stream-K tiles from tile t_off = wr G,
-    finds every cut tile's slots in step order.  (The schedule takes the hybrid only when the
-    stream-K part has at least one step per CTA.)"""
-    rng = random.Random(5)
-    for _ in range(600):
-        G = rng.choice([132, 148, 160])
-        wr = rng.randint(1, 4)
-        rem = rng.randint(1, G * 6 // 10)
-        n_tiles = wr * G + rem
-        total = rng.randint(max(2, -(-G // rem)), 120 + G // rem)  # every CTA >= 1 step
-        T = rem * total
-        assert T >= G
-        t_off = wr * G
-        covered, written, whole = {}, {}, set()
-        for b in range(G):
-            g0 = _sk_start(b, T, G)
-            n = wr * total + _sk_start(b + 1, T, G) - g0
-            it = 0
-            while it < n:
-                if it < wr * total:
-                    lt = it // total
-                    t, k0, ln = b + lt * G, 0, total
-                else:
-                    ts, k0 = divmod(g0 + it - wr * total, total)
-                    t = t_off + ts
-                    ln = min(total - k0, n - it)
-                for k in range(k0, k0 + ln):
-                    assert (t, k) not in covered
-                    covered[(t, k)] = b
-                if k0 == 0 and ln == total:
-                    whole.add(t)
-                else:
-                    slot = 0 if it == wr * total else 1
-                    assert (b, slot) not in written
-                    written[(b, slot)] = (t, k0, ln)
-                it += ln
-        assert len(covered) == n_tiles * total
-        assert all(t in whole for t in range(t_off))
-        owner = lambda g: ((g + 1) * G - 1) // T  # noqa: E731
-        for y in range(rem):
-            t, gs = t_off + y, y * total
-            bf, bl = owner(gs), owner(gs + total - 1)
-            if bf == bl:
-                assert t in whole
-                continue
-            ks = 0
-            for b in range(bf, bl + 1):
-                slot = 0 if _sk_start(b, T, G) >= gs else 1
-                tt, k0, ln = written[(b, slot)]
-                assert (tt, k0) == (t, ks)
-                ks += ln
-            assert ks == total
-
-
 def _gemv_stages(u0, u1, KB, blk=4):
     """The kernel's stage walk: (row tile, first block, blocks, segment, ends segment)."""
     out, u, seg = [], u0, 0
@@ -179,35 +122,26 @@ def test_few_token_partition():
 
 def test_step_cursor_matches_division():
     """The dequant groups advance (tile, step) by two steps without dividing; every tile has
-    at least two steps, so one advance wraps at most once.  With whole rounds before a
-    stream-K part (hybrid), the cursor re-derives its position by division while its step lies
-    in the first stream-K tile's span, and walks tiles one by one after that."""
+    at least two steps, so one advance wraps at most once."""
     rng = random.Random(11)
     for _ in range(3000):
         total, streamk = rng.randint(2, 70), rng.random() < 0.5
-        wr = rng.choice([0, 0, 1, 2, 5]) if streamk else 0
         G, g0 = rng.randint(1, 148), rng.randint(0, 500)
         bx = rng.randrange(G)
 
         def at(it):
-            if streamk and it >= wr * total:
-                ts, k = divmod(g0 + it - wr * total, total)
-                return wr * G + ts, k
+            if streamk:
+                return divmod(g0 + it, total)
             lt = it // total
             return bx + lt * G, it - lt * total
         for g in (0, 1):
             t, k = at(g)
-            it = g
-            for _ in range(90):
+            for it in range(g, g + 120, 2):
                 assert (t, k) == at(it)
-                it += 2
-                if streamk and wr > 0 and wr * total <= it < wr * total + total + 2:
-                    t, k = at(it)
-                    continue
                 k += 2
                 if k >= total:
                     k -= total
-                    t += 1 if (streamk and it >= wr * total) else G
+                    t += 1 if streamk else G
 
 
 def test_gemm_plan_properties():
@@ -242,29 +176,20 @@ def test_gemm_plan_properties():
             tiles = ((rows + 127) // 128) * ((M + tt - 1) // tt)
             wide = ((rows + 127) // 128) * ((M + (512 if M > 256 else tt) - 1)
                                            // (512 if M > 256 else tt))
-            if wide < G:
-                assert p["streamk"] == 1
+            assert p["streamk"] == (1 if wide < G else 0)
+            if p["streamk"]:
                 assert p["bt"] == (256 if M > 256 else p["bt"])
                 assert p["grid"] == min(tiles * steps, G)
                 assert p["partial_bytes"] == p["grid"] * 2 * tt * 128 * 4
             else:
-                # Whole tiles, or whole rounds and a stream-K remainder when the last round
-                # would be at most 60 % full (hybrid, streamk = 2).
-                rem = tiles % G
-                hybrid = rem > 0 and rem * 10 <= G * 6 and rem * steps >= G
-                assert tiles >= G and p["grid"] == G
-                assert p["streamk"] == (2 if hybrid else 0)
-                assert p["partial_bytes"] == (G * 2 * tt * 128 * 4 if hybrid else 0)
+                assert p["grid"] == G and tiles >= G and p["partial_bytes"] == 0
         if M > 32:  # the few-token forward has its own slots; larger M uses these GEMMs only
             need = abi.qlora_workspace_bytes(M, N, K, r)
             for trans in (False, True):
                 rows, steps = (K, N // 64) if trans else (N, K // 64)
                 steps += ((r + 15) // 16 * 16 + 63) // 64
                 for s2 in (100, 132, 148, 160):
-                    q = abi.qlora_gemm_plan(M, rows, steps, s2)
-                    # (a hybrid plan runs whole tiles when the workspace lacks its slots)
-                    if q["streamk"] == 1:
-                        assert q["partial_bytes"] <= need
+                    assert abi.qlora_gemm_plan(M, rows, steps, s2)["partial_bytes"] <= need
 
 
 def test_gemm_plan_headline_tile():
@@ -387,13 +312,11 @@ def test_backward_side_sms():
             assert s1 == 0
         steps = N // 64 + ((R + 15) // 16 * 16 + 63) // 64
         full = abi.qlora_gemm_plan(M, K, steps, sms)
-        if M <= 256 or full["streamk"]:  # stream-K or hybrid alone: no side kernel
+        if M <= 256 or full["streamk"]:
             assert s == 0
         if s == 0:
             continue
         seen += 1
-        # (a launch that leaves SMs to the side kernel runs whole tiles even where a plain
-        # launch on that many SMs would take the hybrid schedule)
         part = abi.qlora_gemm_plan(M, K, steps, sms - s)
-        assert part["streamk"] in (0, 2) and part["grid"] == sms - s
+        assert part["streamk"] == 0 and part["grid"] == sms - s
     assert seen > 20
