@@ -144,6 +144,63 @@ def test_step_cursor_matches_division():
                     t += 1 if streamk else G
 
 
+def test_swiglu_pair_schedule():
+    """The SwiGLU epilogue's tile order (qlora_gemm_kernel's paired schedule): CTA b takes
+    pairs q = b, b + G, ... of (gate row tile j, token tile tq), each as the gate tile
+    tq * row_tiles + j and then the up tile tq * row_tiles + j + half.  Checked: every tile of
+    every token tile is computed exactly once, each up tile right after its own gate tile by the
+    same CTA, and the dequant cursor's division-free walk (two steps at a time, j advanced by G
+    and wrapped into tq) lands where the division formula does."""
+    rng = random.Random(23)
+    for _ in range(400):
+        half = rng.randint(1, 120)        # gate row tiles (I / 128)
+        row_tiles = 2 * half
+        token_tiles = rng.randint(1, 12)
+        G = rng.choice([132, 148, 160])
+        total = rng.randint(2, 70)
+        pairs = half * token_tiles
+
+        def at(b, it):
+            lt, k = divmod(it, total)
+            q = b + (lt >> 1) * G
+            tq, j = divmod(q, half)
+            return tq * row_tiles + j + (lt & 1) * half, k
+        seen = {}
+        for b in range(G):
+            my_pairs = (pairs - 1 - b) // G + 1 if b < pairs else 0
+            n = 2 * my_pairs * total
+            order = []
+            for it in range(0, n, total):
+                t, k = at(b, it)
+                assert k == 0
+                assert t not in seen
+                seen[t] = b
+                order.append(t)
+            for i in range(0, len(order), 2):
+                gate, up = order[i], order[i + 1]
+                assert up == gate + half and (gate % row_tiles) < half
+            for g in (0, 1):  # the cursor: set once, then advanced without dividing
+                if n <= g:
+                    continue
+                t, k = at(b, g)
+                lt = g // total
+                q = b + (lt >> 1) * G
+                tq, j = divmod(q, half)
+                for it in range(g, n, 2):
+                    assert (t, k) == at(b, it)
+                    k += 2
+                    if k >= total:
+                        k -= total
+                        lt += 1
+                        if lt % 2 == 0:
+                            j += G
+                            while j >= half:
+                                j -= half
+                                tq += 1
+                        t = tq * row_tiles + j + (lt & 1) * half
+        assert len(seen) == row_tiles * token_tiles
+
+
 def test_gemm_plan_properties():
     """The dequant GEMM's launch plan (qlora_gemm_plan, host only) on random problems:
     * token tiles: one half of M rounded up to 16 for M <= 256, else two halves of a multiple
